@@ -1,0 +1,427 @@
+"""CPU oracle for the Pyramid Sparse Attention (PSA) forward path.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
+the ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import
+this module.  The product path (``video_transformers_b200``) never calls it,
+and this module imports nothing from the product path: the two share no
+kernels, headers, helpers, tables or constants.
+
+Everything here is plain numpy in float64.  Inputs arrive as whatever the
+CUDA path was given (fp32 or bf16 tensors), converted exactly to float64.
+The code follows the definitions as written, with no blocking, fusion or
+reordering beyond what the definition states, so it can be read against the
+pages line by line.
+
+Pages cited (title, then section):
+  [skill]    "psa-pyramid-sparse-attention" skill page: "Core Technique",
+             "Implementation" (pooled KV cache creation).
+  [article]  "PSA: Pyramid Sparse Attention for Efficient Video Understanding
+             and Generation", summary article: "Problem", "Method", "Results".
+  [news]     "[Paper] PSA: Pyramid Sparse Attention ..." news review:
+             "Methodology" items 2 and 4.
+  [abstract] the arXiv abstract of the same paper.
+
+Readings taken where the pages are silent (each is also listed with its
+reason in the design notes):
+  R1  consistency scale = +ln(2^l) logit bias for a level-l pooled token
+      (equivalent to repeating the pooled token 2^l times, which is how
+      [news] Methodology 4 describes pooled KV being brought back to size).
+  R2  sm_scale defaults to 1/sqrt(d) ([news] Methodology 4 combines the
+      query with the selected KV by ordinary scaled dot-product attention).
+  R3  causal visibility of a pooled token: visible to query i iff the last
+      token it averages is <= i.
+  R4  a query row with no visible key gets o = 0, lse = -inf.
+  R5  sampling score: 8 evenly strided rows per query block
+      (row = I*block + s*block/8), softmax over all valid keys at full
+      resolution (keys <= i when causal), block-summed, averaged over the
+      valid samples.
+  R6  antidiagonal score with stride S: per S-group, the mean logit along
+      the antidiagonal of the S x S sub-tile; softmax over key groups
+      (c <= a when causal); block-summed; averaged over the query groups of
+      the block.
+  R7  level assignment: rank blocks by mass (descending, ties to the lower
+      index), exclusive prefix C_J, level = #{t_l <= C_J}, SKIP when that
+      count reaches L.
+  R8  forced rules, applied in this order after R7: blocks holding any token
+      below n_dense_prefix (as query or key block) -> level 0; cosine gate
+      (level >= 1 and blockcos < cos_min -> level 0); causal: J > I -> SKIP,
+      J == I -> level 0.
+  R9  block cosine = mean pairwise cosine over i != j of the block's valid
+      keys; a zero key has unit vector 0; a one-key block scores 1.
+
+Pins: every function here is checked by ``tests/test_oracle_pins.py``
+against closed forms, invariants, brute force or an independent library
+routine; see that file's header for which pin covers which function.
+"""
+from __future__ import annotations
+
+import math
+from typing import Iterable, List, Optional, Sequence, Tuple
+
+import numpy as np
+
+SKIP = 0xFF
+LN2 = math.log(2.0)
+
+
+def _f64(x) -> np.ndarray:
+    """Exact conversion of a torch tensor (fp32/bf16) or array to float64."""
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            return x.detach().to("cpu", torch.float64).numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.asarray(x, dtype=np.float64)
+
+
+# ======================================================================================
+# Stage 1: KV pyramid
+# ======================================================================================
+
+def pool_level(x, level: int) -> np.ndarray:
+    """Level ``level`` of the KV pyramid: every run of g = 2^level consecutive
+    tokens replaced by its mean ([skill] Core Technique, level l holds the
+    KV pooled by 2^l; [skill] Implementation, average pooling over tokens by
+    a factor 2**level taken from the full-resolution cache; [article] Method,
+    the pyramid comes from repeated one-dimensional mean pooling).
+
+    x: [B, H, N, d] -> [B, H, N / g, d].  The direct mean equals the
+    progressive (pairwise) pooling in exact arithmetic.  N must be a
+    multiple of g, so groups never straddle the end of the sequence."""
+    x = _f64(x)
+    B, H, N, d = x.shape
+    g = 1 << level
+    if N % g:
+        raise ValueError("sequence length must be a multiple of the pooling factor")
+    return x.reshape(B, H, N // g, g, d).mean(axis=3)
+
+
+def build_pyramid(k, v, levels: int) -> Tuple[List[np.ndarray], List[np.ndarray]]:
+    """Levels 0..L-1 of K and V; level 0 is the input itself ([skill]
+    Core Technique, level 0 is the unpooled KV)."""
+    kp = [_f64(k)] + [pool_level(k, l) for l in range(1, levels)]
+    vp = [_f64(v)] + [pool_level(v, l) for l in range(1, levels)]
+    return kp, vp
+
+
+def block_cosine(k, block: int) -> np.ndarray:
+    """Intra-block similarity statistic used by the pooling constraint
+    ([article] Method, the understanding-task scorer checks similarity inside
+    each block; [article] Results, a cosine-similarity condition decides
+    whether a block may be pooled).  Reading R9: the
+    mean over ordered pairs i != j of cos(k_i, k_j) over the valid keys of
+    block J, brute force over all pairs.
+
+    k: [B, H, N, d] -> [B, H, nKB]."""
+    k = _f64(k)
+    B, H, N, d = k.shape
+    nkb = -(-N // block)
+    out = np.empty((B, H, nkb))
+    for b in range(B):
+        for h in range(H):
+            for J in range(nkb):
+                keys = k[b, h, J * block:min((J + 1) * block, N)]
+                n = keys.shape[0]
+                if n == 1:
+                    out[b, h, J] = 1.0
+                    continue
+                norms = np.sqrt((keys * keys).sum(axis=1))
+                unit = np.where(norms[:, None] > 0, keys / np.where(norms > 0, norms, 1.0)[:, None], 0.0)
+                total = 0.0
+                for i in range(n):
+                    cos_i = unit @ unit[i]
+                    total += cos_i.sum() - cos_i[i]
+                out[b, h, J] = total / (n * (n - 1))
+    return out
+
+
+# ======================================================================================
+# Stage 2: multi-level mask
+# ======================================================================================
+
+def _softmax_rows(z: np.ndarray) -> np.ndarray:
+    """Row softmax with the max subtracted; rows that are all -inf give 0."""
+    m = z.max(axis=1, keepdims=True)
+    m = np.where(np.isfinite(m), m, 0.0)
+    e = np.exp(z - m)
+    s = e.sum(axis=1, keepdims=True)
+    return np.where(s > 0, e / np.where(s > 0, s, 1.0), 0.0)
+
+
+def _block_sum(p: np.ndarray, width: int, nblocks: int) -> np.ndarray:
+    """Sum the columns of p in consecutive runs of ``width`` (last run ragged)."""
+    rows, cols = p.shape
+    pad = nblocks * width - cols
+    if pad:
+        p = np.concatenate([p, np.zeros((rows, pad))], axis=1)
+    return p.reshape(rows, nblocks, width).sum(axis=2)
+
+
+def sampling_rows(I: int, block: int, N: int, n_samples: int = 8) -> List[int]:
+    """Reading R5: the sampled query rows of block I."""
+    step = block // n_samples
+    return [I * block + s * step for s in range(n_samples) if I * block + s * step < N]
+
+
+def sampling_mass(q, k, block: int, sm_scale: float, causal: bool = False, n_samples: int = 8,
+                  rows: Optional[Iterable[Tuple[int, int, int]]] = None) -> np.ndarray:
+    """Block importance by sampling ([article] Method, the generation-task
+    scorer samples queries).  Reading R5.
+
+    q: [B, Hq, N, d], k: [B, Hkv, N, d].  Returns mass [B, Hq, nQB, nKB];
+    when ``rows`` lists (b, h, I) triples only those rows are filled (the
+    rest stay NaN)."""
+    q = _f64(q)
+    k = _f64(k)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    grp = Hq // Hkv
+    nb = -(-N // block)
+    mass = np.full((B, Hq, nb, nb), np.nan)
+    if rows is None:
+        rows = [(b, h, I) for b in range(B) for h in range(Hq) for I in range(nb)]
+    for b, h, I in rows:
+        keys = k[b, h // grp]
+        r = sampling_rows(I, block, N, n_samples)
+        z = sm_scale * (q[b, h, r] @ keys.T)                       # [ns, N]
+        if causal:
+            j = np.arange(N)
+            z = np.where(j[None, :] <= np.asarray(r)[:, None], z, -np.inf)
+        p = _softmax_rows(z)
+        mass[b, h, I] = _block_sum(p, block, nb).mean(axis=0)
+    return mass
+
+
+def antidiag_logits(qh: np.ndarray, kh: np.ndarray, stride: int, sm_scale: float) -> np.ndarray:
+    """Reading R6 of the understanding-task score ([article] Method, scores
+    come from antidiagonals): for query group a and key group c,
+    A[a, c] = (sm_scale / S) * sum_{s<S} q[a*S + S-1-s] . k[c*S + s].
+
+    qh, kh: [N, d] (one head); returns [N/S, N/S]."""
+    N, d = qh.shape
+    S = stride
+    G = N // S
+    A = np.zeros((G, G))
+    for s in range(S):
+        A += qh[np.arange(G) * S + (S - 1 - s)] @ kh[np.arange(G) * S + s].T
+    return (sm_scale / S) * A
+
+
+def antidiag_mass(q, k, block: int, stride: int, sm_scale: float, causal: bool,
+                  rows: Optional[Iterable[Tuple[int, int, int]]] = None) -> np.ndarray:
+    """Block importance from antidiagonal scores (reading R6): group
+    probabilities P[a, :] = softmax_c A[a, c] (c <= a when causal), then
+    mass[I, J] = mean over the query groups a of block I of sum over the key
+    groups c of block J of P[a, c]."""
+    q = _f64(q)
+    k = _f64(k)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    grp = Hq // Hkv
+    S = stride
+    if N % S:
+        raise ValueError("sequence length must be a multiple of the stride")
+    G = N // S
+    gpb = block // S
+    nb = -(-N // block)
+    mass = np.full((B, Hq, nb, nb), np.nan)
+    want = None if rows is None else {}
+    if rows is not None:
+        for b, h, I in rows:
+            want.setdefault((b, h), []).append(I)
+    for b in range(B):
+        for h in range(Hq):
+            if want is not None and (b, h) not in want:
+                continue
+            A = antidiag_logits(q[b, h], k[b, h // grp], S, sm_scale)
+            if causal:
+                a = np.arange(G)
+                A = np.where(a[None, :] <= a[:, None], A, -np.inf)
+            P = _softmax_rows(A)
+            per_group = _block_sum(P, gpb, nb)                       # [G, nb]
+            Is = range(nb) if want is None else want[(b, h)]
+            for I in Is:
+                mass[b, h, I] = per_group[I * gpb:min((I + 1) * gpb, G)].mean(axis=0)
+    return mass
+
+
+def assign_levels_row(mass_row: Sequence[float], thresholds: Sequence[float], levels: int) -> np.ndarray:
+    """Threshold-based multi-level assignment for one query block ([article]
+    Method, finer levels for critical blocks, coarser for less important
+    ones, the least important skipped entirely; [article] Results, the
+    ablation favours thresholds for building the mask).  Reading R7."""
+    mass_row = np.asarray(mass_row, dtype=np.float64)
+    n = mass_row.shape[0]
+    order = sorted(range(n), key=lambda J: (-mass_row[J], J))
+    out = np.empty(n, dtype=np.int64)
+    C = 0.0
+    for J in order:
+        lev = sum(1 for t in thresholds if t <= C)
+        out[J] = SKIP if lev >= levels else lev
+        C += mass_row[J]
+    return out
+
+
+def exclusive_prefix(mass_row: Sequence[float]) -> np.ndarray:
+    """C_J of reading R7 for every J (used by the ambiguity band)."""
+    mass_row = np.asarray(mass_row, dtype=np.float64)
+    order = sorted(range(mass_row.shape[0]), key=lambda J: (-mass_row[J], J))
+    C = np.empty_like(mass_row)
+    acc = 0.0
+    for J in order:
+        C[J] = acc
+        acc += mass_row[J]
+    return C
+
+
+def apply_forced_rules(levels_row: np.ndarray, I: int, block: int, levels: int, causal: bool,
+                       n_dense_prefix: int = 0, cos_row: Optional[np.ndarray] = None,
+                       cos_min: float = -3.0) -> np.ndarray:
+    """Reading R8."""
+    out = levels_row.copy()
+    n = out.shape[0]
+    for J in range(n):
+        if n_dense_prefix > 0 and (I * block < n_dense_prefix or J * block < n_dense_prefix):
+            out[J] = 0
+        if cos_row is not None and cos_min > -2.0 and out[J] != SKIP and out[J] >= 1 \
+                and cos_row[J] < cos_min:
+            out[J] = 0
+        if causal:
+            if J > I:
+                out[J] = SKIP
+            elif J == I:
+                out[J] = 0
+    return out
+
+
+def make_mask(mass: np.ndarray, thresholds, levels: int, block: int, causal: bool,
+              n_dense_prefix: int = 0, blockcos: Optional[np.ndarray] = None, cos_min: float = -3.0,
+              hq_per_kv: int = 1, rows=None) -> np.ndarray:
+    """mass [B,Hq,nQB,nKB] -> mask uint8 of the same shape (SKIP = 0xFF)."""
+    B, Hq, nqb, nkb = mass.shape
+    out = np.full((B, Hq, nqb, nkb), SKIP, dtype=np.int64)
+    if rows is None:
+        rows = [(b, h, I) for b in range(B) for h in range(Hq) for I in range(nqb)]
+    for b, h, I in rows:
+        lev = assign_levels_row(mass[b, h, I], thresholds, levels)
+        cos_row = None if blockcos is None else blockcos[b, h // hq_per_kv]
+        out[b, h, I] = apply_forced_rules(lev, I, block, levels, causal, n_dense_prefix, cos_row, cos_min)
+    return out.astype(np.uint8)
+
+
+def ambiguous_pairs(mass: np.ndarray, thresholds, eps: float = 1e-6, rows=None,
+                    blockcos: Optional[np.ndarray] = None, cos_min: float = -3.0,
+                    hq_per_kv: int = 1) -> np.ndarray:
+    """Pairs whose level may legitimately differ between an fp32 and an fp64
+    evaluation: some threshold t lies within eps of the range of C_J that
+    near-equal masses (relative eps) allow, or the block cosine lies within
+    eps of cos_min.  Computed from the oracle's masses."""
+    B, Hq, nqb, nkb = mass.shape
+    amb = np.zeros(mass.shape, dtype=bool)
+    if rows is None:
+        rows = [(b, h, I) for b in range(B) for h in range(Hq) for I in range(nqb)]
+    for b, h, I in rows:
+        m = mass[b, h, I]
+        for J in range(nkb):
+            lo = m[m > m[J] * (1 + eps)].sum()
+            hi = m[m >= m[J] * (1 - eps)].sum() - m[J]
+            for t in thresholds:
+                if lo - eps <= t <= hi + eps:
+                    amb[b, h, I, J] = True
+            if blockcos is not None and cos_min > -2.0 and abs(blockcos[b, h // hq_per_kv, J] - cos_min) <= eps:
+                amb[b, h, I, J] = True
+    return amb
+
+
+# ======================================================================================
+# Stage 3: adaptive pyramid attention
+# ======================================================================================
+
+def level_bias(level: int) -> float:
+    """Reading R1 of the consistency scale ([article] Method, a scale factor
+    keeps the attention probabilities consistent across levels):
+    a level-l pooled token stands for 2^l tokens, so its logit gets +ln(2^l)."""
+    return level * LN2
+
+
+def gather_keys(kp, vp, mask_row: Sequence[int], block: int, N: int, b: int, hk: int):
+    """The key set of one query block ([article] Method, each KV block is
+    read at the pyramid level the mask assigns it): for every
+    non-skipped KV block J at level l, the level-l pooled tokens of J.
+
+    Returns (keys [n, d], values [n, d], bias [n], last_token [n])."""
+    ks, vs, bias, last = [], [], [], []
+    for J, l in enumerate(mask_row):
+        l = int(l)
+        if l == SKIP:
+            continue
+        g = 1 << l
+        p0 = (J * block) // g
+        p1 = min((J + 1) * block, N) // g
+        ks.append(kp[l][b, hk, p0:p1])
+        vs.append(vp[l][b, hk, p0:p1])
+        bias.append(np.full(p1 - p0, level_bias(l)))
+        last.append((np.arange(p0, p1) + 1) * g - 1)
+    if not ks:
+        d = kp[0].shape[-1]
+        return np.zeros((0, d)), np.zeros((0, d)), np.zeros(0), np.zeros(0, dtype=np.int64)
+    return np.concatenate(ks), np.concatenate(vs), np.concatenate(bias), np.concatenate(last)
+
+
+def attention(q, kp, vp, mask, block: int, sm_scale: float, causal: bool,
+              rows: Optional[Iterable[Tuple[int, int, int]]] = None):
+    """Adaptive pyramid attention ([article] Method; [news] Methodology 4,
+    ordinary scaled dot-product attention).  For query token i of block I:
+
+        z_p = sm_scale * q_i . K^l[p] + ln(2^l)     over the key set of I
+        o_i = sum_p softmax(z)_p V^l[p],   lse_i = log sum_p exp(z_p)
+
+    with readings R1-R4.  q: [B, Hq, N, d]; kp/vp: lists of the pyramid
+    levels (level 0 first) as returned by :func:`build_pyramid`; mask
+    [B, Hq, nQB, nKB].  Returns (o [B,Hq,N,d], lse [B,Hq,N]); when ``rows``
+    lists (b, h, I) triples only those query blocks are computed (the rest
+    stay NaN)."""
+    q = _f64(q)
+    mask = np.asarray(mask.cpu() if hasattr(mask, "cpu") else mask).astype(np.int64)
+    B, Hq, N, d = q.shape
+    Hkv = kp[0].shape[1]
+    grp = Hq // Hkv
+    nb = -(-N // block)
+    o = np.full((B, Hq, N, d), np.nan)
+    lse = np.full((B, Hq, N), np.nan)
+    if rows is None:
+        rows = [(b, h, I) for b in range(B) for h in range(Hq) for I in range(nb)]
+    for b, h, I in rows:
+        i0, i1 = I * block, min((I + 1) * block, N)
+        keys, vals, bias, last = gather_keys(kp, vp, mask[b, h, I], block, N, b, h // grp)
+        z = sm_scale * (q[b, h, i0:i1] @ keys.T) + bias[None, :]
+        visible = np.ones(z.shape, dtype=bool)
+        if causal:
+            qi = np.arange(i0, i1)
+            visible = last[None, :] <= qi[:, None]
+            z = np.where(visible, z, -np.inf)
+        empty = ~visible.any(axis=1)
+        m = z.max(axis=1, keepdims=True) if z.shape[1] else np.zeros((i1 - i0, 1))
+        m = np.where(empty[:, None], 0.0, m)
+        e = np.exp(z - m)
+        s = e.sum(axis=1)
+        o[b, h, i0:i1] = np.where(empty[:, None], 0.0, (e @ vals) / np.where(empty, 1.0, s)[:, None])
+        lse[b, h, i0:i1] = np.where(empty, -np.inf, m[:, 0] + np.log(np.where(empty, 1.0, s)))
+    return o, lse
+
+
+def executed_flops(mask, N: int, block: int, d: int, causal: bool = False) -> float:
+    """Useful work of one attention call: 4 * d * sum over (b, h, I) of
+    (valid query rows of I) * (pooled key rows fetched for I).  Diagonal
+    blocks count in full under causal masking; tile padding is not work."""
+    m = np.asarray(mask.cpu() if hasattr(mask, "cpu") else mask).astype(np.int64)
+    B, H, nqb, nkb = m.shape
+    qrows = np.array([min((I + 1) * block, N) - I * block for I in range(nqb)], dtype=np.float64)
+    total = 0.0
+    for l in range(4):
+        g = 1 << l
+        krows = np.array([(min((J + 1) * block, N) - J * block) // g for J in range(nkb)], dtype=np.float64)
+        sel = (m == l)
+        total += float((sel * qrows[None, None, :, None] * krows[None, None, None, :]).sum())
+    return 4.0 * d * total

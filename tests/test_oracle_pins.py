@@ -1,0 +1,525 @@
+"""Pins for the CPU oracle: each oracle function is checked against
+something other than itself.
+
+  function              pins
+  --------------------  ---------------------------------------------------------
+  pool_level            hand-computed golden values; constant groups are a fixed
+                        point; a linear ramp pools to the group midpoints (closed
+                        form); direct mean == progressive pairwise pooling
+  block_cosine          closed forms (parallel = 1, orthogonal = 0, antipodal =
+                        -1, single key = 1); the algebraic identity
+                        (|sum u_i|^2 - sum |u_i|^2) / (n(n-1)); scale invariance
+  sampling_mass         sum over J == 1; pure-Python brute force; torch.softmax
+                        (an independent library routine); one-hot alignment
+  antidiag_logits/mass  element-wise brute force; stride 1 reduces to the
+                        block-summed full softmax (torch); sum over J == 1
+  assign_levels_row     hand-computed golden cases; monotone in rank; top = 0
+  apply_forced_rules    hand-computed golden cases
+  attention             all-level-0 == torch SDPA (fp64); expanded-KV SDPA
+                        equivalence; identical-group invariance; NaN in a
+                        skipped block changes nothing; pure-Python brute force
+                        over an exhaustive {0,1,2,3,SKIP} mask; empty rows
+  mutation tests        planted mistakes (bias sign, dropped bias, sum instead of
+                        mean, wrong block width, inclusive prefix, transposed
+                        antidiagonal) each make a pin fail
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.psa_oracle as O
+from oracle.psa_oracle import SKIP
+
+RNG = np.random.default_rng(1234)
+
+
+# --------------------------------------------------------------------------------------
+# helpers that do NOT use the oracle's code paths
+# --------------------------------------------------------------------------------------
+
+def sdpa64(q, k, v, scale, attn_mask=None):
+    """torch's fused SDPA in float64 on the CPU: an independent routine."""
+    qt = torch.as_tensor(q, dtype=torch.float64)[None, None]
+    kt = torch.as_tensor(k, dtype=torch.float64)[None, None]
+    vt = torch.as_tensor(v, dtype=torch.float64)[None, None]
+    m = None if attn_mask is None else torch.as_tensor(attn_mask)[None, None]
+    return torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=m, scale=scale)[0, 0].numpy()
+
+
+def brute_attention_row(qi, i, K, V, mask_row, block, N, scale, causal):
+    """Pure-Python loops: pool each used block on the fly, add ln(2^l),
+    exponentiate, normalise."""
+    zs, vs = [], []
+    d = len(qi)
+    for J, l in enumerate(mask_row):
+        if l == SKIP:
+            continue
+        g = 2 ** l
+        t = J * block
+        while t < min((J + 1) * block, N):
+            kk = [sum(K[t + u][c] for u in range(g)) / g for c in range(d)]
+            vv = [sum(V[t + u][c] for u in range(g)) / g for c in range(d)]
+            if (not causal) or (t + g - 1 <= i):
+                zs.append(scale * sum(qi[c] * kk[c] for c in range(d)) + l * math.log(2.0))
+                vs.append(vv)
+            t += g
+    if not zs:
+        return [0.0] * d, -math.inf
+    m = max(zs)
+    e = [math.exp(z - m) for z in zs]
+    s = sum(e)
+    o = [sum(e[p] * vs[p][c] for p in range(len(e))) / s for c in range(d)]
+    return o, m + math.log(s)
+
+
+def rand(*shape):
+    return RNG.standard_normal(shape)
+
+
+# --------------------------------------------------------------------------------------
+# pyramid
+# --------------------------------------------------------------------------------------
+
+def pin_pyramid_golden(golden_dir, mod=O):
+    g = json.load(open(os.path.join(golden_dir, "pyramid_hand.json")))
+    x = np.array(g["tokens"], dtype=np.float64).reshape(1, 1, -1, 1)
+    err = 0.0
+    for l, want in g["levels"].items():
+        got = mod.pool_level(x, int(l))[0, 0, :, 0]
+        err = max(err, float(np.abs(got - np.array(want)).max()))
+    return err
+
+
+def test_pyramid_golden(golden_dir):
+    assert pin_pyramid_golden(golden_dir) == 0.0
+
+
+def test_pyramid_constant_groups_fixed_point():
+    base = rand(1, 2, 16, 5)
+    x = np.repeat(base, 8, axis=2)                # every aligned 8-group is constant
+    for l in (1, 2, 3):
+        got = O.pool_level(x, l)
+        want = np.repeat(base, 8 >> l, axis=2)
+        assert np.abs(got - want).max() < 1e-14
+
+
+def test_pyramid_linear_ramp_midpoints():
+    N, a, c = 64, 0.37, -1.5
+    t = np.arange(N, dtype=np.float64)
+    x = (a * t + c).reshape(1, 1, N, 1) * np.ones((1, 1, 1, 3))
+    for l in (1, 2, 3):
+        g = 2 ** l
+        p = np.arange(N // g)
+        want = a * (p * g + (g - 1) / 2.0) + c
+        assert np.abs(O.pool_level(x, l)[0, 0, :, 1] - want).max() < 1e-12
+
+
+def test_pyramid_progressive_equals_direct():
+    x = rand(2, 3, 40, 7)
+    prev = x
+    for l in (1, 2, 3):
+        prog = 0.5 * (prev[:, :, 0::2] + prev[:, :, 1::2])
+        assert np.abs(prog - O.pool_level(x, l)).max() < 1e-13
+        prev = prog
+
+
+# --------------------------------------------------------------------------------------
+# block cosine
+# --------------------------------------------------------------------------------------
+
+def test_block_cosine_closed_forms():
+    d = 4
+    e0, e1 = np.eye(d)[0], np.eye(d)[1]
+    k = np.zeros((1, 1, 8, d))
+    k[0, 0, 0:4] = [2 * e0, 3 * e0, 0.5 * e0, 7 * e0]     # parallel -> 1
+    k[0, 0, 4:6] = [e0, e1]                                # orthogonal -> 0
+    k[0, 0, 6:8] = [e1, -4 * e1]                           # antipodal -> -1
+    assert abs(O.block_cosine(k[:, :, 0:4], 4)[0, 0, 0] - 1) < 1e-14
+    assert abs(O.block_cosine(k[:, :, 4:6], 2)[0, 0, 0] - 0) < 1e-14
+    assert abs(O.block_cosine(k[:, :, 6:8], 2)[0, 0, 0] + 1) < 1e-14
+    one = rand(1, 1, 1, d)
+    assert O.block_cosine(one, 4)[0, 0, 0] == 1.0           # single key (ragged tail)
+
+
+def test_block_cosine_identity_and_zero_key():
+    k = rand(1, 2, 37, 6)
+    k[0, 1, 5] = 0.0                                        # a zero key has unit vector 0
+    blk = 16
+    got = O.block_cosine(k, blk)
+    for h in range(2):
+        for J in range(3):
+            keys = k[0, h, J * blk:min((J + 1) * blk, 37)]
+            n = len(keys)
+            nrm = np.linalg.norm(keys, axis=1)
+            u = np.array([keys[i] / nrm[i] if nrm[i] > 0 else np.zeros(6) for i in range(n)])
+            s = u.sum(axis=0)
+            want = (s @ s - (u * u).sum()) / (n * (n - 1))
+            assert abs(got[0, h, J] - want) < 1e-13
+
+
+def test_block_cosine_scale_invariant():
+    k = rand(1, 1, 32, 5)
+    scales = np.abs(rand(1, 1, 32, 1)) + 0.1
+    assert np.abs(O.block_cosine(k, 8) - O.block_cosine(k * scales, 8)).max() < 1e-13
+
+
+# --------------------------------------------------------------------------------------
+# sampling score
+# --------------------------------------------------------------------------------------
+
+def test_sampling_rows_reading():
+    assert O.sampling_rows(0, 64, 1000) == [0, 8, 16, 24, 32, 40, 48, 56]
+    assert O.sampling_rows(2, 128, 300) == [256, 272, 288]       # rows >= N dropped
+    assert O.sampling_rows(1, 128, 10**6) == [128 + 16 * s for s in range(8)]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_sampling_mass_sums_to_one(causal):
+    q, k = rand(1, 4, 200, 8), rand(1, 2, 200, 8)
+    m = O.sampling_mass(q, k, 32, 0.35, causal=causal)
+    assert np.abs(m.sum(axis=-1) - 1).max() < 1e-12
+    if causal:
+        nb = m.shape[2]
+        for I in range(nb):
+            assert np.all(m[:, :, I, I + 1:] == 0)
+
+
+def test_sampling_mass_bruteforce():
+    N, d, blk, scale = 52, 3, 16, 0.7
+    q, k = rand(1, 2, N, d), rand(1, 1, N, d)
+    got = O.sampling_mass(q, k, blk, scale)
+    nb = -(-N // blk)
+    for h in range(2):
+        for I in range(nb):
+            rows = [I * blk + s * (blk // 8) for s in range(8) if I * blk + s * (blk // 8) < N]
+            acc = [0.0] * nb
+            for i in rows:
+                z = [scale * sum(q[0, h, i, c] * k[0, 0, j, c] for c in range(d)) for j in range(N)]
+                mx = max(z)
+                e = [math.exp(x - mx) for x in z]
+                s = sum(e)
+                for j in range(N):
+                    acc[j // blk] += e[j] / s / len(rows)
+            assert np.abs(np.array(acc) - got[0, h, I]).max() < 1e-12
+
+
+def test_sampling_mass_vs_torch_softmax():
+    N, d, blk, scale = 300, 16, 64, 0.25
+    q, k = rand(2, 3, N, d), rand(2, 3, N, d)
+    got = O.sampling_mass(q, k, blk, scale)
+    nb = -(-N // blk)
+    for b in range(2):
+        for h in range(3):
+            P = torch.softmax(torch.tensor(q[b, h]) @ torch.tensor(k[b, h]).T * scale, dim=1).numpy()
+            for I in range(nb):
+                rows = [r for r in range(I * blk, min(I * blk + blk, N)) if (r - I * blk) % (blk // 8) == 0]
+                sums = np.array([P[rows, J * blk:(J + 1) * blk].sum(axis=1).mean() for J in range(nb)])
+                assert np.abs(sums - got[b, h, I]).max() < 1e-12
+
+
+def test_sampling_mass_one_hot():
+    N, d, blk = 256, 16, 32
+    q = np.zeros((1, 1, N, d))
+    k = 0.01 * rand(1, 1, N, d)
+    Jstar = 5
+    k[0, 0, Jstar * blk:(Jstar + 1) * blk, 0] = 1.0
+    q[0, 0, :, 0] = 60.0
+    m = O.sampling_mass(q, k, blk, 1.0)
+    assert np.all(m[0, 0, :, Jstar] > 1 - 1e-12)
+    mask = O.make_mask(m, (0.6, 0.8, 0.9, 0.95), 4, blk, False)
+    assert np.all(mask[0, 0, :, Jstar] == 0)
+    others = np.delete(mask[0, 0], Jstar, axis=1)
+    assert np.all(others == SKIP)
+
+
+# --------------------------------------------------------------------------------------
+# antidiagonal score
+# --------------------------------------------------------------------------------------
+
+def test_antidiag_logits_bruteforce():
+    N, d, S, scale = 24, 3, 4, 0.9
+    qh, kh = rand(N, d), rand(N, d)
+    A = O.antidiag_logits(qh, kh, S, scale)
+    for a in range(N // S):
+        for c in range(N // S):
+            acc = 0.0
+            for s in range(S):
+                i, j = a * S + (S - 1 - s), c * S + s      # bottom-left to top-right of the S x S tile
+                acc += sum(qh[i, x] * kh[j, x] for x in range(d))
+            assert abs(A[a, c] - scale * acc / S) < 1e-12
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_antidiag_stride1_is_block_softmax(causal):
+    N, d, blk, scale = 96, 8, 32, 0.4
+    q, k = rand(1, 2, N, d), rand(1, 1, N, d)
+    got = O.antidiag_mass(q, k, blk, 1, scale, causal)
+    for h in range(2):
+        Z = torch.tensor(q[0, h]) @ torch.tensor(k[0, 0]).T * scale
+        if causal:
+            Z = Z.masked_fill(torch.triu(torch.ones(N, N, dtype=torch.bool), 1), -math.inf)
+        P = torch.softmax(Z, dim=1).numpy()
+        for I in range(N // blk):
+            want = P[I * blk:(I + 1) * blk].reshape(blk, N // blk, blk).sum(axis=2).mean(axis=0)
+            assert np.abs(got[0, h, I] - want).max() < 1e-12
+
+
+def test_antidiag_mass_sums_to_one():
+    q, k = rand(1, 4, 256, 8), rand(1, 2, 256, 8)
+    m = O.antidiag_mass(q, k, 64, 8, 0.3, causal=True)
+    assert np.abs(m.sum(axis=-1) - 1).max() < 1e-12
+    for I in range(4):
+        assert np.all(m[:, :, I, I + 1:] == 0)
+
+
+# --------------------------------------------------------------------------------------
+# level assignment and forced rules
+# --------------------------------------------------------------------------------------
+
+def test_levels_golden(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "levels_hand.json")))
+    for case in g["cases"]:
+        got = O.assign_levels_row(case["mass"], case["thresholds"], case["levels"])
+        assert list(got) == case["expect"], case
+        assert list(O.exclusive_prefix(case["mass"])) == case["prefix"]
+
+
+def test_levels_monotone_in_rank():
+    for _ in range(20):
+        m = RNG.dirichlet(np.ones(50) * 0.3)
+        lev = O.assign_levels_row(m, (0.6, 0.8, 0.9, 0.95), 4)
+        order = sorted(range(50), key=lambda J: (-m[J], J))
+        ranked = [255 if lev[J] == SKIP else lev[J] for J in order]
+        assert ranked == sorted(ranked)
+        assert lev[order[0]] == 0
+
+
+def test_forced_rules_golden(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "forced_hand.json")))
+    for c in g["cases"]:
+        cos = None if c["cos"] is None else np.array(c["cos"])
+        got = O.apply_forced_rules(np.array(c["levels_in"]), c["I"], c["block"], c["L"], c["causal"],
+                                   c["n_dense_prefix"], cos, c["cos_min"])
+        assert list(got) == c["expect"], c
+
+
+# --------------------------------------------------------------------------------------
+# attention
+# --------------------------------------------------------------------------------------
+
+def _pyr(k, v, L):
+    return O.build_pyramid(k, v, L)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_attention_level0_is_dense_sdpa(causal):
+    B, Hq, Hkv, N, d, blk = 1, 4, 2, 200, 16, 32
+    q, k, v = rand(B, Hq, N, d), rand(B, Hkv, N, d), rand(B, Hkv, N, d)
+    nb = -(-N // blk)
+    mask = np.zeros((B, Hq, nb, nb), dtype=np.uint8)
+    kp, vp = _pyr(k, v, 4)
+    o, lse = O.attention(q, kp, vp, mask, blk, 0.3, causal)
+    for h in range(Hq):
+        am = None
+        if causal:
+            am = torch.tril(torch.ones(N, N, dtype=torch.bool))
+        want = sdpa64(q[0, h], k[0, h // 2], v[0, h // 2], 0.3, am)
+        assert np.abs(o[0, h] - want).max() < 1e-12
+        z = 0.3 * q[0, h] @ k[0, h // 2].T
+        if causal:
+            z = np.where(np.tril(np.ones((N, N), dtype=bool)), z, -np.inf)
+        want_lse = torch.logsumexp(torch.tensor(z), dim=1).numpy()
+        assert np.abs(lse[0, h] - want_lse).max() < 1e-12
+
+
+def test_attention_expanded_kv_equivalence():
+    """A level-l pooled token with +ln(2^l) equals that token repeated 2^l
+    times inside a plain softmax."""
+    B, H, N, d, blk, L = 1, 2, 160, 8, 32, 4
+    q, k, v = rand(B, H, N, d), rand(B, H, N, d), rand(B, H, N, d)
+    nb = N // blk
+    gen = np.random.default_rng(7)
+    mask = gen.choice([0, 1, 2, 3, SKIP], size=(B, H, nb, nb)).astype(np.uint8)
+    mask[..., 0] = 2
+    kp, vp = _pyr(k, v, L)
+    o, _ = O.attention(q, kp, vp, mask, blk, 0.4, False)
+    for h in range(H):
+        for I in range(nb):
+            kt, vt = [], []
+            for J in range(nb):
+                l = int(mask[0, h, I, J])
+                if l == SKIP:
+                    continue
+                g = 2 ** l
+                blockk = k[0, h, J * blk:(J + 1) * blk].reshape(blk // g, g, d).mean(axis=1)
+                blockv = v[0, h, J * blk:(J + 1) * blk].reshape(blk // g, g, d).mean(axis=1)
+                kt.append(np.repeat(blockk, g, axis=0))
+                vt.append(np.repeat(blockv, g, axis=0))
+            want = sdpa64(q[0, h, I * blk:(I + 1) * blk], np.concatenate(kt), np.concatenate(vt), 0.4)
+            assert np.abs(o[0, h, I * blk:(I + 1) * blk] - want).max() < 1e-12
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_attention_identical_groups_equal_dense(causal):
+    B, H, d, blk = 1, 2, 8, 32
+    base_k, base_v = rand(B, H, 24, d), rand(B, H, 24, d)
+    k, v = np.repeat(base_k, 8, axis=2), np.repeat(base_v, 8, axis=2)   # N = 192, 8-groups identical
+    N = k.shape[2]
+    q = rand(B, H, N, d)
+    nb = N // blk
+    gen = np.random.default_rng(3)
+    mask = gen.integers(0, 4, size=(B, H, nb, nb)).astype(np.uint8)
+    if causal:
+        # only whole groups in the past are visible under pooling, so compare on a dense
+        # reference that masks at 8-group granularity for off-diagonal blocks
+        for I in range(nb):
+            mask[:, :, I, I] = 0
+    kp, vp = _pyr(k, v, 4)
+    o, _ = O.attention(q, kp, vp, mask, blk, 0.5, causal)
+    for h in range(H):
+        am = None
+        if causal:
+            am = torch.tril(torch.ones(N, N, dtype=torch.bool))
+        want = sdpa64(q[0, h], k[0, h], v[0, h], 0.5, am)
+        assert np.abs(o[0, h] - want).max() < 1e-12
+
+
+def test_attention_skip_ignores_nan():
+    B, H, N, d, blk = 1, 2, 128, 8, 32
+    q, k, v = rand(B, H, N, d), rand(B, H, N, d), rand(B, H, N, d)
+    nb = N // blk
+    mask = np.random.default_rng(5).choice([0, 1, 2, 3], size=(B, H, nb, nb)).astype(np.uint8)
+    mask[0, :, :2, 2] = SKIP
+    kp, vp = _pyr(k, v, 4)
+    o1, l1 = O.attention(q, kp, vp, mask, blk, 0.3, False)
+    k2, v2 = k.copy(), v.copy()
+    k2[:, :, 2 * blk:3 * blk] = np.nan
+    v2[:, :, 2 * blk:3 * blk] = np.nan
+    kp2, vp2 = _pyr(k2, v2, 4)
+    o2, l2 = O.attention(q, kp2, vp2, mask, blk, 0.3, False)
+    assert np.array_equal(o1[:, :, :2 * blk], o2[:, :, :2 * blk])
+    assert np.array_equal(l1[:, :, :2 * blk], l2[:, :, :2 * blk])
+    assert np.isnan(o2[:, :, 2 * blk:]).all()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_attention_bruteforce_exhaustive_mask(causal):
+    """4x4 block grid; the mask lists every value of {0,1,2,3,SKIP} in every
+    row position across the grid (cyclic), N ragged (not a block multiple)."""
+    H, d, blk = 2, 4, 16
+    N = 56                                    # blocks of 16,16,16,8
+    q, k, v = rand(1, H, N, d), rand(1, H, N, d), rand(1, H, N, d)
+    vals = [0, 1, 2, 3, SKIP]
+    mask = np.zeros((1, H, 4, 4), dtype=np.uint8)
+    for h in range(H):
+        for I in range(4):
+            for J in range(4):
+                mask[0, h, I, J] = vals[(I * 4 + J + h) % 5]
+    kp, vp = _pyr(k, v, 4)
+    o, lse = O.attention(q, kp, vp, mask, blk, 0.45, causal)
+    for h in range(H):
+        for i in range(N):
+            want_o, want_lse = brute_attention_row(list(q[0, h, i]), i, k[0, h].tolist(), v[0, h].tolist(),
+                                                   [int(x) for x in mask[0, h, i // blk]], blk, N, 0.45, causal)
+            assert np.abs(o[0, h, i] - np.array(want_o)).max() < 1e-12
+            if math.isinf(want_lse):
+                assert lse[0, h, i] == -math.inf
+            else:
+                assert abs(lse[0, h, i] - want_lse) < 1e-12
+
+
+def test_attention_empty_rows():
+    q, k, v = rand(1, 1, 64, 4), rand(1, 1, 64, 4), rand(1, 1, 64, 4)
+    mask = np.full((1, 1, 2, 2), SKIP, dtype=np.uint8)
+    mask[0, 0, 1, 0] = 1
+    kp, vp = _pyr(k, v, 2)
+    o, lse = O.attention(q, kp, vp, mask, 32, 0.5, False)
+    assert np.all(o[0, 0, :32] == 0) and np.all(lse[0, 0, :32] == -np.inf)
+    assert np.all(np.isfinite(o[0, 0, 32:]))
+
+
+def test_executed_flops_counts():
+    mask = np.array([[[[0, 1], [SKIP, 3]]]], dtype=np.uint8)
+    # N = 48, block 32: q rows 32, 16; k rows level0 32 / level1 16/2=8 ; level3 (16)/8=2
+    f = O.executed_flops(mask, 48, 32, 4)
+    want = 4 * 4 * (32 * 32 + 32 * 8 + 16 * 2)
+    assert f == want
+
+
+# --------------------------------------------------------------------------------------
+# mutation tests: planted mistakes in the oracle must make a pin fail
+# --------------------------------------------------------------------------------------
+
+def _run_identical_groups_pin():
+    try:
+        test_attention_identical_groups_equal_dense(False)
+        return True
+    except AssertionError:
+        return False
+
+
+def test_mutation_bias_sign(monkeypatch):
+    monkeypatch.setattr(O, "level_bias", lambda l: -l * math.log(2.0))
+    assert not _run_identical_groups_pin()
+
+
+def test_mutation_bias_dropped(monkeypatch):
+    monkeypatch.setattr(O, "level_bias", lambda l: 0.0)
+    assert not _run_identical_groups_pin()
+
+
+def test_mutation_pool_sum(monkeypatch, golden_dir):
+    orig = O.pool_level
+    monkeypatch.setattr(O, "pool_level", lambda x, l: orig(x, l) * (1 << l))
+    assert pin_pyramid_golden(golden_dir, O) > 0
+
+
+def test_mutation_block_width(monkeypatch):
+    orig = O._block_sum
+    monkeypatch.setattr(O, "_block_sum", lambda p, w, n: orig(np.roll(p, 1, axis=1), w, n))
+    with pytest.raises(AssertionError):
+        test_sampling_mass_bruteforce()
+
+
+def test_mutation_inclusive_prefix(monkeypatch, golden_dir):
+    def bad(mass_row, thresholds, levels):
+        mass_row = np.asarray(mass_row, dtype=np.float64)
+        order = sorted(range(len(mass_row)), key=lambda J: (-mass_row[J], J))
+        out = np.empty(len(mass_row), dtype=np.int64)
+        C = 0.0
+        for J in order:
+            C += mass_row[J]
+            lev = sum(1 for t in thresholds if t <= C)
+            out[J] = SKIP if lev >= levels else lev
+        return out
+    monkeypatch.setattr(O, "assign_levels_row", bad)
+    with pytest.raises(AssertionError):
+        test_levels_golden(golden_dir)
+
+
+def test_mutation_antidiag_not_reversed(monkeypatch):
+    def bad(qh, kh, stride, sm_scale):
+        N, d = qh.shape
+        G = N // stride
+        A = np.zeros((G, G))
+        for s in range(stride):
+            A += qh[np.arange(G) * stride + s] @ kh[np.arange(G) * stride + s].T
+        return (sm_scale / stride) * A
+    monkeypatch.setattr(O, "antidiag_logits", bad)
+    with pytest.raises(AssertionError):
+        test_antidiag_logits_bruteforce()
+
+
+def test_mutation_transposed_attention_operand(monkeypatch):
+    """Swapping K and V in the key gather must break the dense pin."""
+    orig = O.gather_keys
+
+    def bad(kp, vp, *a, **kw):
+        return orig(vp, kp, *a, **kw)
+    monkeypatch.setattr(O, "gather_keys", bad)
+    with pytest.raises(AssertionError):
+        test_attention_level0_is_dense_sdpa(False)
