@@ -1,0 +1,425 @@
+#!/usr/bin/env python3
+"""Benchmark of the PSA forward path (pyramid -> mask -> attention) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config wan14b] [--impl psa|reference]
+
+One step = one pass of the whole path over one synthetic input of the
+chosen workload (default: the Wan2.1-14B-shaped 720p self-attention, B1 H40
+N75600 d128 bf16, block 128, L 4, sampling mask): psa_build_pyramid,
+psa_make_mask, psa_attention_fwd, all through the C ABI.  Inputs (2.3 GB)
+are larger than L2, so no flush is needed between steps.
+
+value = executed attention FLOPs of all ranks / (max over ranks of the
+device time of K steps) in TFLOP/s, where executed FLOPs count only real
+work: 4 d sum over (b, h, I) of (query rows of I) x (pooled key rows the
+mask fetches for I); skipped blocks and tile padding are not work.
+
+--impl reference times the CPU oracle (the only other implementation of
+this path) on the machine's host cores, on a bounded sample of the same
+workload, in the same unit.  With torchrun (N > 1) every rank runs its own
+full workload instance (weak scaling, no data-path collective); only the
+timing is reduced (max over ranks).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "PSA attn fwd ms/call & achieved TFLOP/s (executed FLOPs) vs B200 BF16 peak"
+UNIT = "TFLOP/s"
+KERNELS_PER_STEP = {"pyramid": 1, "blockcos": 0, "score": 1, "select": 1, "plan": 3, "attention": 1}
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p["bf16_tflops"], p["bf16_tflops_sustained"], p["hbm_gbs"], "measured"
+    except Exception:
+        return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev_index: int):
+        self.dev = dev_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(self.dev)], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def executed_flops(mask: torch.Tensor, N: int, block: int, d: int, levels: int, causal: bool) -> float:
+    """4 d sum_{b,h,I} q_I * sum_{J: M != SKIP} k_J / 2^l (on the device)."""
+    dev = mask.device
+    nb = mask.shape[-1]
+    idx = torch.arange(nb, device=dev)
+    qrows = (torch.clamp((idx + 1) * block, max=N) - idx * block).double()
+    m = mask.long()
+    total = torch.zeros((), dtype=torch.float64, device=dev)
+    for l in range(levels):
+        krows = ((torch.clamp((idx + 1) * block, max=N) - idx * block) // (1 << l)).double()
+        sel = (m == l).double()
+        if causal:
+            sel = sel * torch.tril(torch.ones(nb, nb, device=dev, dtype=torch.float64))
+        total += (sel * qrows[:, None] * krows[None, :]).sum()
+    return 4.0 * d * float(total.item())
+
+
+class Path:
+    """Device buffers and the three ABI calls of one workload instance."""
+
+    def __init__(self, w: W.Workload, q, k, v):
+        import video_transformers_b200 as P
+        self.P, self.w = P, w
+        self.q, self.k, self.v = q, k, v
+        dev = q.device
+        self.shape = P.make_shape(w.B, w.Hq, w.Hkv, w.N, w.d, w.block, w.levels, w.causal,
+                                  P.PSA_DT_FP32 if w.dtype == "fp32" else P.PSA_DT_BF16)
+        mode = P.PSA_MASK_SAMPLE if w.mask_mode == "sample" else P.PSA_MASK_ANTIDIAG
+        self.params = P.make_params(mode, w.thresholds or (0.6, 0.8, 0.9, 0.95)[:w.levels], w.sm_scale,
+                                    stride=w.stride, cos_min=w.cos_min, n_dense_prefix=w.n_dense_prefix)
+        self.kp, self.vp = P.pyramid_buffers(self.shape, dev, q.dtype)
+        nb = w.nqb
+        self.bc = torch.empty(w.B, w.Hkv, nb, dtype=torch.float32, device=dev) if w.cos_min > -2 else None
+        self.mask = torch.empty(w.B, w.Hq, nb, nb, dtype=torch.uint8, device=dev)
+        self.out = torch.empty_like(q)
+        self.mws = P.workspace(P.psa_mask_workspace_bytes(self.shape, self.params), dev)
+        self.aws = P.workspace(P.psa_attention_workspace_bytes(self.shape), dev)
+        self.given_mask = None
+
+    def pyramid(self):
+        self.P.psa_build_pyramid(self.shape, self.k, self.v, self.kp, self.vp, self.bc)
+
+    def make_mask(self):
+        if self.given_mask is not None:
+            self.mask.copy_(self.given_mask)
+        else:
+            self.P.psa_make_mask(self.shape, self.params, self.q, self.k, self.bc, self.mask, None, self.mws)
+
+    def attention(self, mask=None):
+        self.P.psa_attention_fwd(self.shape, self.q, self.k, self.v, self.kp, self.vp,
+                                 self.mask if mask is None else mask, self.w.sm_scale, self.out, None, self.aws)
+
+    def step(self):
+        self.pyramid()
+        self.make_mask()
+        self.attention()
+
+
+# ----------------------------------------------------------------------------- psa arm
+
+def run_psa(args, rank, world, local_rank):
+    import video_transformers_b200 as P
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = W.PRESETS[args.config]
+    q, k, v, gen = W.make_qkv(w, device=dev, seed=w.seed + rank)
+    path = Path(w, q, k, v)
+    if w.mask_mode == "given":
+        path.given_mask = W.make_given_mask(w, gen, device=dev)
+    stream = torch.cuda.current_stream()
+
+    # warm-up, and the executed work of one step (the mask is deterministic)
+    for _ in range(args.warmup):
+        path.step()
+    torch.cuda.synchronize()
+    flops = executed_flops(path.mask, w.N, w.block, w.d, w.levels, w.causal)
+    dense = W.dense_flops(w)
+    n_tiles, n_rows = P.psa_attention_plan_stats(path.shape, path.aws)
+
+    # timed region: K steps, events around each stage
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            path.pyramid()
+            ev[i][1].record(stream)
+            path.make_mask()
+            ev[i][2].record(stream)
+            path.attention()
+            ev[i][3].record(stream)
+        stop.record(stream)
+        torch.cuda.synchronize()
+    total_ms = start.elapsed_time(stop)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    st = P.psa_get_device_status(path.aws) or P.psa_get_device_status(path.mws)
+    if st != P.PSA_OK:
+        raise RuntimeError("device status %d after the timed region" % st)
+    pyr_ms = statistics.mean(ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps))
+    mask_ms = statistics.mean(ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps))
+    attn_ms = statistics.mean(ev[i][2].elapsed_time(ev[i][3]) for i in range(args.steps))
+    ms_per_step = total_ms / args.steps
+    value = flops * world / (ms_per_step * 1e-3) / 1e12
+
+    # dense reference point: same kernel, all-level-0 mask
+    dense_mask = torch.zeros_like(path.mask)
+    dense_ms = None
+    if not args.no_dense:
+        path.attention(dense_mask)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 2
+        e0.record(stream)
+        for _ in range(reps):
+            path.attention(dense_mask)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        dense_ms = e0.elapsed_time(e1) / reps
+        path.attention()          # leave the sparse plan in the workspace
+        torch.cuda.synchronize()
+
+    # end to end through the public API with host buffers
+    e2e = run_e2e(path, w, flops, args, stream) if not args.no_e2e else None
+
+    bf16_burst, bf16_sus, hbm, src = peaks()
+    attn_tflops = flops / (attn_ms * 1e-3) / 1e12
+    pyr_bytes = 2 * w.B * w.Hkv * w.N * w.d * q.element_size() * (1 + sum(2.0 ** -l for l in range(1, w.levels)))
+    hist = torch.bincount(path.mask.flatten().long(), minlength=256).cpu()
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "fp32 in, bf16 MMA",
+        "data": "synthetic (smooth Gaussian field + noise, seeded)" if w.recipe == "field" else "synthetic iid N(0,1)",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "block": w.block,
+                   "levels": w.levels, "causal": w.causal, "mask": w.mask_mode, "thresholds": list(w.thresholds),
+                   "l2": "inputs (%.2f GB) larger than L2; no flush" % ((q.numel() + 2 * k.numel()) * q.element_size() / 1e9),
+                   "step": "psa_build_pyramid + psa_make_mask + psa_attention_fwd",
+                   "parallelism": "replicas, one workload instance per GPU" if world > 1 else "single GPU"},
+        "stages_ms": {"pyramid": pyr_ms, "mask": mask_ms, "attention": attn_ms},
+        "attn_fwd_ms": attn_ms, "attn_fwd_tflops": attn_tflops,
+        "executed_tflop_per_step": flops / 1e12, "dense_tflop": dense / 1e12,
+        "density": flops / dense, "dense_level0_attn_ms": dense_ms,
+        "dense_equiv_speedup": (dense_ms / attn_ms) if dense_ms else None,
+        "level_histogram": {"l0": int(hist[0]), "l1": int(hist[1]), "l2": int(hist[2]), "l3": int(hist[3]),
+                            "skip": int(hist[255])},
+        "plan": {"kv_tiles": n_tiles, "real_kv_rows": n_rows, "padding_frac": 1 - n_rows / max(1, 128 * n_tiles)},
+        "roofline": {"bound": "tensor", "kernel": "attn_kernel (psa_attention_fwd incl. its 3 planner kernels)",
+                     "achieved": attn_tflops, "peak": bf16_sus, "unit": "TFLOP/s", "frac": attn_tflops / bf16_sus,
+                     "peak_kind": "sustained bf16 (%s)" % src, "frac_of_burst": attn_tflops / bf16_burst,
+                     "traffic": None},
+        "pyramid_roofline": {"bound": "hbm", "achieved": pyr_bytes / (pyr_ms * 1e-3) / 1e9, "peak": hbm,
+                             "unit": "GB/s", "frac": pyr_bytes / (pyr_ms * 1e-3) / 1e9 / hbm},
+        "e2e": e2e,
+        "gpu_launches": sum(KERNELS_PER_STEP.values()) * args.steps + (1 if w.cos_min > -2 else 0) * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(w, q, k, v, path, args)
+    return line
+
+
+def run_e2e(path, w, flops, args, stream):
+    """Same step through the public API with pinned host buffers: H2D of q, k,
+    v and D2H of the output and mask inside the timed region."""
+    hq = torch.empty(path.q.shape, dtype=path.q.dtype, pin_memory=True).copy_(path.q)
+    hk = torch.empty(path.k.shape, dtype=path.k.dtype, pin_memory=True).copy_(path.k)
+    hv = torch.empty(path.v.shape, dtype=path.v.dtype, pin_memory=True).copy_(path.v)
+    ho = torch.empty(path.out.shape, dtype=path.out.dtype, pin_memory=True)
+    hm = torch.empty(path.mask.shape, dtype=torch.uint8, pin_memory=True)
+    steps = max(1, min(args.steps, 3))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        path.q.copy_(hq, non_blocking=True)
+        path.k.copy_(hk, non_blocking=True)
+        path.v.copy_(hv, non_blocking=True)
+        path.step()
+        ho.copy_(path.out, non_blocking=True)
+        hm.copy_(path.mask, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    return {"value": flops / (ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": ms, "steps": steps,
+            "h2d_bytes_per_step": (hq.numel() + hk.numel() + hv.numel()) * hq.element_size(),
+            "d2h_bytes_per_step": ho.numel() * ho.element_size() + hm.numel()}
+
+
+# ----------------------------------------------------------------------------- oracle legs
+
+def oracle_sample(w, q, k, v, n_blocks, seed=0, mask_dev=None):
+    """The oracle on a bounded sample: one (b, h), ``n_blocks`` query blocks.
+    Runs the pyramid of that head, the mask rows of the sample, and the
+    attention of those rows.  Returns (seconds, executed flops, description)."""
+    import oracle.psa_oracle as O
+    rng = np.random.default_rng(seed)
+    b, h = 0, int(rng.integers(w.Hq))
+    hk = h // (w.Hq // w.Hkv)
+    Is = sorted(rng.choice(w.nqb, size=min(n_blocks, w.nqb), replace=False).tolist())
+    qh = q[b:b + 1, h:h + 1].cpu()
+    kh = k[b:b + 1, hk:hk + 1].cpu()
+    vh = v[b:b + 1, hk:hk + 1].cpu()
+    t0 = time.perf_counter()
+    kl, vl = O.build_pyramid(kh, vh, w.levels)
+    rows = [(0, 0, I) for I in Is]
+    if w.mask_mode == "given":
+        mask = mask_dev[b:b + 1, h:h + 1].cpu().numpy()
+    else:
+        if w.mask_mode == "sample":
+            mass = O.sampling_mass(qh, kh, w.block, w.sm_scale, w.causal, rows=rows)
+        else:
+            mass = O.antidiag_mass(qh, kh, w.block, w.stride, w.sm_scale, w.causal, rows=rows)
+        cos = O.block_cosine(kh, w.block) if w.cos_min > -2 else None
+        mask = O.make_mask(mass, w.thresholds, w.levels, w.block, w.causal, w.n_dense_prefix, cos, w.cos_min,
+                           1, rows=rows)
+    O.attention(qh, kl, vl, mask, w.block, w.sm_scale, w.causal, rows=rows)
+    dt = time.perf_counter() - t0
+    sub = np.full_like(mask, 0xFF)
+    for _, _, I in rows:
+        sub[0, 0, I] = mask[0, 0, I]
+    fl = O.executed_flops(sub, w.N, w.block, w.d, w.causal)
+    desc = "b=0 h=%d, %d query blocks %s..., pyramid of that KV head, mask rows and attention rows" % (
+        h, len(Is), Is[:4])
+    return dt, fl, desc
+
+
+def cpu_baseline(w, q, k, v, path, args):
+    dt, fl, desc = oracle_sample(w, q, k, v, args.cpu_blocks, mask_dev=path.mask)
+    return {"value": fl / dt / 1e12, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+            "sample": desc, "seconds": dt}
+
+
+def cpu_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max([i.get("num_threads", 1) for i in info] + [1])
+    except Exception:
+        return os.cpu_count()
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    w = W.PRESETS[args.config]
+    q, k, v, gen = W.make_qkv(w, device="cuda" if torch.cuda.is_available() else "cpu")
+    mask = W.make_given_mask(w, gen, device=q.device) if w.mask_mode == "given" else None
+    for _ in range(args.warmup):
+        oracle_sample(w, q, k, v, 1, seed=99, mask_dev=mask)
+    secs, fl, desc = 0.0, 0.0, None
+    for i in range(args.steps):
+        dt, f, desc = oracle_sample(w, q, k, v, args.cpu_blocks, seed=i, mask_dev=mask)
+        secs += dt
+        fl += f
+    value = fl / secs / 1e12
+    return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic, seeded",
+            "impl": "reference",
+            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
+                       "block": w.block, "levels": w.levels, "causal": w.causal, "mask": w.mask_mode},
+            "cpu_baseline": {"value": value, "unit": UNIT, "kind": "oracle", "cores": cpu_threads(),
+                             "sample": "per step: " + desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ----------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default="wan14b", choices=W.ORDER)
+    ap.add_argument("--impl", default="psa", choices=["psa", "reference"])
+    ap.add_argument("--cpu-blocks", type=int, default=3, help="query blocks in the oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_psa(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

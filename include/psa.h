@@ -1,0 +1,195 @@
+/*
+ * psa.h -- C ABI of the Pyramid Sparse Attention (PSA) forward path on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method (pages: "PSA: Pyramid Sparse Attention for Efficient Video
+ * Understanding and Generation", summary article, section Method; the
+ * "psa-pyramid-sparse-attention" skill page, sections Core Technique and
+ * Implementation) has three steps, one entry point each:
+ *
+ *   psa_build_pyramid   KV pyramid: every KV block mean-pooled by 2, 4, 8
+ *   psa_make_mask       per (query block, KV block) pair: a pyramid level
+ *                       0..L-1 or SKIP, finer levels for more important pairs
+ *   psa_attention_fwd   online-softmax attention of every query block over
+ *                       its KV blocks, each read at its assigned level with a
+ *                       +ln(2^l) logit bias
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Tensors are contiguous row-major [B, H, N, d] in device memory, owned by
+ *    the caller, base pointers 16-byte aligned.  Query head h reads KV head
+ *    h / (Hq / Hkv).
+ *  - The library never allocates device memory.  Scratch comes from the
+ *    caller through a workspace pointer whose size the *_workspace_bytes
+ *    query returns.  A workspace must be zero-filled once before its first
+ *    use (it holds the device status word; see psa_get_device_status).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Every call is asynchronous on that stream.
+ *  - Arguments are validated on the host before anything is launched; on a
+ *    validation error nothing is written and the call returns
+ *    PSA_ERR_INVALID_ARG, PSA_ERR_UNSUPPORTED or PSA_ERR_WORKSPACE.  A failed
+ *    launch returns PSA_ERR_CUDA.  psa_last_error() then holds a message for
+ *    the calling thread.
+ *  - Supported set: dtype bf16 or fp32; d in {64, 128}; block in {64, 128};
+ *    1 <= levels <= 4; block and N multiples of 2^(levels-1); Hq a multiple
+ *    of Hkv; N >= 1; B*Hq*N*d < 2^31.  Anything else: PSA_ERR_UNSUPPORTED.
+ *  - Device waits inside the kernels are bounded (about 2 s); a wait that
+ *    runs out records PSA_ERR_TIMEOUT in the workspace status word and the
+ *    kernel returns early instead of hanging.
+ */
+#ifndef PSA_H
+#define PSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PSA_API __attribute__((visibility("default")))
+#else
+#define PSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PSA_OK = 0,
+  PSA_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad enum, misaligned pointer */
+  PSA_ERR_UNSUPPORTED = 2,   /* outside the supported set above */
+  PSA_ERR_WORKSPACE = 3,     /* workspace null or smaller than the query says */
+  PSA_ERR_CUDA = 4,          /* a CUDA runtime/driver call or a launch failed */
+  PSA_ERR_TIMEOUT = 5        /* a bounded device wait ran out (device status word) */
+} psa_status_t;
+
+typedef enum { PSA_DT_BF16 = 0, PSA_DT_FP32 = 1 } psa_dtype_t;
+
+typedef enum {
+  PSA_MASK_SAMPLE = 0,       /* generation task: sampled-query scoring */
+  PSA_MASK_ANTIDIAG = 1      /* understanding task: antidiagonal scoring */
+} psa_mask_mode_t;
+
+#define PSA_SKIP 0xFF
+#define PSA_MAX_LEVELS 4
+#define PSA_MAX_KV_BLOCKS 2048
+
+/* Problem shape.  N is the unpadded token count; the last query/KV block may
+ * be ragged.  causal != 0 hides keys after the query (a pooled token is
+ * visible to query i iff the last token it averages is <= i). */
+typedef struct {
+  int32_t B, Hq, Hkv, N, d;
+  int32_t block;             /* logical query and KV block size, tokens */
+  int32_t levels;            /* L: pyramid levels 0..L-1 (pool 1, 2, 4, 8) */
+  int32_t causal;
+  int32_t dtype;             /* psa_dtype_t of q, k, v, pyramid and output */
+} psa_shape_t;
+
+/* Mask generator parameters (summary article, Method: sampling-based scores
+ * for generation, antidiagonal scores plus an intra-block similarity check
+ * for understanding; Results: threshold-based levels and a cosine condition
+ * for pooling). */
+typedef struct {
+  int32_t mode;              /* psa_mask_mode_t */
+  int32_t n_samples;         /* sampled queries per query block; must be 8 */
+  int32_t stride;            /* antidiagonal stride S in {1, 2, 4, 8, 16}; block % S == 0 */
+  float thresholds[8];       /* ascending cumulative-mass thresholds t_0..t_{L-1} */
+  int32_t n_thresholds;      /* must equal shape.levels */
+  float cos_min;             /* cosine gate; <= -2 disables it */
+  int32_t n_dense_prefix;    /* tokens [0, n) are text: their blocks stay level 0 */
+  float sm_scale;            /* softmax scale of the score; usually 1/sqrt(d) */
+} psa_mask_params_t;
+
+/* ------------------------------------------------------------------------
+ * Stage 1: KV pyramid (skill page, Core Technique / Implementation; summary
+ * article, Method: repeated 1D mean pooling of every KV block).
+ *
+ * Level l (1 <= l < L) of K is [B, Hkv, N / 2^l, d]: token t is the mean of
+ * input tokens t*2^l .. t*2^l + 2^l - 1, summed in fp32 and rounded once to
+ * the shape's dtype (round to nearest even).  Levels 1..L-1 are stored back
+ * to back in one buffer per tensor; psa_pyramid_level_offset gives where
+ * level l starts (bytes, 16-byte aligned).  Level 0 is the input itself and
+ * is not copied.
+ *
+ * blockcos (optional, may be NULL): fp32 [B, Hkv, nKB], nKB = ceil(N/block),
+ * the mean pairwise cosine over i != j of the valid keys of each KV block
+ * (a zero key counts as the zero vector; a one-key block gives 1).  It feeds
+ * the cosine gate of psa_make_mask.
+ * ------------------------------------------------------------------------ */
+PSA_API size_t psa_pyramid_bytes(const psa_shape_t* shape);                   /* per tensor; 0 if L == 1 */
+PSA_API size_t psa_pyramid_level_offset(const psa_shape_t* shape, int level); /* level in [1, L) */
+PSA_API psa_status_t psa_build_pyramid(const psa_shape_t* shape, const void* k, const void* v,
+                               void* k_pyr, void* v_pyr, float* blockcos, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Stage 2: multi-level mask (summary article, Method and Results).
+ *
+ * Score, PSA_MASK_SAMPLE: query block I samples rows I*block + s*block/8,
+ * s = 0..7 (rows >= N dropped); each sampled row takes a softmax of
+ * sm_scale * q.k over all keys (keys <= the row when causal); the block
+ * mass mass[I, J] is the mean over the samples of the probability falling
+ * in KV block J.  Requires N % (block/8) == 0.
+ * Score, PSA_MASK_ANTIDIAG: with stride S, A[a, c] = (sm_scale/S) *
+ * sum_s q[a*S + S-1-s] . k[c*S + s]; softmax over key groups c (c <= a when
+ * causal); mass[I, J] = mean over the query groups of I of the probability
+ * in the key groups of J.  Requires N % S == 0.
+ * Levels: per row (b, h, I) rank J by mass (descending, ties to lower J),
+ * take the exclusive prefix C_J, level = #{t_l <= C_J}, SKIP when that count
+ * reaches L; then blocks holding a token < n_dense_prefix (as query or key
+ * block) -> 0; if cos_min > -2 and level >= 1 and blockcos[b, h_kv, J] <
+ * cos_min -> 0; if causal, J > I -> SKIP and J == I -> 0.
+ *
+ * mask: uint8 [B, Hq, nQB, nKB] (PSA_SKIP = 0xFF).  mass_out (optional):
+ * fp32 [B, Hq, nQB, nKB].  blockcos is required iff cos_min > -2.
+ * nKB <= PSA_MAX_KV_BLOCKS.
+ * ------------------------------------------------------------------------ */
+PSA_API size_t psa_mask_workspace_bytes(const psa_shape_t* shape, const psa_mask_params_t* params);
+PSA_API psa_status_t psa_make_mask(const psa_shape_t* shape, const psa_mask_params_t* params,
+                           const void* q, const void* k, const float* blockcos,
+                           uint8_t* mask, float* mass_out,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Stage 3: adaptive pyramid attention (summary article, Method: each KV
+ * block fetched at its assigned level, a scale factor keeping the
+ * probabilities consistent; news review, Methodology 4: plain scaled
+ * dot-product attention over the selected pooled KV).
+ *
+ * For query token i in block I, over every KV block J with
+ * l = mask[b, h, I, J] != SKIP and every pooled token p of J at level l:
+ *   z_p = sm_scale * q_i . K^l[p] + l * ln 2,
+ *   out_i = sum_p softmax(z)_p V^l[p],   lse_i = ln sum_p exp(z_p).
+ * Under causal masking p is visible iff (p+1)*2^l - 1 <= i.  A row with no
+ * visible key gets out = 0 and lse = -inf.  Rows >= N are not written.
+ *
+ * k_pyr/v_pyr: the buffers filled by psa_build_pyramid (NULL allowed iff
+ * L == 1).  out: [B, Hq, N, d] in the shape's dtype.  lse (optional): fp32
+ * [B, Hq, N], natural log.  For fp32 inputs the operands are rounded to
+ * bf16 inside the workspace and the products are accumulated in fp32.
+ * ------------------------------------------------------------------------ */
+PSA_API size_t psa_attention_workspace_bytes(const psa_shape_t* shape);
+PSA_API psa_status_t psa_attention_fwd(const psa_shape_t* shape, const void* q, const void* k, const void* v,
+                               const void* k_pyr, const void* v_pyr, const uint8_t* mask,
+                               float sm_scale, void* out, float* lse,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+/* Executed work of the last plan built in `workspace` by psa_attention_fwd:
+ * fills (synchronising on `stream`) the number of 128-row KV tiles and the
+ * number of KV rows that hold real (non-padding) pooled tokens. */
+PSA_API psa_status_t psa_attention_plan_stats(const psa_shape_t* shape, const void* workspace,
+                                      int64_t* n_tiles, int64_t* n_rows, void* stream);
+
+/* Reads the device status word of a workspace (synchronising on `stream`)
+ * and clears it: PSA_OK, or PSA_ERR_TIMEOUT if a bounded wait ran out in a
+ * kernel that used this workspace since the last read. */
+PSA_API psa_status_t psa_get_device_status(void* workspace, void* stream);
+
+/* Message of the last failed call on this thread ("" if none). */
+PSA_API const char* psa_last_error(void);
+
+/* ABI version: 100 * major + minor. */
+PSA_API int32_t psa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PSA_H */

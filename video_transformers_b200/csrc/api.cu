@@ -1,0 +1,452 @@
+// api.cu -- the C ABI of the PSA forward path (declared in include/psa.h):
+// argument validation, workspace layout, TMA descriptor encoding and kernel
+// launches.  Nothing here allocates device memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "internal.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+psa_status_t fail(psa_status_t st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+psa_status_t cuda_fail(cudaError_t e, const char* what) {
+  return fail(PSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+size_t elem_size(int dtype) { return dtype == PSA_DT_FP32 ? 4 : 2; }
+
+// ------------------------------------------------------------------ driver entry point
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// bf16 tensor map over `rank` dims (dims[0] innermost, contiguous), 128-byte
+// swizzle, zero fill outside the tensor.
+psa_status_t encode_bf16(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+                         const uint64_t* strides_bytes, const uint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(PSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t gd[5], gs[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) { gd[i] = dims[i]; bx[i] = box[i]; es[i] = 1; }
+  for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), gd, gs, bx, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return PSA_OK;
+}
+
+// [BH, rows, d] bf16 viewed as 3D {d, rows, BH}, box {64, box_rows, 1}
+psa_status_t map3(CUtensorMap* m, const void* base, int64_t BH, int64_t rows, int d, int box_rows) {
+  const uint64_t dims[3] = {static_cast<uint64_t>(d), static_cast<uint64_t>(rows), static_cast<uint64_t>(BH)};
+  const uint64_t str[2] = {static_cast<uint64_t>(d) * 2, static_cast<uint64_t>(rows) * d * 2};
+  const uint32_t box[3] = {64, static_cast<uint32_t>(box_rows), 1};
+  return encode_bf16(m, base, 3, dims, str, box);
+}
+
+// [BH, N, d] bf16 viewed as 4D {d, step, N/step, BH}, box {64, 1, 128, 1}:
+// one box row per `step` tokens starting at the chosen sub-row.
+psa_status_t map4(CUtensorMap* m, const void* base, int64_t BH, int64_t N, int d, int step) {
+  const uint64_t dims[4] = {static_cast<uint64_t>(d), static_cast<uint64_t>(step), static_cast<uint64_t>(N / step),
+                            static_cast<uint64_t>(BH)};
+  const uint64_t str[3] = {static_cast<uint64_t>(d) * 2, static_cast<uint64_t>(step) * d * 2,
+                           static_cast<uint64_t>(N) * d * 2};
+  const uint32_t box[4] = {64, 1, 128, 1};
+  return encode_bf16(m, base, 4, dims, str, box);
+}
+
+int num_sms() {
+  int dev = 0, n = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+// ------------------------------------------------------------------ validation
+psa_status_t check_shape(const psa_shape_t* s) {
+  if (!s) return fail(PSA_ERR_INVALID_ARG, "shape is NULL");
+  if (s->B < 1 || s->Hq < 1 || s->Hkv < 1 || s->N < 1 || s->d < 1 || s->block < 1 || s->levels < 1)
+    return fail(PSA_ERR_INVALID_ARG, "shape fields must be positive");
+  if (s->dtype != PSA_DT_BF16 && s->dtype != PSA_DT_FP32) return fail(PSA_ERR_INVALID_ARG, "unknown dtype %d", s->dtype);
+  if (s->d != 64 && s->d != 128) return fail(PSA_ERR_UNSUPPORTED, "head dim %d not in {64, 128}", s->d);
+  if (s->block != 64 && s->block != 128) return fail(PSA_ERR_UNSUPPORTED, "block %d not in {64, 128}", s->block);
+  if (s->levels > PSA_MAX_LEVELS) return fail(PSA_ERR_UNSUPPORTED, "levels %d > %d", s->levels, PSA_MAX_LEVELS);
+  const int g = 1 << (s->levels - 1);
+  if (s->block % g || s->N % g) return fail(PSA_ERR_UNSUPPORTED, "block and N must be multiples of 2^(L-1) = %d", g);
+  if (s->Hq % s->Hkv) return fail(PSA_ERR_UNSUPPORTED, "Hq %d not a multiple of Hkv %d", s->Hq, s->Hkv);
+  if (static_cast<int64_t>(s->B) * s->Hq * s->N * s->d >= (1ll << 31))
+    return fail(PSA_ERR_UNSUPPORTED, "B*Hq*N*d must be < 2^31");
+  if (ceil_div(s->N, s->block) > PSA_MAX_KV_BLOCKS) return fail(PSA_ERR_UNSUPPORTED, "more than %d KV blocks", PSA_MAX_KV_BLOCKS);
+  return PSA_OK;
+}
+
+psa_status_t check_ptr(const void* p, const char* name, bool required = true) {
+  if (!p) return required ? fail(PSA_ERR_INVALID_ARG, "%s is NULL", name) : PSA_OK;
+  if (!aligned16(p)) return fail(PSA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return PSA_OK;
+}
+
+#define PSA_TRY(x)                      \
+  do {                                  \
+    psa_status_t st__ = (x);            \
+    if (st__ != PSA_OK) return st__;    \
+  } while (0)
+#define PSA_CUDA(x, what)                              \
+  do {                                                 \
+    cudaError_t e__ = (x);                             \
+    if (e__ != cudaSuccess) return cuda_fail(e__, what); \
+  } while (0)
+
+// ------------------------------------------------------------------ pyramid layout
+size_t level_rows_total(const psa_shape_t* s, int upto) {   // sum over l in [1, upto) of N/2^l
+  size_t r = 0;
+  for (int l = 1; l < upto; ++l) r += static_cast<size_t>(s->N >> l);
+  return r;
+}
+size_t pyr_level_offset(const psa_shape_t* s, int level, size_t esize) {
+  return static_cast<size_t>(s->B) * s->Hkv * level_rows_total(s, level) * s->d * esize;
+}
+size_t pyr_bytes(const psa_shape_t* s, size_t esize) { return pyr_level_offset(s, s->levels, esize); }
+
+// ------------------------------------------------------------------ mask workspace
+struct MaskLayout {
+  size_t status, blocklse, rowlse, q16, k16, total;
+  int rows, step, rpb, cols, cpb;
+};
+MaskLayout mask_layout(const psa_shape_t* s, const psa_mask_params_t* p) {
+  MaskLayout L{};
+  const int nqb = static_cast<int>(ceil_div(s->N, s->block));
+  const int nkb = nqb;
+  if (p->mode == PSA_MASK_SAMPLE) {
+    L.step = s->block / 8;
+    L.rpb = 8;
+    L.rows = nqb * 8;
+    L.cols = s->N;
+    L.cpb = s->block;
+  } else {
+    L.step = p->stride;
+    L.rpb = s->block / p->stride;
+    L.rows = s->N / p->stride;
+    L.cols = s->N / p->stride;
+    L.cpb = s->block / p->stride;
+  }
+  const size_t BHq = static_cast<size_t>(s->B) * s->Hq;
+  size_t off = 256;
+  L.status = 0;
+  L.blocklse = off; off = align_up(off + BHq * nkb * L.rows * 4, 256);
+  L.rowlse = off;   off = align_up(off + BHq * L.rows * 4, 256);
+  if (s->dtype == PSA_DT_FP32) {
+    L.q16 = off; off = align_up(off + BHq * s->N * s->d * 2, 256);
+    L.k16 = off; off = align_up(off + static_cast<size_t>(s->B) * s->Hkv * s->N * s->d * 2, 256);
+  }
+  L.total = off;
+  return L;
+}
+
+psa_status_t check_mask_params(const psa_shape_t* s, const psa_mask_params_t* p) {
+  if (!p) return fail(PSA_ERR_INVALID_ARG, "params is NULL");
+  if (p->mode != PSA_MASK_SAMPLE && p->mode != PSA_MASK_ANTIDIAG) return fail(PSA_ERR_INVALID_ARG, "unknown mask mode %d", p->mode);
+  if (p->n_thresholds != s->levels) return fail(PSA_ERR_INVALID_ARG, "n_thresholds %d != levels %d", p->n_thresholds, s->levels);
+  for (int i = 0; i < p->n_thresholds; ++i)
+    if (!(p->thresholds[i] == p->thresholds[i])) return fail(PSA_ERR_INVALID_ARG, "threshold %d is NaN", i);
+  if (!(p->sm_scale > 0.f) || p->sm_scale != p->sm_scale) return fail(PSA_ERR_INVALID_ARG, "sm_scale must be > 0");
+  if (p->n_dense_prefix < 0) return fail(PSA_ERR_INVALID_ARG, "n_dense_prefix < 0");
+  if (p->mode == PSA_MASK_SAMPLE) {
+    if (p->n_samples != 8) return fail(PSA_ERR_UNSUPPORTED, "n_samples must be 8");
+    if (s->N % (s->block / 8)) return fail(PSA_ERR_UNSUPPORTED, "sampling needs N %% (block/8) == 0");
+  } else {
+    const int S = p->stride;
+    if (S != 1 && S != 2 && S != 4 && S != 8 && S != 16) return fail(PSA_ERR_UNSUPPORTED, "stride %d not in {1,2,4,8,16}", S);
+    if (s->N % S) return fail(PSA_ERR_UNSUPPORTED, "antidiagonal scoring needs N %% stride == 0");
+    if (s->block / S < 8) return fail(PSA_ERR_UNSUPPORTED, "block / stride must be >= 8");
+  }
+  return PSA_OK;
+}
+
+// ------------------------------------------------------------------ attention workspace
+struct AttnLayout {
+  size_t status, stats, nseg, ntile, nrows, seg_off, tile_off, hist, queue, tile_seg_off, segs;
+  size_t q16, k16, v16, kp16, vp16, total;
+  int n_items, n_qtiles, n_hist;
+  int64_t max_tiles, max_segs;
+};
+AttnLayout attn_layout(const psa_shape_t* s) {
+  AttnLayout L{};
+  const int nkb = static_cast<int>(ceil_div(s->N, s->block));
+  L.n_qtiles = static_cast<int>(ceil_div(s->N, 128));
+  L.n_items = s->B * s->Hq * L.n_qtiles;
+  L.n_hist = nkb + 2;
+  L.max_tiles = static_cast<int64_t>(L.n_items) * nkb;
+  const int per_level = s->block == 64 ? 2 * nkb : nkb;
+  L.max_segs = static_cast<int64_t>(L.n_items) * (per_level + s->levels);
+  const size_t n = static_cast<size_t>(L.n_items);
+  size_t off = 0;
+  L.status = off; L.stats = 16; off = 256;
+  L.nseg = off;     off = align_up(off + n * 4, 256);
+  L.ntile = off;    off = align_up(off + n * 4, 256);
+  L.nrows = off;    off = align_up(off + n * 4, 256);
+  L.seg_off = off;  off = align_up(off + (n + 1) * 4, 256);
+  L.tile_off = off; off = align_up(off + (n + 1) * 4, 256);
+  L.hist = off;     off = align_up(off + static_cast<size_t>(L.n_hist) * 4, 256);
+  L.queue = off;    off = align_up(off + n * 4, 256);
+  L.tile_seg_off = off; off = align_up(off + static_cast<size_t>(L.max_tiles + 1) * 4, 256);
+  L.segs = off;     off = align_up(off + static_cast<size_t>(L.max_segs) * 4, 256);
+  if (s->dtype == PSA_DT_FP32) {
+    const size_t qn = static_cast<size_t>(s->B) * s->Hq * s->N * s->d;
+    const size_t kn = static_cast<size_t>(s->B) * s->Hkv * s->N * s->d;
+    L.q16 = off;  off = align_up(off + qn * 2, 256);
+    L.k16 = off;  off = align_up(off + kn * 2, 256);
+    L.v16 = off;  off = align_up(off + kn * 2, 256);
+    L.kp16 = off; off = align_up(off + pyr_bytes(s, 2), 256);
+    L.vp16 = off; off = align_up(off + pyr_bytes(s, 2), 256);
+  }
+  L.total = off;
+  return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* psa_last_error(void) { return g_err; }
+int32_t psa_version(void) { return 100; }
+
+size_t psa_pyramid_bytes(const psa_shape_t* s) {
+  if (check_shape(s) != PSA_OK) return 0;
+  return pyr_bytes(s, elem_size(s->dtype));
+}
+
+size_t psa_pyramid_level_offset(const psa_shape_t* s, int level) {
+  if (check_shape(s) != PSA_OK || level < 1 || level >= s->levels) return 0;
+  return pyr_level_offset(s, level, elem_size(s->dtype));
+}
+
+psa_status_t psa_build_pyramid(const psa_shape_t* s, const void* k, const void* v, void* k_pyr, void* v_pyr,
+                               float* blockcos, void* stream) {
+  g_err[0] = 0;
+  PSA_TRY(check_shape(s));
+  PSA_TRY(check_ptr(k, "k"));
+  PSA_TRY(check_ptr(v, "v"));
+  if (s->levels > 1) {
+    PSA_TRY(check_ptr(k_pyr, "k_pyr"));
+    PSA_TRY(check_ptr(v_pyr, "v_pyr"));
+  }
+  PSA_TRY(check_ptr(blockcos, "blockcos", false));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t es = elem_size(s->dtype);
+  size_t off[PSA_MAX_LEVELS] = {0, 0, 0, 0};
+  for (int l = 1; l < s->levels; ++l) off[l] = pyr_level_offset(s, l, es);
+  const int64_t BH = static_cast<int64_t>(s->B) * s->Hkv;
+  PSA_CUDA(psa::launch_pyramid(k, v, k_pyr, v_pyr, BH, s->N, s->d, s->levels, static_cast<int>(es), off, st),
+           "pyramid launch");
+  if (blockcos) PSA_CUDA(psa::launch_blockcos(k, blockcos, BH, s->N, s->d, s->block, static_cast<int>(es), st), "blockcos launch");
+  return PSA_OK;
+}
+
+size_t psa_mask_workspace_bytes(const psa_shape_t* s, const psa_mask_params_t* p) {
+  if (check_shape(s) != PSA_OK || check_mask_params(s, p) != PSA_OK) return 0;
+  return mask_layout(s, p).total;
+}
+
+psa_status_t psa_make_mask(const psa_shape_t* s, const psa_mask_params_t* p, const void* q, const void* k,
+                           const float* blockcos, uint8_t* mask, float* mass_out, void* ws, size_t ws_bytes,
+                           void* stream) {
+  g_err[0] = 0;
+  PSA_TRY(check_shape(s));
+  PSA_TRY(check_mask_params(s, p));
+  PSA_TRY(check_ptr(q, "q"));
+  PSA_TRY(check_ptr(k, "k"));
+  if (!mask) return fail(PSA_ERR_INVALID_ARG, "mask is NULL");
+  PSA_TRY(check_ptr(mass_out, "mass_out", false));
+  if (p->cos_min > -2.f) PSA_TRY(check_ptr(blockcos, "blockcos (required when cos_min > -2)"));
+  const MaskLayout L = mask_layout(s, p);
+  if (!ws || !aligned16(ws)) return fail(PSA_ERR_WORKSPACE, "workspace is NULL or not 16-byte aligned");
+  if (ws_bytes < L.total) return fail(PSA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, L.total);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  const int64_t BHq = static_cast<int64_t>(s->B) * s->Hq, BHkv = static_cast<int64_t>(s->B) * s->Hkv;
+  const void* q16 = q;
+  const void* k16 = k;
+  if (s->dtype == PSA_DT_FP32) {
+    PSA_CUDA(psa::launch_cast_bf16(static_cast<const float*>(q), w + L.q16, BHq * s->N * s->d, st), "cast q");
+    PSA_CUDA(psa::launch_cast_bf16(static_cast<const float*>(k), w + L.k16, BHkv * s->N * s->d, st), "cast k");
+    q16 = w + L.q16;
+    k16 = w + L.k16;
+  }
+  CUtensorMap mA, mB;
+  PSA_TRY(map4(&mA, q16, BHq, s->N, s->d, L.step));
+  PSA_TRY(map4(&mB, k16, BHkv, s->N, s->d, p->mode == PSA_MASK_SAMPLE ? 1 : p->stride));
+  psa::ScoreArgs sa{};
+  const int nkb = static_cast<int>(ceil_div(s->N, s->block));
+  sa.BHq = static_cast<int>(BHq); sa.Hq = s->Hq; sa.Hkv = s->Hkv; sa.N = s->N; sa.d = s->d;
+  sa.block = s->block; sa.nkb = nkb; sa.mode = p->mode; sa.step = L.step;
+  sa.S = p->mode == PSA_MASK_SAMPLE ? 1 : p->stride;
+  sa.rows = L.rows; sa.cols = L.cols; sa.rows_per_block = L.rpb; sa.cols_per_block = L.cpb;
+  sa.causal = s->causal != 0;
+  const float sc = p->mode == PSA_MASK_SAMPLE ? p->sm_scale : p->sm_scale / static_cast<float>(p->stride);
+  sa.scale_log2 = sc * 1.4426950408889634f;
+  sa.blocklse = reinterpret_cast<float*>(w + L.blocklse);
+  sa.rowlse = reinterpret_cast<float*>(w + L.rowlse);
+  sa.status = reinterpret_cast<int*>(w + L.status);
+  PSA_CUDA(psa::launch_score(&mA, &mB, sa, num_sms(), st), "score launch");
+  psa::SelectArgs se{};
+  se.B = s->B; se.Hq = s->Hq; se.Hkv = s->Hkv; se.N = s->N; se.block = s->block;
+  se.nqb = nkb; se.nkb = nkb; se.levels = s->levels; se.causal = s->causal != 0;
+  se.mode = p->mode; se.S = sa.S; se.rows = L.rows; se.rows_per_block = L.rpb; se.step = L.step;
+  for (int i = 0; i < 8; ++i) se.thresholds[i] = i < p->n_thresholds ? p->thresholds[i] : 3.0e38f;
+  se.cos_min = p->cos_min;
+  se.n_dense_prefix = p->n_dense_prefix;
+  se.blocklse = sa.blocklse;
+  se.rowlse = sa.rowlse;
+  se.blockcos = p->cos_min > -2.f ? blockcos : nullptr;
+  se.mask = mask;
+  se.mass_out = mass_out;
+  PSA_CUDA(psa::launch_select(se, st), "select launch");
+  return PSA_OK;
+}
+
+size_t psa_attention_workspace_bytes(const psa_shape_t* s) {
+  if (check_shape(s) != PSA_OK) return 0;
+  return attn_layout(s).total;
+}
+
+psa_status_t psa_attention_fwd(const psa_shape_t* s, const void* q, const void* k, const void* v, const void* k_pyr,
+                               const void* v_pyr, const uint8_t* mask, float sm_scale, void* out, float* lse,
+                               void* ws, size_t ws_bytes, void* stream) {
+  g_err[0] = 0;
+  PSA_TRY(check_shape(s));
+  PSA_TRY(check_ptr(q, "q"));
+  PSA_TRY(check_ptr(k, "k"));
+  PSA_TRY(check_ptr(v, "v"));
+  PSA_TRY(check_ptr(out, "out"));
+  if (s->levels > 1) {
+    PSA_TRY(check_ptr(k_pyr, "k_pyr"));
+    PSA_TRY(check_ptr(v_pyr, "v_pyr"));
+  }
+  if (!mask) return fail(PSA_ERR_INVALID_ARG, "mask is NULL");
+  PSA_TRY(check_ptr(lse, "lse", false));
+  if (!(sm_scale > 0.f) || sm_scale != sm_scale) return fail(PSA_ERR_INVALID_ARG, "sm_scale must be > 0");
+  const AttnLayout L = attn_layout(s);
+  if (L.max_segs >= (1ll << 31) || L.max_tiles >= (1ll << 31))
+    return fail(PSA_ERR_UNSUPPORTED, "tile plan would exceed 2^31 entries");
+  if (!ws || !aligned16(ws)) return fail(PSA_ERR_WORKSPACE, "workspace is NULL or not 16-byte aligned");
+  if (ws_bytes < L.total) return fail(PSA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, L.total);
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  const int64_t BHq = static_cast<int64_t>(s->B) * s->Hq, BHkv = static_cast<int64_t>(s->B) * s->Hkv;
+  const void* q16 = q;
+  const void* k16 = k;
+  const void* v16 = v;
+  const char* kp16 = static_cast<const char*>(k_pyr);
+  const char* vp16 = static_cast<const char*>(v_pyr);
+  if (s->dtype == PSA_DT_FP32) {
+    PSA_CUDA(psa::launch_cast_bf16(static_cast<const float*>(q), w + L.q16, BHq * s->N * s->d, st), "cast q");
+    PSA_CUDA(psa::launch_cast_bf16(static_cast<const float*>(k), w + L.k16, BHkv * s->N * s->d, st), "cast k");
+    PSA_CUDA(psa::launch_cast_bf16(static_cast<const float*>(v), w + L.v16, BHkv * s->N * s->d, st), "cast v");
+    const int64_t pn = static_cast<int64_t>(pyr_bytes(s, 4) / 4);
+    if (pn > 0) {
+      PSA_CUDA(psa::launch_cast_bf16(static_cast<const float*>(k_pyr), w + L.kp16, pn, st), "cast k_pyr");
+      PSA_CUDA(psa::launch_cast_bf16(static_cast<const float*>(v_pyr), w + L.vp16, pn, st), "cast v_pyr");
+    }
+    q16 = w + L.q16; k16 = w + L.k16; v16 = w + L.v16;
+    kp16 = w + L.kp16; vp16 = w + L.vp16;
+  }
+  CUtensorMap maps[9];
+  PSA_TRY(map3(&maps[0], q16, BHq, s->N, s->d, 128));
+  for (int l = 0; l < s->levels; ++l) {
+    const void* kb = l == 0 ? k16 : static_cast<const void*>(kp16 + pyr_level_offset(s, l, 2));
+    const void* vb = l == 0 ? v16 : static_cast<const void*>(vp16 + pyr_level_offset(s, l, 2));
+    PSA_TRY(map3(&maps[1 + l], kb, BHkv, s->N >> l, s->d, s->block >> l));
+    PSA_TRY(map3(&maps[1 + s->levels + l], vb, BHkv, s->N >> l, s->d, s->block >> l));
+  }
+  const int nkb = static_cast<int>(ceil_div(s->N, s->block));
+  psa::PlanArgs pa{};
+  pa.B = s->B; pa.Hq = s->Hq; pa.N = s->N; pa.block = s->block; pa.nqb = nkb; pa.nkb = nkb;
+  pa.levels = s->levels; pa.causal = s->causal != 0; pa.n_items = L.n_items; pa.mask = mask;
+  pa.item_nseg = reinterpret_cast<int*>(w + L.nseg);
+  pa.item_ntile = reinterpret_cast<int*>(w + L.ntile);
+  pa.item_rows = reinterpret_cast<int*>(w + L.nrows);
+  pa.item_seg_off = reinterpret_cast<int*>(w + L.seg_off);
+  pa.item_tile_off = reinterpret_cast<int*>(w + L.tile_off);
+  pa.tile_seg_off = reinterpret_cast<int*>(w + L.tile_seg_off);
+  pa.segs = reinterpret_cast<int*>(w + L.segs);
+  pa.queue = reinterpret_cast<int*>(w + L.queue);
+  pa.hist = reinterpret_cast<int*>(w + L.hist);
+  pa.n_hist = L.n_hist;
+  pa.stats = reinterpret_cast<long long*>(w + L.stats);
+  PSA_CUDA(psa::launch_plan(pa, st), "plan launch");
+
+  psa::AttnArgs aa{};
+  aa.B = s->B; aa.Hq = s->Hq; aa.Hkv = s->Hkv; aa.N = s->N; aa.d = s->d; aa.block = s->block;
+  aa.levels = s->levels; aa.causal = s->causal != 0; aa.n_items = L.n_items; aa.n_qtiles = L.n_qtiles;
+  aa.scale_log2 = sm_scale * 1.4426950408889634f;
+  aa.item_tile_off = pa.item_tile_off;
+  aa.tile_seg_off = pa.tile_seg_off;
+  aa.segs = pa.segs;
+  aa.queue = pa.queue;
+  aa.out = out;
+  aa.out_fp32 = s->dtype == PSA_DT_FP32;
+  aa.lse = lse;
+  aa.status = reinterpret_cast<int*>(w + L.status);
+  PSA_CUDA(psa::launch_attention(maps, aa, num_sms(), st), "attention launch");
+  return PSA_OK;
+}
+
+psa_status_t psa_attention_plan_stats(const psa_shape_t* s, const void* ws, int64_t* n_tiles, int64_t* n_rows,
+                                      void* stream) {
+  g_err[0] = 0;
+  PSA_TRY(check_shape(s));
+  if (!ws || !n_tiles || !n_rows) return fail(PSA_ERR_INVALID_ARG, "NULL argument");
+  const AttnLayout L = attn_layout(s);
+  long long st[2] = {0, 0};
+  cudaStream_t str = static_cast<cudaStream_t>(stream);
+  PSA_CUDA(cudaMemcpyAsync(st, static_cast<const char*>(ws) + L.stats, sizeof(st), cudaMemcpyDeviceToHost, str), "stats copy");
+  PSA_CUDA(cudaStreamSynchronize(str), "stats sync");
+  *n_tiles = st[0];
+  *n_rows = st[1];
+  return PSA_OK;
+}
+
+psa_status_t psa_get_device_status(void* ws, void* stream) {
+  g_err[0] = 0;
+  if (!ws) return fail(PSA_ERR_INVALID_ARG, "workspace is NULL");
+  int word = 0;
+  cudaStream_t str = static_cast<cudaStream_t>(stream);
+  PSA_CUDA(cudaMemcpyAsync(&word, ws, sizeof(int), cudaMemcpyDeviceToHost, str), "status copy");
+  PSA_CUDA(cudaMemsetAsync(ws, 0, sizeof(int), str), "status clear");
+  PSA_CUDA(cudaStreamSynchronize(str), "status sync");
+  if (word == 0) return PSA_OK;
+  return fail(static_cast<psa_status_t>(word), "device status word %d (a bounded wait ran out)", word);
+}
+
+}  // extern "C"

@@ -1,0 +1,102 @@
+// internal.h -- declarations shared by the PSA library's translation units.
+// Not part of the public ABI (include/psa.h is).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/psa.h"
+
+namespace psa {
+
+// ---- stage 1 -------------------------------------------------------------
+// Pools K and V ([BH, N, d], elem = 2 (bf16) or 4 (fp32)) into levels
+// 1..L-1 written at the given byte offsets of k_pyr / v_pyr.
+cudaError_t launch_pyramid(const void* k, const void* v, void* k_pyr, void* v_pyr, int64_t BH,
+                           int N, int d, int levels, int elem, const size_t* level_off,
+                           cudaStream_t s);
+cudaError_t launch_blockcos(const void* k, float* out, int64_t BH, int N, int d, int block,
+                            int elem, cudaStream_t s);
+cudaError_t launch_cast_bf16(const float* src, void* dst, int64_t n, cudaStream_t s);
+
+// ---- stage 2 -------------------------------------------------------------
+struct ScoreArgs {
+  int BHq, Hq, Hkv, N, d, block, nkb;
+  int mode;            // 0 sampling, 1 antidiagonal
+  int step;            // token distance between rows of the A view (block/8 or S)
+  int S;               // antidiagonal stride (1 for sampling)
+  int rows;            // score rows per head (nqb*8 or N/S)
+  int cols;            // score columns per head (N or N/S)
+  int rows_per_block;  // 8 (sampling) or block/S
+  int cols_per_block;  // block (sampling) or block/S
+  int causal;
+  float scale_log2;    // softmax scale * log2(e)
+  float* blocklse;     // [BHq][nkb][rows]  log2-domain logsumexp of each block
+  float* rowlse;       // [BHq][rows]
+  int* status;
+};
+cudaError_t launch_score(const CUtensorMap* mapA, const CUtensorMap* mapB, const ScoreArgs& a,
+                         int num_sms, cudaStream_t s);
+
+struct SelectArgs {
+  int B, Hq, Hkv, N, block, nqb, nkb, levels, causal;
+  int mode, S, rows, rows_per_block, step;
+  float thresholds[8];
+  float cos_min;
+  int n_dense_prefix;
+  const float* blocklse;
+  const float* rowlse;
+  const float* blockcos;
+  uint8_t* mask;
+  float* mass_out;
+};
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t s);
+
+// ---- stage 3 -------------------------------------------------------------
+struct PlanArgs {
+  int B, Hq, N, block, nqb, nkb, levels, causal;
+  int n_items;           // query tiles of 128 rows: B*Hq*ceil(N/128)
+  const uint8_t* mask;
+  int* item_nseg;        // [n_items]   segments per item (pads included)
+  int* item_ntile;       // [n_items]
+  int* item_rows;        // [n_items]   real (non-padding) KV rows per item
+  int* item_seg_off;     // [n_items+1]
+  int* item_tile_off;    // [n_items+1]
+  int* tile_seg_off;     // [max_tiles+1]
+  int* segs;             // [max_segs]
+  int* queue;            // [n_items]  item ids, most tiles first
+  int* hist;             // [n_hist]   scratch for the counting sort
+  int n_hist;
+  long long* stats;      // [2] tiles, real kv rows
+};
+cudaError_t launch_plan(const PlanArgs& a, cudaStream_t s);
+
+struct AttnArgs {
+  int B, Hq, Hkv, N, d, block, levels, causal;
+  int n_items, n_qtiles;  // n_qtiles = ceil(N/128) per head
+  float scale_log2;       // sm_scale * log2(e)
+  const int* item_tile_off;
+  const int* tile_seg_off;
+  const int* segs;
+  const int* queue;
+  void* out;              // [B,Hq,N,d] bf16 or fp32
+  int out_fp32;
+  float* lse;             // [B,Hq,N] or null
+  int* status;
+};
+// maps: [0] = Q (3D view [d, N, B*Hq], box 64 x 128), [1 + l] = K level l,
+// [1 + L + l] = V level l (3D views [d, N/2^l, B*Hkv], box 64 x block/2^l).
+cudaError_t launch_attention(const CUtensorMap* maps, const AttnArgs& a, int num_sms,
+                             cudaStream_t s);
+
+// Segment word of the tile plan: bits [0,2) level, [2,4) half mask (bit 0:
+// query rows 0..63 of the tile use it, bit 1: rows 64..127; 0 marks a
+// padding segment of zeros), [4,32) KV block index.
+__host__ __device__ inline int seg_level(int w) { return w & 3; }
+__host__ __device__ inline int seg_half(int w) { return (w >> 2) & 3; }
+__host__ __device__ inline int seg_block(int w) { return w >> 4; }
+__host__ __device__ inline int make_seg(int J, int l, int half) { return (J << 4) | (half << 2) | l; }
+
+}  // namespace psa
