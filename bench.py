@@ -170,20 +170,41 @@ class Path:
 
 # ----------------------------------------------------------------------------- psa arm
 
+T0 = time.time()
+
+
+def log(args, msg):
+    if args.verbose:
+        sys.stderr.write("[bench %7.2fs] %s\n" % (time.time() - T0, msg))
+        sys.stderr.flush()
+
+
 def run_psa(args, rank, world, local_rank):
     import video_transformers_b200 as P
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w = W.PRESETS[args.config]
+    log(args, "generating %s inputs" % w.name)
     q, k, v, gen = W.make_qkv(w, device=dev, seed=w.seed + rank)
+    torch.cuda.synchronize()
+    log(args, "inputs ready")
     path = Path(w, q, k, v)
     if w.mask_mode == "given":
         path.given_mask = W.make_given_mask(w, gen, device=dev)
     stream = torch.cuda.current_stream()
 
     # warm-up, and the executed work of one step (the mask is deterministic)
-    for _ in range(args.warmup):
-        path.step()
+    for i in range(args.warmup):
+        if args.verbose:
+            for name, fn in (("pyramid", path.pyramid), ("mask", path.make_mask), ("attention", path.attention)):
+                t = time.time()
+                fn()
+                torch.cuda.synchronize()
+                log(args, "warm-up %d %s %.3f s status %d/%d" % (i, name, time.time() - t,
+                                                                P.psa_get_device_status(path.mws),
+                                                                P.psa_get_device_status(path.aws)))
+        else:
+            path.step()
     torch.cuda.synchronize()
     flops = executed_flops(path.mask, w.N, w.block, w.d, w.levels, w.causal)
     dense = W.dense_flops(w)
@@ -396,6 +417,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--verbose", action="store_true", help="progress and per-stage warm-up times on stderr")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

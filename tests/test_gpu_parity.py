@@ -106,8 +106,8 @@ def check_mask(w, q, k, rows=None):
 
 
 @pytest.mark.parametrize("name,grid,heads,n_text", [
-    ("wan1.3b", (3, 10, 13), (2, 2), None),          # N = 390: ragged last block of 6
-    ("cogvideox5b", (3, 10, 15), (3, 3), 26),         # text prefix, N = 476
+    ("wan1.3b", (3, 10, 12), (2, 2), None),          # N = 360: ragged last block of 40
+    ("cogvideox5b", (3, 10, 15), (3, 3), 30),         # text prefix, N = 480: ragged last block of 32
     ("wan14b", (4, 12, 16), (2, 2), None),           # block 128, N = 768
     ("wan14b", (3, 9, 16), (2, 2), None),            # N = 432: ragged
 ])
@@ -187,8 +187,8 @@ def test_attention_tiny_given_mask():
 
 
 @pytest.mark.parametrize("name,grid,heads,n_text", [
-    ("wan1.3b", (3, 10, 13), (2, 2), None),
-    ("cogvideox5b", (3, 10, 15), (2, 2), 26),
+    ("wan1.3b", (3, 10, 12), (2, 2), None),
+    ("cogvideox5b", (3, 10, 15), (2, 2), 30),
     ("qwen2.5vl", (6, 8, 16), (7, 1), None),
     ("wan14b", (4, 12, 16), (2, 2), None),
     ("wan14b", (3, 9, 16), (2, 2), None),

@@ -208,4 +208,5 @@ def pyramid_level(shape: Shape, buf: torch.Tensor, level: int) -> torch.Tensor:
 
 def workspace(nbytes: int, device) -> torch.Tensor:
     """A zero-filled workspace (the status word must start at 0)."""
-    return torch.zeros(max(1, (nbytes + 15) // 16), dtype=torch.int64, device=device).view(torch.uint8)[:max(nbytes, 16)]
+    n16 = max(1, (nbytes + 15) // 16)
+    return torch.zeros(2 * n16, dtype=torch.int64, device=device).view(torch.uint8)[:max(nbytes, 16)]
