@@ -302,3 +302,26 @@ def test_attention_plan_stats_and_status():
     # 4 query tiles of two 64-row blocks: both halves agree -> one 64-row and one 8-row segment
     assert nr == 4 * (64 + 8) and nt == 4
     assert P.psa_get_device_status(ws) == P.PSA_OK
+
+
+@pytest.mark.parametrize("d,block", [(128, 128), (64, 64)])
+def test_attention_many_items_per_cta_with_rescale(d, block):
+    """More query tiles than SMs (every CTA of the persistent grid takes
+    several items), and keys of the late KV blocks scaled up so the running
+    max of some rows of a warp jumps by more than the lazy-rescale threshold
+    while others do not."""
+    g = gen(71)
+    H, N = 40, 1024
+    q, k, v = randn(g, 1, H, N, d), randn(g, 1, H, N, d), randn(g, 1, H, N, d)
+    k[:, :, N // 2:] *= 6.0
+    nb = N // block
+    m = torch.randint(0, 5, (1, H, nb, nb), generator=g)
+    mask = torch.where(m == 4, torch.full_like(m, SKIP), m).to(torch.uint8)
+    mask[:, :, :, nb - 1] = 0
+    w = W.Workload("many", B=1, Hq=H, Hkv=H, d=d, block=block, levels=4, causal=False, dtype="bf16",
+                   recipe="iid", n_iid=N)
+    shape = shape_for(w)
+    kp, vp, _ = run_pyramid(shape, k, v)
+    out, lse, _ = run_attention(shape, q, k, v, kp, vp, mask.to(DEV), w.sm_scale)
+    rows = [(0, h, I) for h in range(0, H, 7) for I in range(nb)]
+    assert_attn(w, q, k, v, kp, vp, mask, out, lse, rows=rows)

@@ -166,17 +166,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // drain: wait for every TMA this warp issued before the CTA may exit
     if (lane == 0) {
-      const uint64_t t0 = globaltimer();
-      if (qcnt > 0) {
-        while (!mbar_try_wait(smem_u32(&sh->q_full), (qcnt - 1) & 1))
-          if (globaltimer() - t0 > kWaitLimitNs) { atomicExch(a.status, kDevTimeout); break; }
-      }
+      if (qcnt > 0) drain_wait(smem_u32(&sh->q_full), (qcnt - 1) & 1, a.status);
       for (uint32_t st = 0; st < NST; ++st) {
-        if (kv_it > st) {
-          const uint32_t n = (kv_it - 1 - st) / NST;
-          while (!mbar_try_wait(smem_u32(&sh->kv_full[st]), n & 1))
-            if (globaltimer() - t0 > kWaitLimitNs) { atomicExch(a.status, kDevTimeout); break; }
-        }
+        if (kv_it > st) drain_wait(smem_u32(&sh->kv_full[st]), ((kv_it - 1 - st) / NST) & 1, a.status);
       }
     }
   } else if (warp == 1) {
@@ -241,9 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++icnt;
       }
       umma_commit(smem_u32(&sh->drain));
-      const uint64_t t0 = globaltimer();
-      while (!mbar_try_wait(smem_u32(&sh->drain), 0))
-        if (globaltimer() - t0 > kWaitLimitNs) { atomicExch(a.status, kDevTimeout); break; }
+      drain_wait(smem_u32(&sh->drain), 0, a.status);
     }
   } else {
     // =============================== softmax ===============================
@@ -301,24 +291,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 1; c < 128; ++c) mt = fmaxf(mt, s[c]);
         const float mnew = fmaxf(m, mt);
-        if (mnew > m + kRescaleThreshold || (m == -CUDART_INF_F && mnew != -CUDART_INF_F)) {
-          if (m != -CUDART_INF_F) {
-            const float f = fast_exp2(m - mnew);
-            lsum *= f;
-            // O holds tiles 0..j-1: wait for the PV of tile j-1, then scale it
-            if (!warp_wait(smem_u32(&sh->o_ready), (pv - 1) & 1, abort, a.status)) { ok = false; break; }
-            tc_fence_after();
+        // Lazy rescaling: a row moves its reference max only when the new max
+        // exceeds it by more than kRescaleThreshold (or on its first visible
+        // key).  O lives in TMEM and is read/written with warp-collective
+        // tcgen05.ld/st, so the decision to touch O is taken per warp.
+        const bool first = m == -CUDART_INF_F && mnew != -CUDART_INF_F;
+        const bool grow = m != -CUDART_INF_F && mnew > m + kRescaleThreshold;
+        if (__any_sync(0xffffffffu, grow)) {
+          const float f = grow ? fast_exp2(m - mnew) : 1.0f;
+          lsum *= f;
+          if (grow) m = mnew;
+          // O holds tiles 0..j-1: wait for the PV of tile j-1, then scale it
+          if (!warp_wait(smem_u32(&sh->o_ready), (pv - 1) & 1, abort, a.status)) { ok = false; break; }
+          tc_fence_after();
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t o[32];
-              tmem_ld32(tmem + 256 + c * 32 + lane_off, o);
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tmem + 256 + c * 32 + lane_off, o);
 #pragma unroll
-              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
-              tmem_st32(tmem + 256 + c * 32 + lane_off, o);
-            }
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+            tmem_st32(tmem + 256 + c * 32 + lane_off, o);
           }
-          m = mnew;
         }
+        if (first) m = mnew;
         const float mu = m == -CUDART_INF_F ? 0.f : m;
         float ps = 0.f;
         uint32_t pk[64];
@@ -336,7 +331,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(smem_u32(&sh->p_full[buf]));
       }
       if (!ok) break;
-      // epilogue: O / l
+      // epilogue: O / l.  Wait for the PVs of the last two tiles in order (the
+      // parity of a phase two behind would alias the one awaited).
+      if (n >= 2 && !warp_wait(smem_u32(&sh->o_ready), (pv - 2) & 1, abort, a.status)) { ok = false; break; }
       if (!warp_wait(smem_u32(&sh->o_ready), (pv - 1) & 1, abort, a.status)) { ok = false; break; }
       tc_fence_after();
       const float inv = lsum > 0.f ? 1.0f / lsum : 0.f;
@@ -375,7 +372,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 512);
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, 512);
+  }
 }
 
 template <int D, bool F32>

@@ -109,15 +109,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // drain: every armed stage must have landed before the CTA exits
-      const uint32_t armed = it;
-      for (int st = 0; st < kStages; ++st) {
-        if (armed > static_cast<uint32_t>(st)) {
-          const uint32_t n = (armed - 1 - st) / kStages;   // last use index of this stage
-          const uint64_t t0 = globaltimer();
-          while (!mbar_try_wait(smem_u32(&sh->full[st]), n & 1)) {
-            if (globaltimer() - t0 > kWaitLimitNs) { atomicExch(a.status, kDevTimeout); break; }
-          }
-        }
+      for (uint32_t st = 0; st < static_cast<uint32_t>(kStages); ++st) {
+        if (it > st) drain_wait(smem_u32(&sh->full[st]), ((it - 1 - st) / kStages) & 1, a.status);
       }
     }
   } else if (warp == 1) {
@@ -152,10 +145,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       umma_commit(smem_u32(&sh->drain));
-      const uint64_t t0 = globaltimer();
-      while (!mbar_try_wait(smem_u32(&sh->drain), 0)) {
-        if (globaltimer() - t0 > kWaitLimitNs) { atomicExch(a.status, kDevTimeout); break; }
-      }
+      drain_wait(smem_u32(&sh->drain), 0, a.status);
     }
   } else {
     // ---------------- epilogue: per (row, block) log-sum-exp ----------------
@@ -225,7 +215,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 256);
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, 256);
+  }
 }
 
 // ----------------------------------------------------------------------------

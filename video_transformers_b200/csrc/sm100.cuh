@@ -15,8 +15,10 @@ namespace psa {
 
 // Status word codes written into the workspace (match psa_status_t).
 constexpr int kDevTimeout = 5;
-// A bounded wait gives up after this many nanoseconds of %globaltimer.
+// A bounded wait gives up after this many nanoseconds of %globaltimer, or
+// after kWaitLimitIters polls, whichever comes first.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr uint32_t kWaitLimitIters = 1u << 26;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -66,11 +68,22 @@ __device__ __forceinline__ bool bounded_wait(uint32_t bar, uint32_t parity, vola
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 31u) == 0) {
       if (*abort) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
+      if (globaltimer() - t0 > kWaitLimitNs || i >= kWaitLimitIters) {
         *abort = 1;
         atomicExch(status, kDevTimeout);
         return false;
       }
+    }
+  }
+}
+
+// Wait used while a CTA winds down: no abort flag, same two limits.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, int* status) {
+  const uint64_t t0 = globaltimer();
+  for (uint32_t i = 0; !mbar_try_wait(bar, parity); ++i) {
+    if (globaltimer() - t0 > kWaitLimitNs || i >= kWaitLimitIters) {
+      atomicExch(status, kDevTimeout);
+      return;
     }
   }
 }
