@@ -200,9 +200,11 @@ def run_psa(args, rank, world, local_rank):
                 t = time.time()
                 fn()
                 torch.cuda.synchronize()
-                log(args, "warm-up %d %s %.3f s status %d/%d" % (i, name, time.time() - t,
-                                                                P.psa_get_device_status(path.mws),
-                                                                P.psa_get_device_status(path.aws)))
+                sm, sa = P.psa_get_device_status(path.mws), None
+                msg = P.psa_last_error() if sm else ""
+                sa = P.psa_get_device_status(path.aws)
+                msg += P.psa_last_error() if sa else ""
+                log(args, "warm-up %d %s %.3f s status %d/%d %s" % (i, name, time.time() - t, sm, sa, msg))
         else:
             path.step()
     torch.cuda.synchronize()

@@ -180,7 +180,10 @@ PSA_API psa_status_t psa_attention_plan_stats(const psa_shape_t* shape, const vo
 
 /* Reads the device status word of a workspace (synchronising on `stream`)
  * and clears it: PSA_OK, or PSA_ERR_TIMEOUT if a bounded wait ran out in a
- * kernel that used this workspace since the last read. */
+ * kernel that used this workspace since the last read.  On a time-out,
+ * psa_last_error() names the wait that gave up first (its site number, CTA,
+ * thread and progress counters).  The status word and that record occupy
+ * the first 36 bytes of every workspace. */
 PSA_API psa_status_t psa_get_device_status(void* workspace, void* stream);
 
 /* Message of the last failed call on this thread ("" if none). */

@@ -210,7 +210,7 @@ AttnLayout attn_layout(const psa_shape_t* s) {
   L.max_segs = static_cast<int64_t>(L.n_items) * (per_level + s->levels);
   const size_t n = static_cast<size_t>(L.n_items);
   size_t off = 0;
-  L.status = off; L.stats = 16; off = 256;
+  L.status = off; L.stats = 64; off = 256;   // [0, 36): status word + time-out record
   L.nseg = off;     off = align_up(off + n * 4, 256);
   L.ntile = off;    off = align_up(off + n * 4, 256);
   L.nrows = off;    off = align_up(off + n * 4, 256);
@@ -440,13 +440,15 @@ psa_status_t psa_attention_plan_stats(const psa_shape_t* s, const void* ws, int6
 psa_status_t psa_get_device_status(void* ws, void* stream) {
   g_err[0] = 0;
   if (!ws) return fail(PSA_ERR_INVALID_ARG, "workspace is NULL");
-  int word = 0;
+  int w[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
   cudaStream_t str = static_cast<cudaStream_t>(stream);
-  PSA_CUDA(cudaMemcpyAsync(&word, ws, sizeof(int), cudaMemcpyDeviceToHost, str), "status copy");
-  PSA_CUDA(cudaMemsetAsync(ws, 0, sizeof(int), str), "status clear");
+  PSA_CUDA(cudaMemcpyAsync(w, ws, sizeof(w), cudaMemcpyDeviceToHost, str), "status copy");
+  PSA_CUDA(cudaMemsetAsync(ws, 0, sizeof(w), str), "status clear");
   PSA_CUDA(cudaStreamSynchronize(str), "status sync");
-  if (word == 0) return PSA_OK;
-  return fail(static_cast<psa_status_t>(word), "device status word %d (a bounded wait ran out)", word);
+  if (w[0] == 0) return PSA_OK;
+  return fail(static_cast<psa_status_t>(w[0]),
+              "device status %d: a bounded wait ran out (site %d, block %d, thread %d, counters %d %d %d %d)",
+              w[0], w[2], w[3], w[4], w[5], w[6], w[7], w[8]);
 }
 
 }  // extern "C"

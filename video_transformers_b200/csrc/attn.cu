@@ -107,7 +107,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int b = bh / a.Hq, h = bh - b * a.Hq;
       const int hkv = b * a.Hkv + h / (a.Hq / a.Hkv);
       const int q0 = tq * 128;
-      if (!warp_wait(smem_u32(&sh->q_empty), (qcnt & 1) ^ 1, abort, a.status)) { ok = false; break; }
+      if (!warp_wait(smem_u32(&sh->q_empty), (qcnt & 1) ^ 1, abort, a.status, 11, idx, qcnt, kv_it, 0)) { ok = false; break; }
       if (lane == 0) {
         const uint32_t bar = smem_u32(&sh->q_full);
         mbar_arrive_expect_tx(bar, QB);
@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++qcnt;
       for (int t = t0; t < t1; ++t, ++kv_it) {
         const int st = kv_it % NST;
-        if (!warp_wait(smem_u32(&sh->kv_empty[st]), ((kv_it / NST) & 1) ^ 1, abort, a.status)) { ok = false; break; }
+        if (!warp_wait(smem_u32(&sh->kv_empty[st]), ((kv_it / NST) & 1) ^ 1, abort, a.status, 12, idx, t - t0, kv_it, 0)) { ok = false; break; }
         const int sb = a.tile_seg_off[t], se = a.tile_seg_off[t + 1];
         const uint32_t bar = smem_u32(&sh->kv_full[st]);
         if (lane == 0) {
@@ -183,9 +183,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t st = (kv_it + jj) % NST;
         const uint32_t buf = (T + jj) & 1;
         if (first_of_item && icnt > 0) {
-          if (!bounded_wait(smem_u32(&sh->o_free), (icnt - 1) & 1, abort, a.status)) return false;
+          if (!bounded_wait(smem_u32(&sh->o_free), (icnt - 1) & 1, abort, a.status, 21, icnt, jj, T, kv_it)) return false;
         }
-        if (!bounded_wait(smem_u32(&sh->p_full[buf]), ((T + jj) >> 1) & 1, abort, a.status)) return false;
+        if (!bounded_wait(smem_u32(&sh->p_full[buf]), ((T + jj) >> 1) & 1, abort, a.status, 22, icnt, jj, T, kv_it)) return false;
         tc_fence_after();
         const uint32_t sV_st = smem_u32(sV + st * QB);
 #pragma unroll
@@ -202,14 +202,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int t0 = a.item_tile_off[item], t1 = a.item_tile_off[item + 1];
         const uint32_t n = static_cast<uint32_t>(t1 - t0);
         if (n == 0) continue;
-        if (!bounded_wait(smem_u32(&sh->q_full), qcnt & 1, abort, a.status)) { ok = false; break; }
+        if (!bounded_wait(smem_u32(&sh->q_full), qcnt & 1, abort, a.status, 23, idx, qcnt, T, kv_it)) { ok = false; break; }
         tc_fence_after();
         ++qcnt;
         const uint32_t sQb = smem_u32(sQ);
         for (uint32_t j = 0; j < n && ok; ++j) {
           const uint32_t st = (kv_it + j) % NST;
           const uint32_t buf = (T + j) & 1;
-          if (!bounded_wait(smem_u32(&sh->kv_full[st]), ((kv_it + j) / NST) & 1, abort, a.status)) { ok = false; break; }
+          if (!bounded_wait(smem_u32(&sh->kv_full[st]), ((kv_it + j) / NST) & 1, abort, a.status, 24, idx, j, T, kv_it)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sK_st = smem_u32(sK + st * QB);
 #pragma unroll
@@ -267,8 +267,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < n; ++j, ++kv_it, ++T, ++pv) {
         const int st = kv_it % NST;
         const int buf = T & 1;
-        if (!warp_wait(smem_u32(&sh->s_full[buf]), (T >> 1) & 1, abort, a.status)) { ok = false; break; }
-        if (!warp_wait(smem_u32(&sh->kv_full[st]), (kv_it / NST) & 1, abort, a.status)) { ok = false; break; }
+        if (!warp_wait(smem_u32(&sh->s_full[buf]), (T >> 1) & 1, abort, a.status, 31, idx, j, T, kv_it)) { ok = false; break; }
+        if (!warp_wait(smem_u32(&sh->kv_full[st]), (kv_it / NST) & 1, abort, a.status, 32, idx, j, T, kv_it)) { ok = false; break; }
         tc_fence_after();
         float s[128];
 #pragma unroll
@@ -302,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           lsum *= f;
           if (grow) m = mnew;
           // O holds tiles 0..j-1: wait for the PV of tile j-1, then scale it
-          if (!warp_wait(smem_u32(&sh->o_ready), (pv - 1) & 1, abort, a.status)) { ok = false; break; }
+          if (!warp_wait(smem_u32(&sh->o_ready), (pv - 1) & 1, abort, a.status, 33, idx, j, pv, 0)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
@@ -333,8 +333,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       // epilogue: O / l.  Wait for the PVs of the last two tiles in order (the
       // parity of a phase two behind would alias the one awaited).
-      if (n >= 2 && !warp_wait(smem_u32(&sh->o_ready), (pv - 2) & 1, abort, a.status)) { ok = false; break; }
-      if (!warp_wait(smem_u32(&sh->o_ready), (pv - 1) & 1, abort, a.status)) { ok = false; break; }
+      if (n >= 2 && !warp_wait(smem_u32(&sh->o_ready), (pv - 2) & 1, abort, a.status, 34, idx, n, pv, 0)) { ok = false; break; }
+      if (!warp_wait(smem_u32(&sh->o_ready), (pv - 1) & 1, abort, a.status, 35, idx, n, pv, 0)) { ok = false; break; }
       tc_fence_after();
       const float inv = lsum > 0.f ? 1.0f / lsum : 0.f;
 #pragma unroll 1

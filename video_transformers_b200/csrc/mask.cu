@@ -92,7 +92,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int ct = 0; ct < nct && ok; ++ct) {
           for (int kc = 0; kc < nk; ++kc, ++it) {
             const int st = it % kStages;
-            if (!bounded_wait(smem_u32(&sh->empty[st]), ((it / kStages) & 1) ^ 1, abort, a.status)) { ok = false; break; }
+            if (!bounded_wait(smem_u32(&sh->empty[st]), ((it / kStages) & 1) ^ 1, abort, a.status, 41, item, ct, kc, it)) { ok = false; break; }
             const uint32_t bar = smem_u32(&sh->full[st]);
             mbar_arrive_expect_tx(bar, kStageBytes);
             const uint32_t dA = smem_u32(tiles + st * kStageBytes);
@@ -125,12 +125,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nct = tiles_for(r0);
         for (int ct = 0; ct < nct && ok; ++ct, ++t) {
           const int buf = t & 1;
-          if (!bounded_wait(smem_u32(&sh->s_empty[buf]), ((t >> 1) & 1) ^ 1, abort, a.status)) { ok = false; break; }
+          if (!bounded_wait(smem_u32(&sh->s_empty[buf]), ((t >> 1) & 1) ^ 1, abort, a.status, 42, item, ct, t, it)) { ok = false; break; }
           tc_fence_after();
           const uint32_t dS = tmem + buf * 128;
           for (int kc = 0; kc < nk; ++kc, ++it) {
             const int st = it % kStages;
-            if (!bounded_wait(smem_u32(&sh->full[st]), (it / kStages) & 1, abort, a.status)) { ok = false; break; }
+            if (!bounded_wait(smem_u32(&sh->full[st]), (it / kStages) & 1, abort, a.status, 43, item, ct, kc, it)) { ok = false; break; }
             tc_fence_after();
             const uint32_t sA = smem_u32(tiles + st * kStageBytes);
             const uint32_t sB = sA + kChunkBytes;
@@ -162,7 +162,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float M = -CUDART_INF_F, Ssum = 0.f;
       for (int ct = 0; ct < nct; ++ct, ++t) {
         const int buf = t & 1;
-        if (!warp_wait(smem_u32(&sh->s_full[buf]), (t >> 1) & 1, abort, a.status)) { ok = false; break; }
+        if (!warp_wait(smem_u32(&sh->s_full[buf]), (t >> 1) & 1, abort, a.status, 44, item, ct, t, 0)) { ok = false; break; }
         tc_fence_after();
         float z[128];
 #pragma unroll

@@ -18,7 +18,7 @@ constexpr int kDevTimeout = 5;
 // A bounded wait gives up after this many nanoseconds of %globaltimer, or
 // after kWaitLimitIters polls, whichever comes first.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
-constexpr uint32_t kWaitLimitIters = 1u << 26;
+constexpr uint32_t kWaitLimitIters = 1u << 30;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -56,12 +56,30 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for phase `parity` of an mbarrier, giving up after kWaitLimitNs or as
-// soon as another thread of the CTA has raised *abort.  On a time-out the
-// thread raises *abort and records kDevTimeout in *status (global memory).
-// Returns false when the caller must abandon its work.
-__device__ __forceinline__ bool bounded_wait(uint32_t bar, uint32_t parity, volatile int* abort,
-                                             int* status) {
+// The first bounded wait that runs out in a kernel records where it gave up
+// next to the status word: status[1] = 1 (record taken), status[2] = wait
+// site, [3] = block, [4] = thread, [5..8] = four caller counters.
+__device__ __forceinline__ void record_timeout(int* status, int site, int c0, int c1, int c2, int c3) {
+  atomicExch(status, kDevTimeout);
+  if (atomicCAS(status + 1, 0, 1) == 0) {
+    status[2] = site;
+    status[3] = static_cast<int>(blockIdx.x);
+    status[4] = static_cast<int>(threadIdx.x);
+    status[5] = c0;
+    status[6] = c1;
+    status[7] = c2;
+    status[8] = c3;
+    __threadfence();
+  }
+}
+
+// Wait for phase `parity` of an mbarrier, giving up after kWaitLimitNs (or
+// kWaitLimitIters polls), or as soon as another thread of the CTA has raised
+// *abort.  On its own time-out the thread raises *abort and records the wait
+// site and counters (record_timeout).  Returns false when the caller must
+// abandon its work.
+__device__ __forceinline__ bool bounded_wait(uint32_t bar, uint32_t parity, volatile int* abort, int* status,
+                                             int site = 0, int c0 = 0, int c1 = 0, int c2 = 0, int c3 = 0) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t i = 1;; ++i) {
@@ -70,7 +88,7 @@ __device__ __forceinline__ bool bounded_wait(uint32_t bar, uint32_t parity, vola
       if (*abort) return false;
       if (globaltimer() - t0 > kWaitLimitNs || i >= kWaitLimitIters) {
         *abort = 1;
-        atomicExch(status, kDevTimeout);
+        record_timeout(status, site, c0, c1, c2, c3);
         return false;
       }
     }
@@ -82,7 +100,7 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, int* s
   const uint64_t t0 = globaltimer();
   for (uint32_t i = 0; !mbar_try_wait(bar, parity); ++i) {
     if (globaltimer() - t0 > kWaitLimitNs || i >= kWaitLimitIters) {
-      atomicExch(status, kDevTimeout);
+      record_timeout(status, 90, static_cast<int>(parity), 0, 0, 0);
       return;
     }
   }
@@ -90,9 +108,9 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, int* s
 
 // Warp-uniform form for code that continues into .sync.aligned instructions:
 // every lane waits, and the warp gives up together if any lane gave up.
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort,
-                                          int* status) {
-  const bool ok = bounded_wait(bar, parity, abort, status);
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort, int* status,
+                                          int site = 0, int c0 = 0, int c1 = 0, int c2 = 0, int c3 = 0) {
+  const bool ok = bounded_wait(bar, parity, abort, status, site, c0, c1, c2, c3);
   return __all_sync(0xffffffffu, ok);
 }
 
