@@ -38,7 +38,7 @@ struct AttnShared {
   uint64_t q_full, q_empty;
   uint64_t kv_full[NST], kv_empty[NST];
   uint64_t s_full[2], p_full[2];
-  uint64_t o_ready, o_free, drain;
+  uint64_t o_ready, o_final, o_free, drain;
   uint32_t tmem_base;
   int abort;
   int flags[NST];
@@ -80,6 +80,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&sh->p_full[i]), 128);
     }
     mbar_init(smem_u32(&sh->o_ready), 1);
+    mbar_init(smem_u32(&sh->o_final), 1);
     mbar_init(smem_u32(&sh->o_free), 128);
     mbar_init(smem_u32(&sh->drain), 1);
     sh->abort = 0;
@@ -228,6 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!ok) break;
         if (!issue_pv(n - 1, n == 1)) { ok = false; break; }
+        umma_commit(smem_u32(&sh->o_final));   // O of this item is complete
         kv_it += n;
         T += n;
         ++icnt;
@@ -241,7 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = q * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     const int my_half_bit = 1 << (row >> 6);
-    uint32_t kv_it = 0, T = 0, pv = 0;
+    uint32_t kv_it = 0, T = 0, pv = 0, icnt = 0;
     bool ok = true;
     for (int idx = blockIdx.x; idx < a.n_items && ok; idx += gridDim.x) {
       const int item = a.queue[idx];
@@ -331,10 +333,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(smem_u32(&sh->p_full[buf]));
       }
       if (!ok) break;
-      // epilogue: O / l.  Wait for the PVs of the last two tiles in order (the
-      // parity of a phase two behind would alias the one awaited).
-      if (n >= 2 && !warp_wait(smem_u32(&sh->o_ready), (pv - 2) & 1, abort, a.status, 34, idx, n, pv, 0)) { ok = false; break; }
-      if (!warp_wait(smem_u32(&sh->o_ready), (pv - 1) & 1, abort, a.status, 35, idx, n, pv, 0)) { ok = false; break; }
+      // epilogue: O / l, once the item's last PV is done (o_final completes
+      // once per item; the MMA cannot start the next item's PVs before o_free,
+      // so its phases never run two ahead of this wait)
+      if (!warp_wait(smem_u32(&sh->o_final), icnt & 1, abort, a.status, 35, idx, n, pv, icnt)) { ok = false; break; }
+      ++icnt;
       tc_fence_after();
       const float inv = lsum > 0.f ? 1.0f / lsum : 0.f;
 #pragma unroll 1
