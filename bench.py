@@ -183,7 +183,7 @@ def run_psa(args, rank, world, local_rank):
     import video_transformers_b200 as P
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    w = W.PRESETS[args.config]
+    w = workload(args)
     log(args, "generating %s inputs" % w.name)
     q, k, v, gen = W.make_qkv(w, device=dev, seed=w.seed + rank)
     torch.cuda.synchronize()
@@ -384,7 +384,7 @@ def cpu_threads():
 def run_reference(args, rank, world):
     if rank != 0:
         return None
-    w = W.PRESETS[args.config]
+    w = workload(args)
     q, k, v, gen = W.make_qkv(w, device="cuda" if torch.cuda.is_available() else "cpu")
     mask = W.make_given_mask(w, gen, device=q.device) if w.mask_mode == "given" else None
     for _ in range(args.warmup):
@@ -408,6 +408,17 @@ def run_reference(args, rank, world):
 
 # ----------------------------------------------------------------------------- main
 
+def workload(args) -> W.Workload:
+    """The chosen preset; --heads shrinks it (same shape per head) for
+    profiling captures that must stay a few GB on the device."""
+    w = W.PRESETS[args.config]
+    if args.heads:
+        hq = args.heads
+        hkv = max(1, hq * w.Hkv // w.Hq)
+        w = w.replace(name="%s[Hq=%d]" % (w.name, hq), Hq=hq, Hkv=hkv)
+    return w
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -415,11 +426,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--config", default="wan14b", choices=W.ORDER)
     ap.add_argument("--impl", default="psa", choices=["psa", "reference"])
-    ap.add_argument("--cpu-blocks", type=int, default=3, help="query blocks in the oracle sample")
+    ap.add_argument("--cpu-blocks", type=int, default=40, help="query blocks in the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--verbose", action="store_true", help="progress and per-stage warm-up times on stderr")
+    ap.add_argument("--heads", type=int, default=0, help="override the query head count (profiling captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
