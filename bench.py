@@ -110,6 +110,22 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- helpers
 
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """Device time of the timed region, max over ranks (every rank takes
+    this collective at the same point)."""
+    if world <= 1:
+        return ms
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tflops(flops_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank runs its own workload instance of
+    `flops_per_rank` executed FLOPs per step (weak scaling)."""
+    return flops_per_rank * world / (ms_per_step * 1e-3) / 1e12
+
+
 def executed_flops(mask: torch.Tensor, N: int, block: int, d: int, levels: int, causal: bool) -> float:
     """4 d sum_{b,h,I} q_I * sum_{J: M != SKIP} k_J / 2^l (on the device)."""
     dev = mask.device
@@ -230,11 +246,7 @@ def run_psa(args, rank, world, local_rank):
             ev[i][3].record(stream)
         stop.record(stream)
         torch.cuda.synchronize()
-    total_ms = start.elapsed_time(stop)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(start.elapsed_time(stop), world, dev)
     st = P.psa_get_device_status(path.aws) or P.psa_get_device_status(path.mws)
     if st != P.PSA_OK:
         raise RuntimeError("device status %d after the timed region" % st)
@@ -242,7 +254,7 @@ def run_psa(args, rank, world, local_rank):
     mask_ms = statistics.mean(ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps))
     attn_ms = statistics.mean(ev[i][2].elapsed_time(ev[i][3]) for i in range(args.steps))
     ms_per_step = total_ms / args.steps
-    value = flops * world / (ms_per_step * 1e-3) / 1e12
+    value = aggregate_tflops(flops, world, ms_per_step)
 
     # dense reference point: same kernel, all-level-0 mask
     dense_mask = torch.zeros_like(path.mask)
