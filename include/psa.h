@@ -172,6 +172,31 @@ PSA_API psa_status_t psa_attention_fwd(const psa_shape_t* shape, const void* q, 
                                float sm_scale, void* out, float* lse,
                                void* workspace, size_t workspace_bytes, void* stream);
 
+/* psa_attention_fwd without a workspace argument, for callers that cannot
+ * allocate device memory themselves: for example a plugin inside a host
+ * framework that owns every device allocation, or a latency-critical loop
+ * where cudaMalloc's implicit device synchronisation is not acceptable.  The
+ * pages have no counterpart; this is an interface convenience only.
+ *
+ * The workspace is a file-scope device array of PSA_STATIC_WORKSPACE_BYTES
+ * (32 MiB) inside libpsa.so; every GPU that loads the library holds it until
+ * the process exits.  Shapes whose psa_attention_workspace_bytes exceeds it
+ * are rejected with PSA_ERR_WORKSPACE before anything is launched (it covers,
+ * for example, the Qwen2.5-VL- and Wan2.1-1.3B-shaped problems, not the
+ * Wan2.1-14B-shaped one).  The first call on each device looks up the
+ * array's device address (cudaGetSymbolAddress, with that device current),
+ * so make that first call before any stream capture.  No device memory is
+ * allocated or freed.  All calls share the one array and it keeps the last
+ * call's contents; each call clears the 36-byte status header it needs at
+ * zero, and calls that overlap on the GPU (other streams, other threads)
+ * race on the array.  Time-out reports from the kernel stay inside the
+ * array and are not readable through psa_get_device_status. */
+#define PSA_STATIC_WORKSPACE_BYTES (32u << 20)
+PSA_API psa_status_t psa_attention_fwd_static(const psa_shape_t* shape, const void* q, const void* k,
+                                              const void* v, const void* k_pyr, const void* v_pyr,
+                                              const uint8_t* mask, float sm_scale, void* out, float* lse,
+                                              void* stream);
+
 /* Executed work of the last plan built in `workspace` by psa_attention_fwd:
  * fills (synchronising on `stream`) the number of 128-row KV tiles and the
  * number of KV rows that hold real (non-padding) pooled tokens. */

@@ -27,7 +27,7 @@ PSA_SKIP = 0xFF
 EXPORTS = [
     "psa_pyramid_bytes", "psa_pyramid_level_offset", "psa_build_pyramid",
     "psa_mask_workspace_bytes", "psa_make_mask",
-    "psa_attention_workspace_bytes", "psa_attention_fwd", "psa_attention_plan_stats",
+    "psa_attention_workspace_bytes", "psa_attention_fwd", "psa_attention_fwd_static", "psa_attention_plan_stats",
     "psa_get_device_status", "psa_last_error", "psa_version",
 ]
 
@@ -66,6 +66,7 @@ def _load():
         "psa_make_mask": (I, [S, MP, P, P, P, P, P, P, Z, P]),
         "psa_attention_workspace_bytes": (Z, [S]),
         "psa_attention_fwd": (I, [S, P, P, P, P, P, P, F, P, P, P, Z, P]),
+        "psa_attention_fwd_static": (I, [S, P, P, P, P, P, P, F, P, P, P]),
         "psa_attention_plan_stats": (I, [S, P, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64), P]),
         "psa_get_device_status": (I, [P, P]),
         "psa_last_error": (ctypes.c_char_p, []),
@@ -175,6 +176,16 @@ def psa_attention_fwd(shape: Shape, q, k, v, k_pyr, v_pyr, mask, sm_scale: float
                                  ctypes.c_float(sm_scale), _ptr(out, "out"), _ptr(lse, "lse", False),
                                  _ptr(workspace, "workspace"), workspace.numel() * workspace.element_size(),
                                  _stream(stream)))
+
+
+def psa_attention_fwd_static(shape: Shape, q, k, v, k_pyr, v_pyr, mask, sm_scale: float, out, lse, stream=None):
+    """psa_attention_fwd on the library's own static device workspace (no
+    workspace argument; for callers that cannot allocate device memory)."""
+    L1 = shape.levels > 1
+    _check(lib().psa_attention_fwd_static(ctypes.byref(shape), _ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"),
+                                          _ptr(k_pyr, "k_pyr", L1), _ptr(v_pyr, "v_pyr", L1), _ptr(mask, "mask"),
+                                          ctypes.c_float(sm_scale), _ptr(out, "out"), _ptr(lse, "lse", False),
+                                          _stream(stream)))
 
 
 def psa_attention_plan_stats(shape: Shape, workspace, stream=None):

@@ -7,6 +7,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "internal.h"
 
@@ -452,3 +453,62 @@ psa_status_t psa_get_device_status(void* ws, void* stream) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ static workspace
+// The workspace of psa_attention_fwd_static: one array per device, reserved
+// when the library's device code is loaded.  Host code may not use the
+// array's name as a pointer (it is a host-side shadow); the device address
+// comes from cudaGetSymbolAddress, once per device, with that device current.
+static __device__ __align__(256) unsigned char g_static_workspace[PSA_STATIC_WORKSPACE_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mutex;
+void* g_static_ptr[kMaxDevices] = {};
+
+psa_status_t static_workspace(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(PSA_ERR_UNSUPPORTED, "device %d beyond %d", dev, kMaxDevices);
+  std::lock_guard<std::mutex> lock(g_static_mutex);
+  if (!g_static_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_workspace);
+    if (e != cudaSuccess || !p) return cuda_fail(e, "cudaGetSymbolAddress of the static workspace");
+    g_static_ptr[dev] = p;
+  }
+  *out = g_static_ptr[dev];
+  return PSA_OK;
+}
+}  // namespace
+
+extern "C" psa_status_t psa_attention_fwd_static(const psa_shape_t* s, const void* q, const void* k, const void* v,
+                                                 const void* k_pyr, const void* v_pyr, const uint8_t* mask,
+                                                 float sm_scale, void* out, float* lse, void* stream) {
+  g_err[0] = 0;
+  PSA_TRY(check_shape(s));
+  const size_t need = attn_layout(s).total;
+  if (need > PSA_STATIC_WORKSPACE_BYTES)
+    return fail(PSA_ERR_WORKSPACE, "this shape needs a %zu-byte workspace; the static workspace holds %u bytes",
+                need, PSA_STATIC_WORKSPACE_BYTES);
+  // the remaining argument checks of psa_attention_fwd, so that nothing is
+  // enqueued for a call that will be rejected
+  PSA_TRY(check_ptr(q, "q"));
+  PSA_TRY(check_ptr(k, "k"));
+  PSA_TRY(check_ptr(v, "v"));
+  PSA_TRY(check_ptr(out, "out"));
+  if (s->levels > 1) {
+    PSA_TRY(check_ptr(k_pyr, "k_pyr"));
+    PSA_TRY(check_ptr(v_pyr, "v_pyr"));
+  }
+  if (!mask) return fail(PSA_ERR_INVALID_ARG, "mask is NULL");
+  PSA_TRY(check_ptr(lse, "lse", false));
+  if (!(sm_scale > 0.f) || sm_scale != sm_scale) return fail(PSA_ERR_INVALID_ARG, "sm_scale must be > 0");
+  void* ws = nullptr;
+  PSA_TRY(static_workspace(&ws));
+  // the status header must start at zero; everything else is rewritten by the plan
+  PSA_CUDA(cudaMemsetAsync(ws, 0, 256, static_cast<cudaStream_t>(stream)), "static workspace header clear");
+  return psa_attention_fwd(s, q, k, v, k_pyr, v_pyr, mask, sm_scale, out, lse, ws, PSA_STATIC_WORKSPACE_BYTES,
+                           stream);
+}
