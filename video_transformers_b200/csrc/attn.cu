@@ -5,18 +5,23 @@
 // size from the hardware tile size; news review, Methodology 4: ordinary
 // scaled dot-product attention over the pooled KV).
 //
-// One persistent CTA per SM, 6 warps:
-//   warp 0      TMA producer: Q of the work item, then per 128-row KV tile one
-//               box per (segment, 64-channel chunk) of the level-l K and V
-//               maps, plus a per-column record (level bias, validity, last
-//               covered token, query-half mask) written to shared memory.
-//   warp 1      tcgen05 issuer (one thread): S = Q K^T into one of two TMEM
-//               S buffers, O += P V with P read from TMEM.
-//   warps 2..5  softmax, one query row per thread: S from TMEM, logit
-//               z = s * scale * log2(e) + l (the +ln 2^l bias in log2 units),
-//               online max / sum with lazy rescaling of O, P (bf16) back into
-//               the S buffer, and the final O / l and lse store.
-// Every wait is bounded; a time-out sets the workspace status word.
+// Two persistent CTAs per SM, 6 warps each:
+//   warp 0      TMA producer.  Per 128-row KV tile: one box per (segment,
+//               64-channel chunk) of the level-l K and V maps, issued by the
+//               lane that owns the segment, plus a small record of the tile
+//               (per 16-column chunk level, or per-column bias/validity when
+//               a tile has padding, a ragged block, a causal edge or a
+//               query-half mask) in a two-deep ring.
+//   warp 1      tcgen05 issuer (one thread): S = Q K^T into TMEM, then, once
+//               the softmax has written P over S, O += P V (P read from TMEM).
+//   warps 2..5  softmax, one query row per thread: exp2 argument
+//               s * scale * log2(e) + l - m (the +ln 2^l bias in log2 units),
+//               lazy rescaling of O in TMEM, P as bf16 back into TMEM, and
+//               the final O / l and lse store.
+// Each CTA has one S, K and V buffer, so its own MMAs and softmax alternate;
+// the second CTA on the SM keeps the tensor core busy meanwhile.
+// Every wait is bounded; a time-out sets the workspace status word and
+// records where it happened.
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
@@ -27,43 +32,44 @@ namespace psa {
 namespace {
 
 constexpr int kThreads = 192;
-constexpr float kRescaleThreshold = 8.0f;   // log2 units: P stays <= 256
+constexpr float kRescaleThreshold = 8.0f;   // log2 units: P stays <= 2^(8+3)
 
 struct AttnMaps {
   CUtensorMap m[9];
 };
 
-template <int NST>
-struct AttnShared {
-  uint64_t q_full, q_empty;
-  uint64_t kv_full[NST], kv_empty[NST];
-  uint64_t s_full[2], p_full[2];
-  uint64_t o_ready, o_final, o_free, drain;
-  uint32_t tmem_base;
-  int abort;
-  int flags[NST];
-  float bias[NST][128];
-  int info[NST][128];   // (last covered token << 2) | query-half mask
+// Record of one KV tile, written by the producer for the softmax.
+struct alignas(16) TileInfo {
+  float cb[8];          // level of each 16-column chunk (fast tiles)
+  int fast;             // every column valid, no per-row check needed
+  int rowcheck;         // slow tiles: some column needs the causal / half test
+  int pad[6];
+  float bias[128];      // slow tiles: level, or -inf for padding / past-the-end rows
+  int info[128];        // slow tiles: (last covered token << 2) | query-half mask
 };
 
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
+struct AttnShared {
+  uint64_t q_full, q_empty, k_full, k_empty, v_full, v_empty;
+  uint64_t i_full[2], i_empty[2];
+  uint64_t s_full, p_full, o_final, o_free, drain;
+  uint32_t tmem_base;
+  int abort;
+  TileInfo ti[2];
+};
 
 template <int D, bool OUT_F32>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     attn_kernel(const __grid_constant__ AttnMaps maps, const AttnArgs a) {
-  constexpr int NST = D == 128 ? 2 : 4;
   constexpr int QB = D * 256;          // bytes of a 128-row tile of D bf16 channels
   constexpr int KC = D / 64;           // 64-channel chunks
-  using Shared = AttnShared<NST>;
+  constexpr uint32_t kTmemCols = 256;  // S: columns [0,128), O: [128, 128 + D)
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = base;
   uint8_t* sK = sQ + QB;
-  uint8_t* sV = sK + NST * QB;
-  Shared* sh = reinterpret_cast<Shared*>(sV + NST * QB);
+  uint8_t* sV = sK + QB;
+  AttnShared* sh = reinterpret_cast<AttnShared*>(sV + QB);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int L = a.levels;
@@ -71,26 +77,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&sh->q_full), 1);
     mbar_init(smem_u32(&sh->q_empty), 1);
-    for (int i = 0; i < NST; ++i) {
-      mbar_init(smem_u32(&sh->kv_full[i]), 32);
-      mbar_init(smem_u32(&sh->kv_empty[i]), 1);
-    }
+    mbar_init(smem_u32(&sh->k_full), 1);
+    mbar_init(smem_u32(&sh->k_empty), 1);
+    mbar_init(smem_u32(&sh->v_full), 1);
+    mbar_init(smem_u32(&sh->v_empty), 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&sh->s_full[i]), 1);
-      mbar_init(smem_u32(&sh->p_full[i]), 128);
+      mbar_init(smem_u32(&sh->i_full[i]), 32);
+      mbar_init(smem_u32(&sh->i_empty[i]), 128);
     }
-    mbar_init(smem_u32(&sh->o_ready), 1);
+    mbar_init(smem_u32(&sh->s_full), 1);
+    mbar_init(smem_u32(&sh->p_full), 128);
     mbar_init(smem_u32(&sh->o_final), 1);
     mbar_init(smem_u32(&sh->o_free), 128);
     mbar_init(smem_u32(&sh->drain), 1);
     sh->abort = 0;
     fence_mbar_init();
   }
-  if (warp == 1) { tmem_alloc(smem_u32(&sh->tmem_base), 512); tmem_relinquish(); }
+  if (warp == 1) { tmem_alloc(smem_u32(&sh->tmem_base), kTmemCols); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sh->tmem_base;
+  const uint32_t tS = tmem, tO = tmem + 128;
   volatile int* abort = &sh->abort;
 
   if (warp == 0) {
@@ -98,7 +106,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       for (int i = 0; i < 1 + 2 * L; ++i) tma_prefetch_desc(&maps.m[i]);
     }
-    uint32_t kv_it = 0, qcnt = 0;
+    uint32_t kcnt = 0, qcnt = 0;
     bool ok = true;
     for (int idx = blockIdx.x; idx < a.n_items && ok; idx += gridDim.x) {
       const int item = a.queue[idx];
@@ -108,7 +116,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int b = bh / a.Hq, h = bh - b * a.Hq;
       const int hkv = b * a.Hkv + h / (a.Hq / a.Hkv);
       const int q0 = tq * 128;
-      if (!warp_wait(smem_u32(&sh->q_empty), (qcnt & 1) ^ 1, abort, a.status, 11, idx, qcnt, kv_it, 0)) { ok = false; break; }
+      if (!warp_wait(smem_u32(&sh->q_empty), (qcnt & 1) ^ 1, abort, a.status, 11, idx, qcnt, kcnt, 0)) { ok = false; break; }
       if (lane == 0) {
         const uint32_t bar = smem_u32(&sh->q_full);
         mbar_arrive_expect_tx(bar, QB);
@@ -116,60 +124,91 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kc = 0; kc < KC; ++kc) tma_load_3d(smem_u32(sQ + kc * 16384), &maps.m[0], bar, kc * 64, q0, bh);
       }
       ++qcnt;
-      for (int t = t0; t < t1; ++t, ++kv_it) {
-        const int st = kv_it % NST;
-        if (!warp_wait(smem_u32(&sh->kv_empty[st]), ((kv_it / NST) & 1) ^ 1, abort, a.status, 12, idx, t - t0, kv_it, 0)) { ok = false; break; }
-        const int sb = a.tile_seg_off[t], se = a.tile_seg_off[t + 1];
-        const uint32_t bar = smem_u32(&sh->kv_full[st]);
-        if (lane == 0) {
-          mbar_expect_tx(bar, 2 * QB);
-          const uint32_t dK = smem_u32(sK + st * QB), dV = smem_u32(sV + st * QB);
-          int r = 0;
-          for (int s = sb; s < se; ++s) {
-            const int w = a.segs[s];
-            const int l = seg_level(w), half = seg_half(w), J = seg_block(w);
-            const int rows = a.block >> l;
-            const int prow = half ? J * rows : (a.N >> l);   // padding reads past the end: zeros
+      for (int t = t0; t < t1; ++t, ++kcnt) {
+        // this tile's segments: lane s owns segment s (at most 16)
+        const int sb = a.tile_seg_off[t], nseg = a.tile_seg_off[t + 1] - sb;
+        const int w = lane < nseg ? a.segs[sb + lane] : 0;
+        const int l = seg_level(w), half = seg_half(w), J = seg_block(w);
+        const int rows = lane < nseg ? (a.block >> l) : 0;
+        int r = rows;                                   // inclusive scan -> exclusive row offset
 #pragma unroll
-            for (int kc = 0; kc < KC; ++kc) {
-              tma_load_3d(dK + kc * 16384 + r * 128, &maps.m[1 + l], bar, kc * 64, prow, hkv);
-              tma_load_3d(dV + kc * 16384 + r * 128, &maps.m[1 + L + l], bar, kc * 64, prow, hkv);
-            }
-            r += rows;
-          }
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, r, o);
+          if (lane >= o) r += y;
         }
-        // per-column record of this tile
-        bool need = false;
-        int r = 0;
-        for (int s = sb; s < se; ++s) {
-          const int w = a.segs[s];
-          const int l = seg_level(w), half = seg_half(w), J = seg_block(w);
-          const int rows = a.block >> l;
+        r -= rows;
+        const int nl = a.N >> l;
+        const int prow = half ? J * rows : nl;          // padding reads past the end: zeros
+
+        // K
+        if (!warp_wait(smem_u32(&sh->k_empty), (kcnt & 1) ^ 1, abort, a.status, 12, idx, t - t0, kcnt, 0)) { ok = false; break; }
+        if (lane == 0) mbar_arrive_expect_tx(smem_u32(&sh->k_full), QB);
+        __syncwarp();
+        if (lane < nseg) {
+#pragma unroll
+          for (int kc = 0; kc < KC; ++kc)
+            tma_load_3d(smem_u32(sK + kc * 16384 + r * 128), &maps.m[1 + l], smem_u32(&sh->k_full), kc * 64, prow, hkv);
+        }
+
+        // tile record
+        const int slot = kcnt & 1;
+        if (!warp_wait(smem_u32(&sh->i_empty[slot]), ((kcnt >> 1) & 1) ^ 1, abort, a.status, 13, idx, t - t0, kcnt, 0)) { ok = false; break; }
+        TileInfo& ti = sh->ti[slot];
+        const int last_tok = ((J * rows + rows) << l) - 1;   // last token covered by the segment
+        const bool seg_pad = lane < nseg && half == 0;
+        const bool seg_ragged = lane < nseg && half != 0 && J * rows + rows > nl;
+        const bool seg_check = lane < nseg && half != 0 && (half != 3 || (a.causal && last_tok > q0));
+        const bool fast = !__any_sync(0xffffffffu, seg_pad || seg_ragged || seg_check);
+        const bool rowcheck = __any_sync(0xffffffffu, seg_check);
+        if (fast) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const unsigned bal = __ballot_sync(0xffffffffu, lane < nseg && r <= 16 * k);
+            const int lev = __shfl_sync(0xffffffffu, l, __popc(bal) - 1);
+            if (lane == k) ti.cb[k] = static_cast<float>(lev);
+          }
+        } else {
 #pragma unroll
           for (int m = 0; m < 4; ++m) {
             const int c = lane + 32 * m;
-            if (c >= r && c < r + rows) {
-              const int p = J * rows + (c - r);
-              const bool valid = half != 0 && p < (a.N >> l);
-              const int last = ((p + 1) << l) - 1;
-              sh->bias[st][c] = valid ? static_cast<float>(l) : -CUDART_INF_F;
-              sh->info[st][c] = (last << 2) | half;
-              need |= valid && (half != 3 || (a.causal && last > q0));
+            float bias = -CUDART_INF_F;
+            int inf = 0;
+            for (int s = 0; s < nseg; ++s) {
+              const int rs = __shfl_sync(0xffffffffu, r, s);
+              const int ws = __shfl_sync(0xffffffffu, w, s);
+              const int ls = seg_level(ws), hs = seg_half(ws), Js = seg_block(ws);
+              const int rws = a.block >> ls;
+              if (c >= rs && c < rs + rws) {
+                const int p = Js * rws + (c - rs);
+                const bool valid = hs != 0 && p < (a.N >> ls);
+                bias = valid ? static_cast<float>(ls) : -CUDART_INF_F;
+                inf = ((((p + 1) << ls) - 1) << 2) | hs;
+              }
             }
+            ti.bias[c] = bias;
+            ti.info[c] = inf;
           }
-          r += rows;
         }
-        const bool any = __any_sync(0xffffffffu, need);
-        if (lane == 0) sh->flags[st] = any ? 1 : 0;
+        if (lane == 0) { ti.fast = fast ? 1 : 0; ti.rowcheck = rowcheck ? 1 : 0; }
+        mbar_arrive(smem_u32(&sh->i_full[slot]));
+
+        // V
+        if (!warp_wait(smem_u32(&sh->v_empty), (kcnt & 1) ^ 1, abort, a.status, 14, idx, t - t0, kcnt, 0)) { ok = false; break; }
+        if (lane == 0) mbar_arrive_expect_tx(smem_u32(&sh->v_full), QB);
         __syncwarp();
-        mbar_arrive(bar);
+        if (lane < nseg) {
+#pragma unroll
+          for (int kc = 0; kc < KC; ++kc)
+            tma_load_3d(smem_u32(sV + kc * 16384 + r * 128), &maps.m[1 + L + l], smem_u32(&sh->v_full), kc * 64, prow, hkv);
+        }
       }
     }
-    // drain: wait for every TMA this warp issued before the CTA may exit
+    // drain: every TMA this warp issued must land before the CTA exits
     if (lane == 0) {
       if (qcnt > 0) drain_wait(smem_u32(&sh->q_full), (qcnt - 1) & 1, a.status);
-      for (uint32_t st = 0; st < NST; ++st) {
-        if (kv_it > st) drain_wait(smem_u32(&sh->kv_full[st]), ((kv_it - 1 - st) / NST) & 1, a.status);
+      if (kcnt > 0) {
+        drain_wait(smem_u32(&sh->k_full), (kcnt - 1) & 1, a.status);
+        drain_wait(smem_u32(&sh->v_full), (kcnt - 1) & 1, a.status);
       }
     }
   } else if (warp == 1) {
@@ -177,61 +216,46 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, 128, false);
       constexpr uint32_t idO = idesc_bf16_f32(128, D, true);
-      const uint32_t tO = tmem + 256;
-      uint32_t kv_it = 0, T = 0, qcnt = 0, icnt = 0;
+      uint32_t kcnt = 0, qcnt = 0, icnt = 0;
       bool ok = true;
-      auto issue_pv = [&](uint32_t jj, bool first_of_item) -> bool {
-        const uint32_t st = (kv_it + jj) % NST;
-        const uint32_t buf = (T + jj) & 1;
-        if (first_of_item && icnt > 0) {
-          if (!bounded_wait(smem_u32(&sh->o_free), (icnt - 1) & 1, abort, a.status, 21, icnt, jj, T, kv_it)) return false;
-        }
-        if (!bounded_wait(smem_u32(&sh->p_full[buf]), ((T + jj) >> 1) & 1, abort, a.status, 22, icnt, jj, T, kv_it)) return false;
-        tc_fence_after();
-        const uint32_t sV_st = smem_u32(sV + st * QB);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          umma_ts(tO, tmem + buf * 128 + k * 8, sdesc_sw128(sV_st + k * 2048, 16384, 1024), idO,
-                  (first_of_item && k == 0) ? 0u : 1u);
-        }
-        umma_commit(smem_u32(&sh->kv_empty[st]));
-        umma_commit(smem_u32(&sh->o_ready));
-        return true;
-      };
       for (int idx = blockIdx.x; idx < a.n_items && ok; idx += gridDim.x) {
         const int item = a.queue[idx];
         const int t0 = a.item_tile_off[item], t1 = a.item_tile_off[item + 1];
         const uint32_t n = static_cast<uint32_t>(t1 - t0);
         if (n == 0) continue;
-        if (!bounded_wait(smem_u32(&sh->q_full), qcnt & 1, abort, a.status, 23, idx, qcnt, T, kv_it)) { ok = false; break; }
+        if (!bounded_wait(smem_u32(&sh->q_full), qcnt & 1, abort, a.status, 23, idx, qcnt, kcnt, 0)) { ok = false; break; }
         tc_fence_after();
         ++qcnt;
-        const uint32_t sQb = smem_u32(sQ);
-        for (uint32_t j = 0; j < n && ok; ++j) {
-          const uint32_t st = (kv_it + j) % NST;
-          const uint32_t buf = (T + j) & 1;
-          if (!bounded_wait(smem_u32(&sh->kv_full[st]), ((kv_it + j) / NST) & 1, abort, a.status, 24, idx, j, T, kv_it)) { ok = false; break; }
+        const uint32_t sQb = smem_u32(sQ), sKb = smem_u32(sK), sVb = smem_u32(sV);
+        for (uint32_t j = 0; j < n; ++j, ++kcnt) {
+          // S = Q K^T
+          if (!bounded_wait(smem_u32(&sh->k_full), kcnt & 1, abort, a.status, 24, idx, j, kcnt, 0)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sK_st = smem_u32(sK + st * QB);
 #pragma unroll
           for (int kc = 0; kc < KC; ++kc) {
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              umma_ss(tmem + buf * 128, sdesc_sw128(sQb + kc * 16384 + 32 * k, 16, 1024),
-                      sdesc_sw128(sK_st + kc * 16384 + 32 * k, 16, 1024), idS, (kc | k) != 0);
+              umma_ss(tS, sdesc_sw128(sQb + kc * 16384 + 32 * k, 16, 1024),
+                      sdesc_sw128(sKb + kc * 16384 + 32 * k, 16, 1024), idS, (kc | k) != 0);
             }
           }
-          umma_commit(smem_u32(&sh->s_full[buf]));
+          umma_commit(smem_u32(&sh->s_full));
+          umma_commit(smem_u32(&sh->k_empty));
           if (j + 1 == n) umma_commit(smem_u32(&sh->q_empty));
-          if (j >= 1) {
-            if (!issue_pv(j - 1, j == 1)) { ok = false; break; }
+          // O += P V, once the softmax has written P
+          if (!bounded_wait(smem_u32(&sh->p_full), kcnt & 1, abort, a.status, 25, idx, j, kcnt, 0)) { ok = false; break; }
+          if (j == 0 && icnt > 0) {
+            if (!bounded_wait(smem_u32(&sh->o_free), (icnt - 1) & 1, abort, a.status, 21, idx, icnt, kcnt, 0)) { ok = false; break; }
           }
+          if (!bounded_wait(smem_u32(&sh->v_full), kcnt & 1, abort, a.status, 26, idx, j, kcnt, 0)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            umma_ts(tO, tS + k * 8, sdesc_sw128(sVb + k * 2048, 16384, 1024), idO, (j == 0 && k == 0) ? 0u : 1u);
+          }
+          umma_commit(smem_u32(&sh->v_empty));
+          if (j + 1 == n) umma_commit(smem_u32(&sh->o_final));
         }
-        if (!ok) break;
-        if (!issue_pv(n - 1, n == 1)) { ok = false; break; }
-        umma_commit(smem_u32(&sh->o_final));   // O of this item is complete
-        kv_it += n;
-        T += n;
         ++icnt;
       }
       umma_commit(smem_u32(&sh->drain));
@@ -243,7 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = q * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     const int my_half_bit = 1 << (row >> 6);
-    uint32_t kv_it = 0, T = 0, pv = 0, icnt = 0;
+    uint32_t kcnt = 0, icnt = 0;
     bool ok = true;
     for (int idx = blockIdx.x; idx < a.n_items && ok; idx += gridDim.x) {
       const int item = a.queue[idx];
@@ -266,84 +290,129 @@ __global__ void __launch_bounds__(kThreads, 1)
         continue;
       }
       float m = -CUDART_INF_F, lsum = 0.f;
-      for (int j = 0; j < n; ++j, ++kv_it, ++T, ++pv) {
-        const int st = kv_it % NST;
-        const int buf = T & 1;
-        if (!warp_wait(smem_u32(&sh->s_full[buf]), (T >> 1) & 1, abort, a.status, 31, idx, j, T, kv_it)) { ok = false; break; }
-        if (!warp_wait(smem_u32(&sh->kv_full[st]), (kv_it / NST) & 1, abort, a.status, 32, idx, j, T, kv_it)) { ok = false; break; }
+      for (int j = 0; j < n; ++j, ++kcnt) {
+        const int slot = kcnt & 1;
+        if (!warp_wait(smem_u32(&sh->s_full), kcnt & 1, abort, a.status, 31, idx, j, kcnt, 0)) { ok = false; break; }
+        if (!warp_wait(smem_u32(&sh->i_full[slot]), (kcnt >> 1) & 1, abort, a.status, 32, idx, j, kcnt, 0)) { ok = false; break; }
         tc_fence_after();
-        float s[128];
+        const TileInfo& ti = sh->ti[slot];
+        uint32_t sr[128];
+        tmem_ld128(tS + lane_off, sr);
+        float* s = reinterpret_cast<float*>(sr);
+        // exp2 argument of column c in chunk k: s[c] * sc + cb[k] - m
+        float sc = a.scale_log2;
+        float cb[8];
+        float mt;
+        if (ti.fast) {
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          uint32_t raw[32];
-          tmem_ld32(tmem + buf * 128 + c4 * 32 + lane_off, raw);
+          for (int k = 0; k < 8; ++k) cb[k] = ti.cb[k];
+          float cmax[8];
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            s[c4 * 32 + i] = fmaf(__uint_as_float(raw[i]), a.scale_log2, sh->bias[st][c4 * 32 + i]);
-        }
-        if (sh->flags[st]) {
-#pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            const int inf = sh->info[st][c];
-            const bool vis = (inf & my_half_bit) && (!a.causal || (inf >> 2) <= tok);
-            s[c] = vis ? s[c] : -CUDART_INF_F;
+          for (int k = 0; k < 8; ++k) {
+            float x0 = fmaxf(s[16 * k + 0], s[16 * k + 1]), x1 = fmaxf(s[16 * k + 2], s[16 * k + 3]);
+            float x2 = fmaxf(s[16 * k + 4], s[16 * k + 5]), x3 = fmaxf(s[16 * k + 6], s[16 * k + 7]);
+            float x4 = fmaxf(s[16 * k + 8], s[16 * k + 9]), x5 = fmaxf(s[16 * k + 10], s[16 * k + 11]);
+            float x6 = fmaxf(s[16 * k + 12], s[16 * k + 13]), x7 = fmaxf(s[16 * k + 14], s[16 * k + 15]);
+            x0 = fmaxf(x0, x1); x2 = fmaxf(x2, x3); x4 = fmaxf(x4, x5); x6 = fmaxf(x6, x7);
+            cmax[k] = fmaf(fmaxf(fmaxf(x0, x2), fmaxf(x4, x6)), sc, cb[k]);
           }
-        }
-        float mt = s[0];
+          mt = fmaxf(fmaxf(fmaxf(cmax[0], cmax[1]), fmaxf(cmax[2], cmax[3])),
+                     fmaxf(fmaxf(cmax[4], cmax[5]), fmaxf(cmax[6], cmax[7])));
+        } else {
+          // per-column bias (padding, ragged tails) and, if needed, the
+          // causal / query-half test; afterwards s holds the full argument
 #pragma unroll
-        for (int c = 1; c < 128; ++c) mt = fmaxf(mt, s[c]);
+          for (int c4 = 0; c4 < 32; ++c4) {
+            const float4 bv = *reinterpret_cast<const float4*>(&ti.bias[4 * c4]);
+            s[4 * c4 + 0] = fmaf(s[4 * c4 + 0], sc, bv.x);
+            s[4 * c4 + 1] = fmaf(s[4 * c4 + 1], sc, bv.y);
+            s[4 * c4 + 2] = fmaf(s[4 * c4 + 2], sc, bv.z);
+            s[4 * c4 + 3] = fmaf(s[4 * c4 + 3], sc, bv.w);
+          }
+          if (ti.rowcheck) {
+#pragma unroll
+            for (int c4 = 0; c4 < 32; ++c4) {
+              const int4 iv = *reinterpret_cast<const int4*>(&ti.info[4 * c4]);
+              const int iw[4] = {iv.x, iv.y, iv.z, iv.w};
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const bool vis = (iw[u] & my_half_bit) && (!a.causal || (iw[u] >> 2) <= tok);
+                s[4 * c4 + u] = vis ? s[4 * c4 + u] : -CUDART_INF_F;
+              }
+            }
+          }
+          sc = 1.0f;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) cb[k] = 0.f;
+          float x[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) x[u] = s[u];
+#pragma unroll
+          for (int c = 8; c < 128; c += 8) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) x[u] = fmaxf(x[u], s[c + u]);
+          }
+          mt = fmaxf(fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3])), fmaxf(fmaxf(x[4], x[5]), fmaxf(x[6], x[7])));
+        }
+        // the tile record may be reused once read
+        mbar_arrive(smem_u32(&sh->i_empty[slot]));
+
         const float mnew = fmaxf(m, mt);
         // Lazy rescaling: a row moves its reference max only when the new max
         // exceeds it by more than kRescaleThreshold (or on its first visible
-        // key).  O lives in TMEM and is read/written with warp-collective
-        // tcgen05.ld/st, so the decision to touch O is taken per warp.
+        // key).  O is read and written with warp-collective tcgen05.ld/st, so
+        // the decision to touch O is taken per warp.  The PV of the previous
+        // tile is complete: its commit preceded this tile's S.
         const bool first = m == -CUDART_INF_F && mnew != -CUDART_INF_F;
         const bool grow = m != -CUDART_INF_F && mnew > m + kRescaleThreshold;
         if (__any_sync(0xffffffffu, grow)) {
           const float f = grow ? fast_exp2(m - mnew) : 1.0f;
           lsum *= f;
           if (grow) m = mnew;
-          // O holds tiles 0..j-1: wait for the PV of tile j-1, then scale it
-          if (!warp_wait(smem_u32(&sh->o_ready), (pv - 1) & 1, abort, a.status, 33, idx, j, pv, 0)) { ok = false; break; }
-          tc_fence_after();
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
-            tmem_ld32(tmem + 256 + c * 32 + lane_off, o);
+            tmem_ld32(tO + c * 32 + lane_off, o);
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
-            tmem_st32(tmem + 256 + c * 32 + lane_off, o);
+            tmem_st32(tO + c * 32 + lane_off, o);
           }
         }
         if (first) m = mnew;
         const float mu = m == -CUDART_INF_F ? 0.f : m;
-        float ps = 0.f;
         uint32_t pk[64];
+        float part[8];
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const float p0 = fast_exp2(s[2 * i] - mu), p1 = fast_exp2(s[2 * i + 1] - mu);
-          ps += p0 + p1;
-          pk[i] = pack_bf16(p0, p1);
+        for (int k = 0; k < 8; ++k) {
+          const float off = cb[k] - mu;
+          float acc = 0.f;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float p0 = fast_exp2(fmaf(s[16 * k + 2 * i], sc, off));
+            const float p1 = fast_exp2(fmaf(s[16 * k + 2 * i + 1], sc, off));
+            acc += p0 + p1;
+            pk[8 * k + i] = pack_bf16(p0, p1);
+          }
+          part[k] = acc;
         }
-        lsum += ps;
-        tmem_st32(tmem + buf * 128 + lane_off, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
-        tmem_st32(tmem + buf * 128 + 32 + lane_off, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
+        lsum += ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
+        tmem_st64(tS + lane_off, pk);
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(smem_u32(&sh->p_full[buf]));
+        mbar_arrive(smem_u32(&sh->p_full));
       }
       if (!ok) break;
-      // epilogue: O / l, once the item's last PV is done (o_final completes
-      // once per item; the MMA cannot start the next item's PVs before o_free,
-      // so its phases never run two ahead of this wait)
-      if (!warp_wait(smem_u32(&sh->o_final), icnt & 1, abort, a.status, 35, idx, n, pv, icnt)) { ok = false; break; }
+      // epilogue: O / l once the item's last PV is done (o_final completes
+      // once per item and cannot run ahead: the next item's first PV waits
+      // for o_free)
+      if (!warp_wait(smem_u32(&sh->o_final), icnt & 1, abort, a.status, 35, idx, n, kcnt, icnt)) { ok = false; break; }
       ++icnt;
       tc_fence_after();
       const float inv = lsum > 0.f ? 1.0f / lsum : 0.f;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
-        tmem_ld32(tmem + 256 + c * 32 + lane_off, o);
+        tmem_ld32(tO + c * 32 + lane_off, o);
         if (tok < a.N) {
           if (OUT_F32) {
             float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow * D + c * 32);
@@ -377,18 +446,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   if (warp == 1) {
     __syncwarp();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 
 template <int D, bool F32>
 cudaError_t launch_one(const AttnMaps& maps, const AttnArgs& a, int num_sms, cudaStream_t s) {
-  constexpr int NST = D == 128 ? 2 : 4;
-  const size_t smem = 1024 + static_cast<size_t>(D) * 256 * (1 + 2 * NST) + sizeof(AttnShared<NST>);
+  const size_t smem = 1024 + static_cast<size_t>(D) * 256 * 3 + sizeof(AttnShared);
   cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, F32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const int grid = a.n_items < num_sms ? a.n_items : num_sms;
+  const int grid = a.n_items < 2 * num_sms ? a.n_items : 2 * num_sms;
   attn_kernel<D, F32><<<grid, kThreads, smem, s>>>(maps, a);
   return cudaGetLastError();
 }
