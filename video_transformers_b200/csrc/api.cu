@@ -404,6 +404,7 @@ psa_status_t psa_attention_fwd(const psa_shape_t* s, const void* q, const void* 
   pa.queue = reinterpret_cast<int*>(w + L.queue);
   pa.hist = reinterpret_cast<int*>(w + L.hist);
   pa.n_hist = L.n_hist;
+  pa.lpt_queue = 0;
   pa.stats = reinterpret_cast<long long*>(w + L.stats);
   PSA_CUDA(psa::launch_plan(pa, st), "plan launch");
 

@@ -66,7 +66,8 @@ struct PlanArgs {
   int* item_tile_off;    // [n_items+1]
   int* tile_seg_off;     // [max_tiles+1]
   int* segs;             // [max_segs]
-  int* queue;            // [n_items]  item ids, most tiles first
+  int* queue;            // [n_items]  item ids in processing order
+  int lpt_queue;         // 1: most tiles first; 0: natural (head-major) order
   int* hist;             // [n_hist]   scratch for the counting sort
   int n_hist;
   long long* stats;      // [2] tiles, real kv rows

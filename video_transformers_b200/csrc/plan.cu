@@ -14,9 +14,9 @@
 // padding segments that read zeros.
 //
 // plan_count (warp per item) -> plan_scan (one CTA) -> plan_fill (warp per
-// item).  The queue lists items by tile count, largest first, so a
-// persistent kernel that deals them out round-robin ends its CTAs close
-// together.
+// item).  The queue is either head-major (items in their natural order, so
+// the CTAs running at one time share one head's KV in L2) or sorted by tile
+// count, largest first (the longest-processing-time order).
 #include "internal.h"
 
 namespace psa {
@@ -195,13 +195,12 @@ __global__ void plan_fill(const PlanArgs a) {
         rem -= sz;
       }
     }
-    if (ntile > 0) {
+    if (a.lpt_queue) {
       const int bin = min(ntile, a.n_hist - 1);
       const int pos = atomicAdd(&a.hist[bin], 1);
       a.queue[pos] = warp;
     } else {
-      const int pos = atomicAdd(&a.hist[0], 1);
-      a.queue[pos] = warp;
+      a.queue[warp] = warp;
     }
   }
 }
