@@ -25,6 +25,7 @@
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
+#include "exp2_poly.h"
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -32,6 +33,10 @@ namespace psa {
 namespace {
 
 constexpr int kThreads = 192;
+// Of every 8 column pairs of a full tile, this many take their exponential
+// on the FMA pipe (exp2_fma2) instead of the special-function unit, which
+// would otherwise be the busiest unit of the softmax warps.
+constexpr int kPolyPairs = 2;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: P stays <= 2^(8+3)
 
 struct AttnMaps {
@@ -56,6 +61,53 @@ struct AttnShared {
   int abort;
   TileInfo ti[2];
 };
+
+// 2^x for two lanes at once on the FMA pipe, x <= 20: Cody-Waite split
+// x = n + f with n = round(x) (adding 1.5 * 2^23 rounds to an integer in the
+// low mantissa bits) and f in [-1/2, 1/2]; 2^f from the Remez polynomial of
+// exp2_poly.h; 2^n added to the exponent field as an integer.  Inputs below
+// -126 are clamped there (the result is then <= 2^-126, not 0), so it is
+// used only where every column is a real key.
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  x.x = fmaxf(x.x, -126.0f);
+  x.y = fmaxf(x.y, -126.0f);
+  const float2 t = __fadd2_rn(x, make_float2(12582912.0f, 12582912.0f));
+  const float2 n = __fadd2_rn(t, make_float2(-12582912.0f, -12582912.0f));
+  const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), x);
+  float2 p = __ffma2_rn(make_float2(kExp2Poly3, kExp2Poly3), f, make_float2(kExp2Poly2, kExp2Poly2));
+  p = __ffma2_rn(p, f, make_float2(kExp2Poly1, kExp2Poly1));
+  p = __ffma2_rn(p, f, make_float2(kExp2Poly0, kExp2Poly0));
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
+// P for one tile row: p = 2^(s * sc + cb[k] - mu) per 16-column chunk k,
+// packed to bf16 pairs; returns the row sum of p (fp32).
+template <int POLY>
+__device__ __forceinline__ float tile_probs(const float* s, float sc, const float (&cb)[8], float mu,
+                                            uint32_t (&pk)[64]) {
+  const float2 sc2 = make_float2(sc, sc);
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float2 off = make_float2(cb[k] - mu, cb[k] - mu);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float2 x = __ffma2_rn(make_float2(s[16 * k + 2 * i], s[16 * k + 2 * i + 1]), sc2, off);
+      float2 p;
+      if (i < POLY) {
+        p = exp2_fma2(x);
+      } else {
+        p.x = fast_exp2(x.x);
+        p.y = fast_exp2(x.y);
+      }
+      acc[i & 3] = __fadd2_rn(acc[i & 3], p);
+      pk[8 * k + i] = pack_bf16(p.x, p.y);
+    }
+  }
+  const float2 t = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+  return t.x + t.y;
+}
 
 template <int D, bool OUT_F32>
 __global__ void __launch_bounds__(kThreads, 2)
@@ -303,7 +355,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         float sc = a.scale_log2;
         float cb[8];
         float mt;
-        if (ti.fast) {
+        const bool fast_tile = ti.fast != 0;
+        if (fast_tile) {
 #pragma unroll
           for (int k = 0; k < 8; ++k) cb[k] = ti.cb[k];
           float cmax[8];
@@ -381,21 +434,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (first) m = mnew;
         const float mu = m == -CUDART_INF_F ? 0.f : m;
         uint32_t pk[64];
-        float part[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const float off = cb[k] - mu;
-          float acc = 0.f;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float p0 = fast_exp2(fmaf(s[16 * k + 2 * i], sc, off));
-            const float p1 = fast_exp2(fmaf(s[16 * k + 2 * i + 1], sc, off));
-            acc += p0 + p1;
-            pk[8 * k + i] = pack_bf16(p0, p1);
-          }
-          part[k] = acc;
-        }
-        lsum += ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
+        // full tiles split the exponentials between MUFU and the FMA pipe;
+        // tiles with masked columns (p must be exactly 0 there) use MUFU only
+        lsum += fast_tile ? tile_probs<kPolyPairs>(s, sc, cb, mu, pk) : tile_probs<0>(s, sc, cb, mu, pk);
         tmem_st64(tS + lane_off, pk);
         tmem_st_wait();
         tc_fence_before();
