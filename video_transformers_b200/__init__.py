@@ -51,11 +51,11 @@ class MaskParams(ctypes.Structure):
                 ("sm_scale", ctypes.c_float)]
 
 
-def _load():
-    if not os.path.exists(LIB_PATH):
+def _load(path: str = LIB_PATH):
+    if not os.path.exists(path):
         raise ImportError("libpsa.so is not built (run: python -m video_transformers_b200.build); "
                           "the PSA path has no CPU fallback")
-    lib = ctypes.CDLL(LIB_PATH)
+    lib = ctypes.CDLL(path)
     P, S, I, F, Z = ctypes.c_void_p, ctypes.POINTER(Shape), ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
     MP = ctypes.POINTER(MaskParams)
     sig = {

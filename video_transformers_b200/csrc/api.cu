@@ -387,8 +387,9 @@ psa_status_t psa_attention_fwd(const psa_shape_t* s, const void* q, const void* 
   for (int l = 0; l < s->levels; ++l) {
     const void* kb = l == 0 ? k16 : static_cast<const void*>(kp16 + pyr_level_offset(s, l, 2));
     const void* vb = l == 0 ? v16 : static_cast<const void*>(vp16 + pyr_level_offset(s, l, 2));
-    PSA_TRY(map3(&maps[1 + l], kb, BHkv, s->N >> l, s->d, s->block >> l));
-    PSA_TRY(map3(&maps[1 + s->levels + l], vb, BHkv, s->N >> l, s->d, s->block >> l));
+    const int box = (s->block >> l) < 64 ? (s->block >> l) : 64;   // KV sub-tiles are 64 rows
+    PSA_TRY(map3(&maps[1 + l], kb, BHkv, s->N >> l, s->d, box));
+    PSA_TRY(map3(&maps[1 + s->levels + l], vb, BHkv, s->N >> l, s->d, box));
   }
   const int nkb = static_cast<int>(ceil_div(s->N, s->block));
   psa::PlanArgs pa{};
@@ -413,6 +414,7 @@ psa_status_t psa_attention_fwd(const psa_shape_t* s, const void* q, const void* 
   aa.levels = s->levels; aa.causal = s->causal != 0; aa.n_items = L.n_items; aa.n_qtiles = L.n_qtiles;
   aa.scale_log2 = sm_scale * 1.4426950408889634f;
   aa.item_tile_off = pa.item_tile_off;
+  aa.item_rows = pa.item_rows;
   aa.tile_seg_off = pa.tile_seg_off;
   aa.segs = pa.segs;
   aa.queue = pa.queue;

@@ -5,21 +5,24 @@
 // size from the hardware tile size; news review, Methodology 4: ordinary
 // scaled dot-product attention over the pooled KV).
 //
-// Two persistent CTAs per SM, 6 warps each:
-//   warp 0      TMA producer.  Per 128-row KV tile: one box per (segment,
-//               64-channel chunk) of the level-l K and V maps, issued by the
-//               lane that owns the segment, plus a small record of the tile
-//               (per 16-column chunk level, or per-column bias/validity when
-//               a tile has padding, a ragged block, a causal edge or a
-//               query-half mask) in a two-deep ring.
-//   warp 1      tcgen05 issuer (one thread): S = Q K^T into TMEM, then, once
-//               the softmax has written P over S, O += P V (P read from TMEM).
+// Two persistent CTAs per SM, 6 warps each.  A work item is a 128-row query
+// tile; its KV side is the planner's list of 128-row KV tiles, processed as
+// 64-row sub-tiles so that one sub-tile's S = Q K^T runs on the tensor core
+// while the softmax works on the previous one.
+//   warp 0      TMA producer.  Per sub-tile: one box per (segment, 64-channel
+//               chunk) of the level-l K and V maps, issued by the lane that
+//               owns the segment, into two-stage K and V rings; plus a small
+//               record of the sub-tile (the level of each 16-column chunk, or
+//               a per-column bias/validity when it holds padding, a ragged
+//               block, a causal edge or a query-half mask).
+//   warp 1      tcgen05 issuer (one thread): S_j = Q K_j^T (M 128, N 64) into
+//               one of two TMEM S buffers, then O += P_{j-1} V_{j-1} with P
+//               read from TMEM.
 //   warps 2..5  softmax, one query row per thread: exp2 argument
 //               s * scale * log2(e) + l - m (the +ln 2^l bias in log2 units),
-//               lazy rescaling of O in TMEM, P as bf16 back into TMEM, and
-//               the final O / l and lse store.
-// Each CTA has one S, K and V buffer, so its own MMAs and softmax alternate;
-// the second CTA on the SM keeps the tensor core busy meanwhile.
+//               lazy rescaling of O in TMEM, P as bf16 back into the S buffer,
+//               and the final O / l and lse store.
+// TMEM per CTA: S buffers at columns [0, 64) and [64, 128), O at [128, 128+D).
 // Every wait is bounded; a time-out sets the workspace status word and
 // records where it happened.
 #include <cuda_bf16.h>
@@ -33,34 +36,47 @@ namespace psa {
 namespace {
 
 constexpr int kThreads = 192;
-// Of every 8 column pairs of a full tile, this many take their exponential
-// on the FMA pipe (exp2_fma2) instead of the special-function unit, which
-// would otherwise be the busiest unit of the softmax warps.
-constexpr int kPolyPairs = 2;
+constexpr int kSub = 64;                    // KV rows per sub-tile
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: P stays <= 2^(8+3)
+// Of every 8 column pairs of a full sub-tile, this many take their
+// exponential on the FMA pipe (exp2_fma2) instead of the special-function
+// unit.  Measured on B200 the special-function unit is not the limit of
+// this kernel, so the default is none.
+#ifndef PSA_POLY_PAIRS
+#define PSA_POLY_PAIRS 0
+#endif
+constexpr int kPolyPairs = PSA_POLY_PAIRS;
 
 struct AttnMaps {
   CUtensorMap m[9];
 };
 
-// Record of one KV tile, written by the producer for the softmax.
-struct alignas(16) TileInfo {
-  float cb[8];          // level of each 16-column chunk (fast tiles)
+// Record of one KV sub-tile, written by the producer for the softmax.
+struct alignas(16) SubInfo {
+  float cb[4];          // level of each 16-column chunk (fast sub-tiles)
   int fast;             // every column valid, no per-row check needed
-  int rowcheck;         // slow tiles: some column needs the causal / half test
-  int pad[6];
-  float bias[128];      // slow tiles: level, or -inf for padding / past-the-end rows
-  int info[128];        // slow tiles: (last covered token << 2) | query-half mask
+  int rowcheck;         // slow sub-tiles: some column needs the causal / half test
+  int pad[2];
+  float bias[kSub];     // slow sub-tiles: level, or -inf for padding / past-the-end rows
+  int info[kSub];       // slow sub-tiles: (last covered token << 2) | query-half mask
 };
 
 struct AttnShared {
-  uint64_t q_full, q_empty, k_full, k_empty, v_full, v_empty;
+  uint64_t q_full, q_empty;
+  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
   uint64_t i_full[2], i_empty[2];
-  uint64_t s_full, p_full, o_final, o_free, drain;
+  uint64_t s_full[2], p_full[2];
+  uint64_t o_ready, o_final, o_free, drain;
   uint32_t tmem_base;
   int abort;
-  TileInfo ti[2];
+  SubInfo ti[2];
 };
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
 
 // 2^x for two lanes at once on the FMA pipe, x <= 20: Cody-Waite split
 // x = n + f with n = round(x) (adding 1.5 * 2^23 rounds to an integer in the
@@ -81,15 +97,15 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
                      __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
 }
 
-// P for one tile row: p = 2^(s * sc + cb[k] - mu) per 16-column chunk k,
+// P for one sub-tile row: p = 2^(s * sc + cb[k] - mu) per 16-column chunk k,
 // packed to bf16 pairs; returns the row sum of p (fp32).
 template <int POLY>
-__device__ __forceinline__ float tile_probs(const float* s, float sc, const float (&cb)[8], float mu,
-                                            uint32_t (&pk)[64]) {
+__device__ __forceinline__ float sub_probs(const float* s, float sc, const float (&cb)[4], float mu,
+                                           uint32_t (&pk)[32]) {
   const float2 sc2 = make_float2(sc, sc);
   float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
+  for (int k = 0; k < 4; ++k) {
     const float2 off = make_float2(cb[k] - mu, cb[k] - mu);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -109,19 +125,23 @@ __device__ __forceinline__ float tile_probs(const float* s, float sc, const floa
   return t.x + t.y;
 }
 
+// number of 64-row sub-tiles of an item with `rows` real KV rows
+__device__ __forceinline__ uint32_t sub_count(int rows) { return static_cast<uint32_t>((rows + kSub - 1) / kSub); }
+
 template <int D, bool OUT_F32>
 __global__ void __launch_bounds__(kThreads, 2)
     attn_kernel(const __grid_constant__ AttnMaps maps, const AttnArgs a) {
-  constexpr int QB = D * 256;          // bytes of a 128-row tile of D bf16 channels
+  constexpr int QB = D * 256;          // bytes of the 128-row Q tile
+  constexpr int SB = D * 128;          // bytes of a 64-row K or V stage
   constexpr int KC = D / 64;           // 64-channel chunks
-  constexpr uint32_t kTmemCols = 256;  // S: columns [0,128), O: [128, 128 + D)
+  constexpr uint32_t kTmemCols = 256;
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = base;
-  uint8_t* sK = sQ + QB;
-  uint8_t* sV = sK + QB;
-  AttnShared* sh = reinterpret_cast<AttnShared*>(sV + QB);
+  uint8_t* sK = sQ + QB;               // two stages
+  uint8_t* sV = sK + 2 * SB;           // two stages
+  AttnShared* sh = reinterpret_cast<AttnShared*>(sV + 2 * SB);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int L = a.levels;
@@ -129,16 +149,17 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&sh->q_full), 1);
     mbar_init(smem_u32(&sh->q_empty), 1);
-    mbar_init(smem_u32(&sh->k_full), 1);
-    mbar_init(smem_u32(&sh->k_empty), 1);
-    mbar_init(smem_u32(&sh->v_full), 1);
-    mbar_init(smem_u32(&sh->v_empty), 1);
     for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&sh->k_full[i]), 1);
+      mbar_init(smem_u32(&sh->k_empty[i]), 1);
+      mbar_init(smem_u32(&sh->v_full[i]), 1);
+      mbar_init(smem_u32(&sh->v_empty[i]), 1);
       mbar_init(smem_u32(&sh->i_full[i]), 32);
       mbar_init(smem_u32(&sh->i_empty[i]), 128);
+      mbar_init(smem_u32(&sh->s_full[i]), 1);
+      mbar_init(smem_u32(&sh->p_full[i]), 128);
     }
-    mbar_init(smem_u32(&sh->s_full), 1);
-    mbar_init(smem_u32(&sh->p_full), 128);
+    mbar_init(smem_u32(&sh->o_ready), 1);
     mbar_init(smem_u32(&sh->o_final), 1);
     mbar_init(smem_u32(&sh->o_free), 128);
     mbar_init(smem_u32(&sh->drain), 1);
@@ -150,7 +171,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sh->tmem_base;
-  const uint32_t tS = tmem, tO = tmem + 128;
+  const uint32_t tO = tmem + 128;
   volatile int* abort = &sh->abort;
 
   if (warp == 0) {
@@ -158,17 +179,18 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (lane == 0) {
       for (int i = 0; i < 1 + 2 * L; ++i) tma_prefetch_desc(&maps.m[i]);
     }
-    uint32_t kcnt = 0, qcnt = 0;
+    uint32_t it = 0, qcnt = 0;       // it: sub-tiles loaded so far
     bool ok = true;
     for (int idx = blockIdx.x; idx < a.n_items && ok; idx += gridDim.x) {
       const int item = a.queue[idx];
       const int t0 = a.item_tile_off[item], t1 = a.item_tile_off[item + 1];
       if (t1 == t0) continue;
+      const uint32_t nsub = sub_count(a.item_rows[item]);
       const int bh = item / a.n_qtiles, tq = item - bh * a.n_qtiles;
       const int b = bh / a.Hq, h = bh - b * a.Hq;
       const int hkv = b * a.Hkv + h / (a.Hq / a.Hkv);
       const int q0 = tq * 128;
-      if (!warp_wait(smem_u32(&sh->q_empty), (qcnt & 1) ^ 1, abort, a.status, 11, idx, qcnt, kcnt, 0)) { ok = false; break; }
+      if (!warp_wait(smem_u32(&sh->q_empty), (qcnt & 1) ^ 1, abort, a.status, 11, idx, qcnt, it, 0)) { ok = false; break; }
       if (lane == 0) {
         const uint32_t bar = smem_u32(&sh->q_full);
         mbar_arrive_expect_tx(bar, QB);
@@ -176,7 +198,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int kc = 0; kc < KC; ++kc) tma_load_3d(smem_u32(sQ + kc * 16384), &maps.m[0], bar, kc * 64, q0, bh);
       }
       ++qcnt;
-      for (int t = t0; t < t1; ++t, ++kcnt) {
+      for (uint32_t j = 0; j < nsub && ok; ++j, ++it) {
+        const int t = t0 + static_cast<int>(j >> 1);
+        const int hs = static_cast<int>(j & 1);          // which 64-row half of the KV tile
         // this tile's segments: lane s owns segment s (at most 16)
         const int sb = a.tile_seg_off[t], nseg = a.tile_seg_off[t + 1] - sb;
         const int w = lane < nseg ? a.segs[sb + lane] : 0;
@@ -190,51 +214,60 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         r -= rows;
         const int nl = a.N >> l;
-        const int prow = half ? J * rows : nl;          // padding reads past the end: zeros
+        // part of the segment inside this half: rows [lo, lo + cnt) of the segment at sub-tile row dst
+        bool mine;
+        int lo, dst, cnt;
+        if (rows > kSub) { mine = lane < nseg; lo = hs * kSub; dst = 0; cnt = kSub; }
+        else { mine = lane < nseg && (r >> 6) == hs; lo = 0; dst = r - hs * kSub; cnt = rows; }
+        const int prow = (half ? J * rows : nl) + lo;   // padding reads past the end: zeros
+        const int st = it & 1;
 
         // K
-        if (!warp_wait(smem_u32(&sh->k_empty), (kcnt & 1) ^ 1, abort, a.status, 12, idx, t - t0, kcnt, 0)) { ok = false; break; }
-        if (lane == 0) mbar_arrive_expect_tx(smem_u32(&sh->k_full), QB);
+        if (!warp_wait(smem_u32(&sh->k_empty[st]), ((it >> 1) & 1) ^ 1, abort, a.status, 12, idx, j, it, 0)) { ok = false; break; }
+        if (lane == 0) mbar_arrive_expect_tx(smem_u32(&sh->k_full[st]), SB);
         __syncwarp();
-        if (lane < nseg) {
+        if (mine) {
 #pragma unroll
           for (int kc = 0; kc < KC; ++kc)
-            tma_load_3d(smem_u32(sK + kc * 16384 + r * 128), &maps.m[1 + l], smem_u32(&sh->k_full), kc * 64, prow, hkv);
+            tma_load_3d(smem_u32(sK + st * SB + kc * 8192 + dst * 128), &maps.m[1 + l], smem_u32(&sh->k_full[st]),
+                        kc * 64, prow, hkv);
         }
 
-        // tile record
-        const int slot = kcnt & 1;
-        if (!warp_wait(smem_u32(&sh->i_empty[slot]), ((kcnt >> 1) & 1) ^ 1, abort, a.status, 13, idx, t - t0, kcnt, 0)) { ok = false; break; }
-        TileInfo& ti = sh->ti[slot];
-        const int last_tok = ((J * rows + rows) << l) - 1;   // last token covered by the segment
-        const bool seg_pad = lane < nseg && half == 0;
-        const bool seg_ragged = lane < nseg && half != 0 && J * rows + rows > nl;
-        const bool seg_check = lane < nseg && half != 0 && (half != 3 || (a.causal && last_tok > q0));
+        // sub-tile record
+        if (!warp_wait(smem_u32(&sh->i_empty[st]), ((it >> 1) & 1) ^ 1, abort, a.status, 13, idx, j, it, 0)) { ok = false; break; }
+        SubInfo& ti = sh->ti[st];
+        const int p_last = J * rows + lo + cnt;                // one past the last pooled row used here
+        const int last_tok = (p_last << l) - 1;                // last token covered
+        const bool seg_pad = mine && half == 0;
+        const bool seg_ragged = mine && half != 0 && p_last > nl;
+        const bool seg_check = mine && half != 0 && (half != 3 || (a.causal && last_tok > q0));
         const bool fast = !__any_sync(0xffffffffu, seg_pad || seg_ragged || seg_check);
         const bool rowcheck = __any_sync(0xffffffffu, seg_check);
         if (fast) {
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const unsigned bal = __ballot_sync(0xffffffffu, lane < nseg && r <= 16 * k);
-            const int lev = __shfl_sync(0xffffffffu, l, __popc(bal) - 1);
+          for (int k = 0; k < 4; ++k) {
+            const unsigned bal = __ballot_sync(0xffffffffu, mine && dst <= 16 * k);
+            const int lev = __shfl_sync(0xffffffffu, l, bal ? 31 - __clz(bal) : 0);
             if (lane == k) ti.cb[k] = static_cast<float>(lev);
           }
         } else {
 #pragma unroll
-          for (int m = 0; m < 4; ++m) {
+          for (int m = 0; m < 2; ++m) {
             const int c = lane + 32 * m;
             float bias = -CUDART_INF_F;
             int inf = 0;
             for (int s = 0; s < nseg; ++s) {
-              const int rs = __shfl_sync(0xffffffffu, r, s);
+              const int ms = __shfl_sync(0xffffffffu, mine ? 1 : 0, s);
+              const int ds = __shfl_sync(0xffffffffu, dst, s);
+              const int cs = __shfl_sync(0xffffffffu, cnt, s);
+              const int los = __shfl_sync(0xffffffffu, lo, s);
               const int ws = __shfl_sync(0xffffffffu, w, s);
-              const int ls = seg_level(ws), hs = seg_half(ws), Js = seg_block(ws);
-              const int rws = a.block >> ls;
-              if (c >= rs && c < rs + rws) {
-                const int p = Js * rws + (c - rs);
-                const bool valid = hs != 0 && p < (a.N >> ls);
+              if (ms && c >= ds && c < ds + cs) {
+                const int ls = seg_level(ws), hf = seg_half(ws), Js = seg_block(ws);
+                const int p = Js * (a.block >> ls) + los + (c - ds);
+                const bool valid = hf != 0 && p < (a.N >> ls);
                 bias = valid ? static_cast<float>(ls) : -CUDART_INF_F;
-                inf = ((((p + 1) << ls) - 1) << 2) | hs;
+                inf = ((((p + 1) << ls) - 1) << 2) | hf;
               }
             }
             ti.bias[c] = bias;
@@ -242,72 +275,86 @@ __global__ void __launch_bounds__(kThreads, 2)
           }
         }
         if (lane == 0) { ti.fast = fast ? 1 : 0; ti.rowcheck = rowcheck ? 1 : 0; }
-        mbar_arrive(smem_u32(&sh->i_full[slot]));
+        mbar_arrive(smem_u32(&sh->i_full[st]));
 
         // V
-        if (!warp_wait(smem_u32(&sh->v_empty), (kcnt & 1) ^ 1, abort, a.status, 14, idx, t - t0, kcnt, 0)) { ok = false; break; }
-        if (lane == 0) mbar_arrive_expect_tx(smem_u32(&sh->v_full), QB);
+        if (!warp_wait(smem_u32(&sh->v_empty[st]), ((it >> 1) & 1) ^ 1, abort, a.status, 14, idx, j, it, 0)) { ok = false; break; }
+        if (lane == 0) mbar_arrive_expect_tx(smem_u32(&sh->v_full[st]), SB);
         __syncwarp();
-        if (lane < nseg) {
+        if (mine) {
 #pragma unroll
           for (int kc = 0; kc < KC; ++kc)
-            tma_load_3d(smem_u32(sV + kc * 16384 + r * 128), &maps.m[1 + L + l], smem_u32(&sh->v_full), kc * 64, prow, hkv);
+            tma_load_3d(smem_u32(sV + st * SB + kc * 8192 + dst * 128), &maps.m[1 + L + l], smem_u32(&sh->v_full[st]),
+                        kc * 64, prow, hkv);
         }
       }
     }
     // drain: every TMA this warp issued must land before the CTA exits
     if (lane == 0) {
       if (qcnt > 0) drain_wait(smem_u32(&sh->q_full), (qcnt - 1) & 1, a.status);
-      if (kcnt > 0) {
-        drain_wait(smem_u32(&sh->k_full), (kcnt - 1) & 1, a.status);
-        drain_wait(smem_u32(&sh->v_full), (kcnt - 1) & 1, a.status);
+      for (uint32_t st = 0; st < 2; ++st) {
+        if (it > st) {
+          drain_wait(smem_u32(&sh->k_full[st]), ((it - 1 - st) >> 1) & 1, a.status);
+          drain_wait(smem_u32(&sh->v_full[st]), ((it - 1 - st) >> 1) & 1, a.status);
+        }
       }
     }
   } else if (warp == 1) {
     // =============================== MMA issuer ===============================
     if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16_f32(128, 128, false);
+      constexpr uint32_t idS = idesc_bf16_f32(128, kSub, false);
       constexpr uint32_t idO = idesc_bf16_f32(128, D, true);
-      uint32_t kcnt = 0, qcnt = 0, icnt = 0;
+      uint32_t it = 0, qcnt = 0, icnt = 0;
       bool ok = true;
+      const uint32_t sQb = smem_u32(sQ), sKb = smem_u32(sK), sVb = smem_u32(sV);
+      // O += P_jj V_jj for sub-tile jj of the current item
+      auto issue_pv = [&](uint32_t jj, bool first_of_item) -> bool {
+        const uint32_t g = it + jj, st = g & 1;
+        if (first_of_item && icnt > 0) {
+          if (!bounded_wait(smem_u32(&sh->o_free), (icnt - 1) & 1, abort, a.status, 21, icnt, jj, g, 0)) return false;
+        }
+        if (!bounded_wait(smem_u32(&sh->p_full[st]), (g >> 1) & 1, abort, a.status, 22, icnt, jj, g, 0)) return false;
+        if (!bounded_wait(smem_u32(&sh->v_full[st]), (g >> 1) & 1, abort, a.status, 26, icnt, jj, g, 0)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < kSub / 16; ++k) {
+          umma_ts(tO, tmem + st * kSub + k * 8, sdesc_sw128(sVb + st * SB + k * 2048, 8192, 1024), idO,
+                  (first_of_item && k == 0) ? 0u : 1u);
+        }
+        umma_commit(smem_u32(&sh->v_empty[st]));
+        umma_commit(smem_u32(&sh->o_ready));
+        return true;
+      };
       for (int idx = blockIdx.x; idx < a.n_items && ok; idx += gridDim.x) {
         const int item = a.queue[idx];
         const int t0 = a.item_tile_off[item], t1 = a.item_tile_off[item + 1];
-        const uint32_t n = static_cast<uint32_t>(t1 - t0);
-        if (n == 0) continue;
-        if (!bounded_wait(smem_u32(&sh->q_full), qcnt & 1, abort, a.status, 23, idx, qcnt, kcnt, 0)) { ok = false; break; }
+        if (t1 == t0) continue;
+        const uint32_t n = sub_count(a.item_rows[item]);
+        if (!bounded_wait(smem_u32(&sh->q_full), qcnt & 1, abort, a.status, 23, idx, qcnt, it, 0)) { ok = false; break; }
         tc_fence_after();
         ++qcnt;
-        const uint32_t sQb = smem_u32(sQ), sKb = smem_u32(sK), sVb = smem_u32(sV);
-        for (uint32_t j = 0; j < n; ++j, ++kcnt) {
-          // S = Q K^T
-          if (!bounded_wait(smem_u32(&sh->k_full), kcnt & 1, abort, a.status, 24, idx, j, kcnt, 0)) { ok = false; break; }
+        for (uint32_t j = 0; j < n && ok; ++j) {
+          const uint32_t g = it + j, st = g & 1;
+          // S_j = Q K_j^T into S buffer st
+          if (!bounded_wait(smem_u32(&sh->k_full[st]), (g >> 1) & 1, abort, a.status, 24, idx, j, g, 0)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int kc = 0; kc < KC; ++kc) {
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              umma_ss(tS, sdesc_sw128(sQb + kc * 16384 + 32 * k, 16, 1024),
-                      sdesc_sw128(sKb + kc * 16384 + 32 * k, 16, 1024), idS, (kc | k) != 0);
+              umma_ss(tmem + st * kSub, sdesc_sw128(sQb + kc * 16384 + 32 * k, 16, 1024),
+                      sdesc_sw128(sKb + st * SB + kc * 8192 + 32 * k, 16, 1024), idS, (kc | k) != 0);
             }
           }
-          umma_commit(smem_u32(&sh->s_full));
-          umma_commit(smem_u32(&sh->k_empty));
+          umma_commit(smem_u32(&sh->s_full[st]));
+          umma_commit(smem_u32(&sh->k_empty[st]));
           if (j + 1 == n) umma_commit(smem_u32(&sh->q_empty));
-          // O += P V, once the softmax has written P
-          if (!bounded_wait(smem_u32(&sh->p_full), kcnt & 1, abort, a.status, 25, idx, j, kcnt, 0)) { ok = false; break; }
-          if (j == 0 && icnt > 0) {
-            if (!bounded_wait(smem_u32(&sh->o_free), (icnt - 1) & 1, abort, a.status, 21, idx, icnt, kcnt, 0)) { ok = false; break; }
-          }
-          if (!bounded_wait(smem_u32(&sh->v_full), kcnt & 1, abort, a.status, 26, idx, j, kcnt, 0)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            umma_ts(tO, tS + k * 8, sdesc_sw128(sVb + k * 2048, 16384, 1024), idO, (j == 0 && k == 0) ? 0u : 1u);
-          }
-          umma_commit(smem_u32(&sh->v_empty));
-          if (j + 1 == n) umma_commit(smem_u32(&sh->o_final));
+          if (j >= 1 && !issue_pv(j - 1, j == 1)) { ok = false; break; }
         }
+        if (!ok) break;
+        if (!issue_pv(n - 1, n == 1)) { ok = false; break; }
+        umma_commit(smem_u32(&sh->o_final));
+        it += n;
         ++icnt;
       }
       umma_commit(smem_u32(&sh->drain));
@@ -319,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int row = q * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     const int my_half_bit = 1 << (row >> 6);
-    uint32_t kcnt = 0, icnt = 0;
+    uint32_t it = 0, icnt = 0;
     bool ok = true;
     for (int idx = blockIdx.x; idx < a.n_items && ok; idx += gridDim.x) {
       const int item = a.queue[idx];
@@ -327,8 +374,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int bh = item / a.n_qtiles, tq = item - bh * a.n_qtiles;
       const int tok = tq * 128 + row;
       const int64_t orow = static_cast<int64_t>(bh) * a.N + tok;
-      const int n = t1 - t0;
-      if (n == 0) {
+      if (t1 == t0) {
         if (tok < a.N) {
           if (OUT_F32) {
             float4* o = reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow * D);
@@ -341,41 +387,42 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         continue;
       }
+      const uint32_t n = sub_count(a.item_rows[item]);
       float m = -CUDART_INF_F, lsum = 0.f;
-      for (int j = 0; j < n; ++j, ++kcnt) {
-        const int slot = kcnt & 1;
-        if (!warp_wait(smem_u32(&sh->s_full), kcnt & 1, abort, a.status, 31, idx, j, kcnt, 0)) { ok = false; break; }
-        if (!warp_wait(smem_u32(&sh->i_full[slot]), (kcnt >> 1) & 1, abort, a.status, 32, idx, j, kcnt, 0)) { ok = false; break; }
+      for (uint32_t j = 0; j < n; ++j, ++it) {
+        const uint32_t st = it & 1;
+        if (!warp_wait(smem_u32(&sh->s_full[st]), (it >> 1) & 1, abort, a.status, 31, idx, j, it, 0)) { ok = false; break; }
+        if (!warp_wait(smem_u32(&sh->i_full[st]), (it >> 1) & 1, abort, a.status, 32, idx, j, it, 0)) { ok = false; break; }
         tc_fence_after();
-        const TileInfo& ti = sh->ti[slot];
-        uint32_t sr[128];
-        tmem_ld128(tS + lane_off, sr);
-        float* s = reinterpret_cast<float*>(sr);
+        const SubInfo& ti = sh->ti[st];
+        uint32_t sr[32], sr2[32];
+        tmem_ld32(tmem + st * kSub + lane_off, sr);
+        tmem_ld32(tmem + st * kSub + 32 + lane_off, sr2);
+        float s[kSub];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) { s[i] = __uint_as_float(sr[i]); s[32 + i] = __uint_as_float(sr2[i]); }
         // exp2 argument of column c in chunk k: s[c] * sc + cb[k] - m
         float sc = a.scale_log2;
-        float cb[8];
+        float cb[4];
         float mt;
         const bool fast_tile = ti.fast != 0;
         if (fast_tile) {
+          const float4 c4 = *reinterpret_cast<const float4*>(ti.cb);
+          cb[0] = c4.x; cb[1] = c4.y; cb[2] = c4.z; cb[3] = c4.w;
+          float cmax[4];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) cb[k] = ti.cb[k];
-          float cmax[8];
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            float x0 = fmaxf(s[16 * k + 0], s[16 * k + 1]), x1 = fmaxf(s[16 * k + 2], s[16 * k + 3]);
-            float x2 = fmaxf(s[16 * k + 4], s[16 * k + 5]), x3 = fmaxf(s[16 * k + 6], s[16 * k + 7]);
-            float x4 = fmaxf(s[16 * k + 8], s[16 * k + 9]), x5 = fmaxf(s[16 * k + 10], s[16 * k + 11]);
-            float x6 = fmaxf(s[16 * k + 12], s[16 * k + 13]), x7 = fmaxf(s[16 * k + 14], s[16 * k + 15]);
-            x0 = fmaxf(x0, x1); x2 = fmaxf(x2, x3); x4 = fmaxf(x4, x5); x6 = fmaxf(x6, x7);
-            cmax[k] = fmaf(fmaxf(fmaxf(x0, x2), fmaxf(x4, x6)), sc, cb[k]);
+          for (int k = 0; k < 4; ++k) {
+            const float* x = s + 16 * k;
+            const float y0 = fmax3(x[0], x[1], x[2]), y1 = fmax3(x[3], x[4], x[5]), y2 = fmax3(x[6], x[7], x[8]);
+            const float y3 = fmax3(x[9], x[10], x[11]), y4 = fmax3(x[12], x[13], x[14]);
+            cmax[k] = fmaf(fmax3(fmax3(y0, y1, y2), fmax3(y3, y4, x[15]), y0), sc, cb[k]);
           }
-          mt = fmaxf(fmaxf(fmaxf(cmax[0], cmax[1]), fmaxf(cmax[2], cmax[3])),
-                     fmaxf(fmaxf(cmax[4], cmax[5]), fmaxf(cmax[6], cmax[7])));
+          mt = fmaxf(fmaxf(cmax[0], cmax[1]), fmaxf(cmax[2], cmax[3]));
         } else {
           // per-column bias (padding, ragged tails) and, if needed, the
           // causal / query-half test; afterwards s holds the full argument
 #pragma unroll
-          for (int c4 = 0; c4 < 32; ++c4) {
+          for (int c4 = 0; c4 < kSub / 4; ++c4) {
             const float4 bv = *reinterpret_cast<const float4*>(&ti.bias[4 * c4]);
             s[4 * c4 + 0] = fmaf(s[4 * c4 + 0], sc, bv.x);
             s[4 * c4 + 1] = fmaf(s[4 * c4 + 1], sc, bv.y);
@@ -384,7 +431,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           }
           if (ti.rowcheck) {
 #pragma unroll
-            for (int c4 = 0; c4 < 32; ++c4) {
+            for (int c4 = 0; c4 < kSub / 4; ++c4) {
               const int4 iv = *reinterpret_cast<const int4*>(&ti.info[4 * c4]);
               const int iw[4] = {iv.x, iv.y, iv.z, iv.w};
 #pragma unroll
@@ -396,32 +443,36 @@ __global__ void __launch_bounds__(kThreads, 2)
           }
           sc = 1.0f;
 #pragma unroll
-          for (int k = 0; k < 8; ++k) cb[k] = 0.f;
+          for (int k = 0; k < 4; ++k) cb[k] = 0.f;
           float x[8];
 #pragma unroll
-          for (int u = 0; u < 8; ++u) x[u] = s[u];
+          for (int u = 0; u < 8; ++u) x[u] = fmax3(s[u], s[8 + u], s[16 + u]);
 #pragma unroll
-          for (int c = 8; c < 128; c += 8) {
+          for (int c = 24; c < kSub; c += 16) {
 #pragma unroll
-            for (int u = 0; u < 8; ++u) x[u] = fmaxf(x[u], s[c + u]);
+            for (int u = 0; u < 8; ++u) x[u] = fmax3(x[u], s[c + u], c + 8 + u < kSub ? s[c + 8 + u] : x[u]);
           }
-          mt = fmaxf(fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3])), fmaxf(fmaxf(x[4], x[5]), fmaxf(x[6], x[7])));
+          mt = fmaxf(fmax3(x[0], x[1], x[2]), fmax3(fmax3(x[3], x[4], x[5]), x[6], x[7]));
         }
-        // the tile record may be reused once read
-        mbar_arrive(smem_u32(&sh->i_empty[slot]));
+        // the sub-tile record may be reused once read
+        mbar_arrive(smem_u32(&sh->i_empty[st]));
 
         const float mnew = fmaxf(m, mt);
         // Lazy rescaling: a row moves its reference max only when the new max
         // exceeds it by more than kRescaleThreshold (or on its first visible
         // key).  O is read and written with warp-collective tcgen05.ld/st, so
-        // the decision to touch O is taken per warp.  The PV of the previous
-        // tile is complete: its commit preceded this tile's S.
+        // the decision to touch O is taken per warp, after the PV of the
+        // previous sub-tile is done (o_ready: PV_{j-2} completed before S_j,
+        // PV_j waits for this sub-tile's P, so the awaited phase is one of
+        // the two the barrier can be in).
         const bool first = m == -CUDART_INF_F && mnew != -CUDART_INF_F;
         const bool grow = m != -CUDART_INF_F && mnew > m + kRescaleThreshold;
         if (__any_sync(0xffffffffu, grow)) {
           const float f = grow ? fast_exp2(m - mnew) : 1.0f;
           lsum *= f;
           if (grow) m = mnew;
+          if (!warp_wait(smem_u32(&sh->o_ready), (it - 1) & 1, abort, a.status, 33, idx, j, it, 0)) { ok = false; break; }
+          tc_fence_after();
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
@@ -433,20 +484,20 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         if (first) m = mnew;
         const float mu = m == -CUDART_INF_F ? 0.f : m;
-        uint32_t pk[64];
-        // full tiles split the exponentials between MUFU and the FMA pipe;
-        // tiles with masked columns (p must be exactly 0 there) use MUFU only
-        lsum += fast_tile ? tile_probs<kPolyPairs>(s, sc, cb, mu, pk) : tile_probs<0>(s, sc, cb, mu, pk);
-        tmem_st64(tS + lane_off, pk);
+        uint32_t pk[32];
+        // sub-tiles with masked columns (p must be exactly 0 there) use the
+        // special-function unit only
+        lsum += fast_tile ? sub_probs<kPolyPairs>(s, sc, cb, mu, pk) : sub_probs<0>(s, sc, cb, mu, pk);
+        tmem_st32(tmem + st * kSub + lane_off, pk);
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(smem_u32(&sh->p_full));
+        mbar_arrive(smem_u32(&sh->p_full[st]));
       }
       if (!ok) break;
       // epilogue: O / l once the item's last PV is done (o_final completes
       // once per item and cannot run ahead: the next item's first PV waits
       // for o_free)
-      if (!warp_wait(smem_u32(&sh->o_final), icnt & 1, abort, a.status, 35, idx, n, kcnt, icnt)) { ok = false; break; }
+      if (!warp_wait(smem_u32(&sh->o_final), icnt & 1, abort, a.status, 35, idx, n, it, icnt)) { ok = false; break; }
       ++icnt;
       tc_fence_after();
       const float inv = lsum > 0.f ? 1.0f / lsum : 0.f;
@@ -493,7 +544,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 
 template <int D, bool F32>
 cudaError_t launch_one(const AttnMaps& maps, const AttnArgs& a, int num_sms, cudaStream_t s) {
-  const size_t smem = 1024 + static_cast<size_t>(D) * 256 * 3 + sizeof(AttnShared);
+  const size_t smem = 1024 + static_cast<size_t>(D) * 256 + 4 * static_cast<size_t>(D) * 128 + sizeof(AttnShared);
   cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, F32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;

@@ -79,6 +79,7 @@ struct AttnArgs {
   int n_items, n_qtiles;  // n_qtiles = ceil(N/128) per head
   float scale_log2;       // sm_scale * log2(e)
   const int* item_tile_off;
+  const int* item_rows;   // real KV rows per item (sub-tiles = ceil(rows / 64))
   const int* tile_seg_off;
   const int* segs;
   const int* queue;
@@ -88,7 +89,7 @@ struct AttnArgs {
   int* status;
 };
 // maps: [0] = Q (3D view [d, N, B*Hq], box 64 x 128), [1 + l] = K level l,
-// [1 + L + l] = V level l (3D views [d, N/2^l, B*Hkv], box 64 x block/2^l).
+// [1 + L + l] = V level l (3D views [d, N/2^l, B*Hkv], box 64 x min(block/2^l, 64)).
 cudaError_t launch_attention(const CUtensorMap* maps, const AttnArgs& a, int num_sms,
                              cudaStream_t s);
 

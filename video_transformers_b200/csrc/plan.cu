@@ -9,9 +9,9 @@
 // list of non-skipped (J, level) segments, each blk / 2^l pooled rows.  The
 // planner orders the segments by level (so sizes descend through powers of
 // two) and cuts the list into 128-row KV tiles; with that order no segment
-// straddles a tile edge and every segment starts on an 8-row boundary.
-// Only the last tile of an item can be partly empty; it is filled with
-// padding segments that read zeros.
+// straddles a tile edge (or the 64-row half of a tile) and every segment
+// starts on a multiple of its own size.  Only the last tile of an item can be
+// partly empty; it is filled with padding segments that read zeros.
 //
 // plan_count (warp per item) -> plan_scan (one CTA) -> plan_fill (warp per
 // item).  The queue is either head-major (items in their natural order, so
@@ -66,14 +66,24 @@ __device__ __forceinline__ int seg_halves(const PlanArgs& a, const ItemGeom& g, 
   return half;
 }
 
-// padding decomposition of `rem` rows into the available box sizes
-__device__ __forceinline__ int pad_count(int rem, int block, int levels) {
+// Padding of the last tile: from row `pos` up to the next multiple of 128,
+// each pad as large as the alignment of its start allows (the lowest set bit
+// of pos, at most 64), so every pad is aligned to its own size and none
+// crosses a 64-row boundary.  pos is a multiple of the smallest segment, so
+// every pad size is one of the available box sizes.
+__device__ __forceinline__ int pad_size(int pos) {
+  const int low = pos & -pos;
+  return low < 64 ? low : 64;
+}
+__device__ __forceinline__ int pad_count(int pos) {
   int n = 0;
-  for (int l = 0; l < levels; ++l) {
-    const int sz = block >> l;
-    while (sz <= 128 && rem >= sz) { rem -= sz; ++n; }
-  }
+  while (pos & 127) { pos += pad_size(pos); ++n; }
   return n;
+}
+__device__ __forceinline__ int level_of_rows(int block, int rows) {
+  int l = 0;
+  while ((block >> l) > rows) ++l;
+  return l;
 }
 
 __global__ void plan_count(const PlanArgs a) {
@@ -90,8 +100,7 @@ __global__ void plan_count(const PlanArgs a) {
     rows += c * (a.block >> l);
   }
   const int ntile = (rows + 127) / 128;
-  const int rem = ntile * 128 - rows;
-  const int npad = pad_count(rem, a.block, a.levels);
+  const int npad = pad_count(rows);
   if (lane == 0) {
     a.item_nseg[warp] = nseg + npad;
     a.item_ntile[warp] = ntile;
@@ -186,14 +195,12 @@ __global__ void plan_fill(const PlanArgs a) {
     }
   }
   if (lane == 0) {
-    int rem = ntile * 128 - row;
-    for (int l = 0; l < a.levels; ++l) {
-      const int sz = a.block >> l;
-      while (sz <= 128 && rem >= sz) {
-        a.segs[seg_base + k] = make_seg(0, l, 0);
-        ++k;
-        rem -= sz;
-      }
+    int pos = row;
+    while (pos & 127) {
+      const int sz = pad_size(pos);
+      a.segs[seg_base + k] = make_seg(0, level_of_rows(a.block, sz), 0);
+      ++k;
+      pos += sz;
     }
     if (a.lpt_queue) {
       const int bin = min(ntile, a.n_hist - 1);
