@@ -198,21 +198,34 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int kc = 0; kc < KC; ++kc) tma_load_3d(smem_u32(sQ + kc * 16384), &maps.m[0], bar, kc * 64, q0, bh);
       }
       ++qcnt;
+      // V loads run one sub-tile behind the K loads: V_j is needed only after
+      // the softmax of sub-tile j, while K_{j+1} is needed right after S_j.
+      bool pv_mine = false;
+      int pv_l = 0, pv_dst = 0, pv_prow = 0;
+      // segment words of the current tile, and of the next one (prefetched)
+      int sb = a.tile_seg_off[t0], nseg = a.tile_seg_off[t0 + 1] - sb;
+      int w = lane < nseg ? a.segs[sb + lane] : 0;
+      int nb = 0, nn = 0, wn = 0;
+      int l = 0, half = 0, J = 0, rows = 0, r = 0;
       for (uint32_t j = 0; j < nsub && ok; ++j, ++it) {
         const int t = t0 + static_cast<int>(j >> 1);
         const int hs = static_cast<int>(j & 1);          // which 64-row half of the KV tile
-        // this tile's segments: lane s owns segment s (at most 16)
-        const int sb = a.tile_seg_off[t], nseg = a.tile_seg_off[t + 1] - sb;
-        const int w = lane < nseg ? a.segs[sb + lane] : 0;
-        const int l = seg_level(w), half = seg_half(w), J = seg_block(w);
-        const int rows = lane < nseg ? (a.block >> l) : 0;
-        int r = rows;                                   // inclusive scan -> exclusive row offset
+        if (hs == 0) {
+          if (j > 0) { sb = nb; nseg = nn; w = wn; }
+          // this tile's segments: lane s owns segment s (at most 16)
+          l = seg_level(w); half = seg_half(w); J = seg_block(w);
+          rows = lane < nseg ? (a.block >> l) : 0;
+          r = rows;                                     // inclusive scan -> exclusive row offset
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_up_sync(0xffffffffu, r, o);
-          if (lane >= o) r += y;
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, r, o);
+            if (lane >= o) r += y;
+          }
+          r -= rows;
+          if (t + 1 < t1) { nb = a.tile_seg_off[t + 1]; nn = a.tile_seg_off[t + 2] - nb; }
+        } else if (t + 1 < t1) {
+          wn = lane < nn ? a.segs[nb + lane] : 0;
         }
-        r -= rows;
         const int nl = a.N >> l;
         // part of the segment inside this half: rows [lo, lo + cnt) of the segment at sub-tile row dst
         bool mine;
@@ -277,15 +290,32 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (lane == 0) { ti.fast = fast ? 1 : 0; ti.rowcheck = rowcheck ? 1 : 0; }
         mbar_arrive(smem_u32(&sh->i_full[st]));
 
-        // V
-        if (!warp_wait(smem_u32(&sh->v_empty[st]), ((it >> 1) & 1) ^ 1, abort, a.status, 14, idx, j, it, 0)) { ok = false; break; }
-        if (lane == 0) mbar_arrive_expect_tx(smem_u32(&sh->v_full[st]), SB);
+        // V of the previous sub-tile
+        if (j > 0) {
+          const uint32_t pst = (it - 1) & 1;
+          if (!warp_wait(smem_u32(&sh->v_empty[pst]), (((it - 1) >> 1) & 1) ^ 1, abort, a.status, 14, idx, j, it, 0)) { ok = false; break; }
+          if (lane == 0) mbar_arrive_expect_tx(smem_u32(&sh->v_full[pst]), SB);
+          __syncwarp();
+          if (pv_mine) {
+#pragma unroll
+            for (int kc = 0; kc < KC; ++kc)
+              tma_load_3d(smem_u32(sV + pst * SB + kc * 8192 + pv_dst * 128), &maps.m[1 + L + pv_l],
+                          smem_u32(&sh->v_full[pst]), kc * 64, pv_prow, hkv);
+          }
+        }
+        pv_mine = mine; pv_l = l; pv_dst = dst; pv_prow = prow;
+      }
+      // V of the item's last sub-tile
+      if (ok) {
+        const uint32_t pst = (it - 1) & 1;
+        if (!warp_wait(smem_u32(&sh->v_empty[pst]), (((it - 1) >> 1) & 1) ^ 1, abort, a.status, 15, idx, 0, it, 0)) { ok = false; break; }
+        if (lane == 0) mbar_arrive_expect_tx(smem_u32(&sh->v_full[pst]), SB);
         __syncwarp();
-        if (mine) {
+        if (pv_mine) {
 #pragma unroll
           for (int kc = 0; kc < KC; ++kc)
-            tma_load_3d(smem_u32(sV + st * SB + kc * 8192 + dst * 128), &maps.m[1 + L + l], smem_u32(&sh->v_full[st]),
-                        kc * 64, prow, hkv);
+            tma_load_3d(smem_u32(sV + pst * SB + kc * 8192 + pv_dst * 128), &maps.m[1 + L + pv_l],
+                        smem_u32(&sh->v_full[pst]), kc * 64, pv_prow, hkv);
         }
       }
     }
@@ -306,7 +336,11 @@ __global__ void __launch_bounds__(kThreads, 2)
       constexpr uint32_t idO = idesc_bf16_f32(128, D, true);
       uint32_t it = 0, qcnt = 0, icnt = 0;
       bool ok = true;
-      const uint32_t sQb = smem_u32(sQ), sKb = smem_u32(sK), sVb = smem_u32(sV);
+      // shared-memory descriptors of the tile bases; a K step or stage is an
+      // offset added to the start-address field (all of smem is < 256 KB)
+      const uint64_t dQ = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dK = sdesc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t dV = sdesc_sw128(smem_u32(sV), 8192, 1024);
       // O += P_jj V_jj for sub-tile jj of the current item
       auto issue_pv = [&](uint32_t jj, bool first_of_item) -> bool {
         const uint32_t g = it + jj, st = g & 1;
@@ -318,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < kSub / 16; ++k) {
-          umma_ts(tO, tmem + st * kSub + k * 8, sdesc_sw128(sVb + st * SB + k * 2048, 8192, 1024), idO,
+          umma_ts(tO, tmem + st * kSub + k * 8, dV + ((st * SB + k * 2048) >> 4), idO,
                   (first_of_item && k == 0) ? 0u : 1u);
         }
         umma_commit(smem_u32(&sh->v_empty[st]));
@@ -342,8 +376,8 @@ __global__ void __launch_bounds__(kThreads, 2)
           for (int kc = 0; kc < KC; ++kc) {
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              umma_ss(tmem + st * kSub, sdesc_sw128(sQb + kc * 16384 + 32 * k, 16, 1024),
-                      sdesc_sw128(sKb + st * SB + kc * 8192 + 32 * k, 16, 1024), idS, (kc | k) != 0);
+              umma_ss(tmem + st * kSub, dQ + ((kc * 16384 + 32 * k) >> 4),
+                      dK + ((st * SB + kc * 8192 + 32 * k) >> 4), idS, (kc | k) != 0);
             }
           }
           umma_commit(smem_u32(&sh->s_full[st]));
