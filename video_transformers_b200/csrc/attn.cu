@@ -61,15 +61,17 @@ struct alignas(16) SubInfo {
   int info[kSub];       // slow sub-tiles: (last covered token << 2) | query-half mask
 };
 
+// NST: depth of the K, V and sub-tile-record rings
+template <int NST>
 struct AttnShared {
   uint64_t q_full, q_empty;
-  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
-  uint64_t i_full[2], i_empty[2];
+  uint64_t k_full[NST], k_empty[NST], v_full[NST], v_empty[NST];
+  uint64_t i_full[NST], i_empty[NST];
   uint64_t s_full[2], p_full[2];
   uint64_t o_ready, o_final, o_free, drain;
   uint32_t tmem_base;
   int abort;
-  SubInfo ti[2];
+  SubInfo ti[NST];
 };
 
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -128,20 +130,21 @@ __device__ __forceinline__ float sub_probs(const float* s, float sc, const float
 // number of 64-row sub-tiles of an item with `rows` real KV rows
 __device__ __forceinline__ uint32_t sub_count(int rows) { return static_cast<uint32_t>((rows + kSub - 1) / kSub); }
 
-template <int D, bool OUT_F32>
-__global__ void __launch_bounds__(kThreads, 2)
+template <int D, bool OUT_F32, int NST, int CTAS>
+__global__ void __launch_bounds__(kThreads, CTAS)
     attn_kernel(const __grid_constant__ AttnMaps maps, const AttnArgs a) {
   constexpr int QB = D * 256;          // bytes of the 128-row Q tile
   constexpr int SB = D * 128;          // bytes of a 64-row K or V stage
   constexpr int KC = D / 64;           // 64-channel chunks
   constexpr uint32_t kTmemCols = 256;
+  using Shared = AttnShared<NST>;
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = base;
-  uint8_t* sK = sQ + QB;               // two stages
-  uint8_t* sV = sK + 2 * SB;           // two stages
-  AttnShared* sh = reinterpret_cast<AttnShared*>(sV + 2 * SB);
+  uint8_t* sK = sQ + QB;               // NST stages
+  uint8_t* sV = sK + NST * SB;         // NST stages
+  Shared* sh = reinterpret_cast<Shared*>(sV + NST * SB);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int L = a.levels;
@@ -149,13 +152,15 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&sh->q_full), 1);
     mbar_init(smem_u32(&sh->q_empty), 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NST; ++i) {
       mbar_init(smem_u32(&sh->k_full[i]), 1);
       mbar_init(smem_u32(&sh->k_empty[i]), 1);
       mbar_init(smem_u32(&sh->v_full[i]), 1);
       mbar_init(smem_u32(&sh->v_empty[i]), 1);
       mbar_init(smem_u32(&sh->i_full[i]), 32);
       mbar_init(smem_u32(&sh->i_empty[i]), 128);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&sh->s_full[i]), 1);
       mbar_init(smem_u32(&sh->p_full[i]), 128);
     }
@@ -233,10 +238,11 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (rows > kSub) { mine = lane < nseg; lo = hs * kSub; dst = 0; cnt = kSub; }
         else { mine = lane < nseg && (r >> 6) == hs; lo = 0; dst = r - hs * kSub; cnt = rows; }
         const int prow = (half ? J * rows : nl) + lo;   // padding reads past the end: zeros
-        const int st = it & 1;
+        const int st = it % NST;
+        const uint32_t ph = (it / NST) & 1;
 
         // K
-        if (!warp_wait(smem_u32(&sh->k_empty[st]), ((it >> 1) & 1) ^ 1, abort, a.status, 12, idx, j, it, 0)) { ok = false; break; }
+        if (!warp_wait(smem_u32(&sh->k_empty[st]), ph ^ 1, abort, a.status, 12, idx, j, it, 0)) { ok = false; break; }
         if (lane == 0) mbar_arrive_expect_tx(smem_u32(&sh->k_full[st]), SB);
         __syncwarp();
         if (mine) {
@@ -247,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
 
         // sub-tile record
-        if (!warp_wait(smem_u32(&sh->i_empty[st]), ((it >> 1) & 1) ^ 1, abort, a.status, 13, idx, j, it, 0)) { ok = false; break; }
+        if (!warp_wait(smem_u32(&sh->i_empty[st]), ph ^ 1, abort, a.status, 13, idx, j, it, 0)) { ok = false; break; }
         SubInfo& ti = sh->ti[st];
         const int p_last = J * rows + lo + cnt;                // one past the last pooled row used here
         const int last_tok = (p_last << l) - 1;                // last token covered
@@ -292,8 +298,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 
         // V of the previous sub-tile
         if (j > 0) {
-          const uint32_t pst = (it - 1) & 1;
-          if (!warp_wait(smem_u32(&sh->v_empty[pst]), (((it - 1) >> 1) & 1) ^ 1, abort, a.status, 14, idx, j, it, 0)) { ok = false; break; }
+          const uint32_t pst = (it - 1) % NST;
+          if (!warp_wait(smem_u32(&sh->v_empty[pst]), (((it - 1) / NST) & 1) ^ 1, abort, a.status, 14, idx, j, it, 0)) { ok = false; break; }
           if (lane == 0) mbar_arrive_expect_tx(smem_u32(&sh->v_full[pst]), SB);
           __syncwarp();
           if (pv_mine) {
@@ -307,8 +313,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       // V of the item's last sub-tile
       if (ok) {
-        const uint32_t pst = (it - 1) & 1;
-        if (!warp_wait(smem_u32(&sh->v_empty[pst]), (((it - 1) >> 1) & 1) ^ 1, abort, a.status, 15, idx, 0, it, 0)) { ok = false; break; }
+        const uint32_t pst = (it - 1) % NST;
+        if (!warp_wait(smem_u32(&sh->v_empty[pst]), (((it - 1) / NST) & 1) ^ 1, abort, a.status, 15, idx, 0, it, 0)) { ok = false; break; }
         if (lane == 0) mbar_arrive_expect_tx(smem_u32(&sh->v_full[pst]), SB);
         __syncwarp();
         if (pv_mine) {
@@ -322,10 +328,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     // drain: every TMA this warp issued must land before the CTA exits
     if (lane == 0) {
       if (qcnt > 0) drain_wait(smem_u32(&sh->q_full), (qcnt - 1) & 1, a.status);
-      for (uint32_t st = 0; st < 2; ++st) {
+      for (uint32_t st = 0; st < static_cast<uint32_t>(NST); ++st) {
         if (it > st) {
-          drain_wait(smem_u32(&sh->k_full[st]), ((it - 1 - st) >> 1) & 1, a.status);
-          drain_wait(smem_u32(&sh->v_full[st]), ((it - 1 - st) >> 1) & 1, a.status);
+          drain_wait(smem_u32(&sh->k_full[st]), ((it - 1 - st) / NST) & 1, a.status);
+          drain_wait(smem_u32(&sh->v_full[st]), ((it - 1 - st) / NST) & 1, a.status);
         }
       }
     }
@@ -343,16 +349,16 @@ __global__ void __launch_bounds__(kThreads, 2)
       const uint64_t dV = sdesc_sw128(smem_u32(sV), 8192, 1024);
       // O += P_jj V_jj for sub-tile jj of the current item
       auto issue_pv = [&](uint32_t jj, bool first_of_item) -> bool {
-        const uint32_t g = it + jj, st = g & 1;
+        const uint32_t g = it + jj, st = g % NST, sb2 = g & 1;
         if (first_of_item && icnt > 0) {
           if (!bounded_wait(smem_u32(&sh->o_free), (icnt - 1) & 1, abort, a.status, 21, icnt, jj, g, 0)) return false;
         }
-        if (!bounded_wait(smem_u32(&sh->p_full[st]), (g >> 1) & 1, abort, a.status, 22, icnt, jj, g, 0)) return false;
-        if (!bounded_wait(smem_u32(&sh->v_full[st]), (g >> 1) & 1, abort, a.status, 26, icnt, jj, g, 0)) return false;
+        if (!bounded_wait(smem_u32(&sh->p_full[sb2]), (g >> 1) & 1, abort, a.status, 22, icnt, jj, g, 0)) return false;
+        if (!bounded_wait(smem_u32(&sh->v_full[st]), (g / NST) & 1, abort, a.status, 26, icnt, jj, g, 0)) return false;
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < kSub / 16; ++k) {
-          umma_ts(tO, tmem + st * kSub + k * 8, dV + ((st * SB + k * 2048) >> 4), idO,
+          umma_ts(tO, tmem + sb2 * kSub + k * 8, dV + ((st * SB + k * 2048) >> 4), idO,
                   (first_of_item && k == 0) ? 0u : 1u);
         }
         umma_commit(smem_u32(&sh->v_empty[st]));
@@ -368,19 +374,19 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc_fence_after();
         ++qcnt;
         for (uint32_t j = 0; j < n && ok; ++j) {
-          const uint32_t g = it + j, st = g & 1;
-          // S_j = Q K_j^T into S buffer st
-          if (!bounded_wait(smem_u32(&sh->k_full[st]), (g >> 1) & 1, abort, a.status, 24, idx, j, g, 0)) { ok = false; break; }
+          const uint32_t g = it + j, st = g % NST, sb2 = g & 1;
+          // S_j = Q K_j^T into S buffer sb2
+          if (!bounded_wait(smem_u32(&sh->k_full[st]), (g / NST) & 1, abort, a.status, 24, idx, j, g, 0)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int kc = 0; kc < KC; ++kc) {
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              umma_ss(tmem + st * kSub, dQ + ((kc * 16384 + 32 * k) >> 4),
+              umma_ss(tmem + sb2 * kSub, dQ + ((kc * 16384 + 32 * k) >> 4),
                       dK + ((st * SB + kc * 8192 + 32 * k) >> 4), idS, (kc | k) != 0);
             }
           }
-          umma_commit(smem_u32(&sh->s_full[st]));
+          umma_commit(smem_u32(&sh->s_full[sb2]));
           umma_commit(smem_u32(&sh->k_empty[st]));
           if (j + 1 == n) umma_commit(smem_u32(&sh->q_empty));
           if (j >= 1 && !issue_pv(j - 1, j == 1)) { ok = false; break; }
@@ -424,14 +430,14 @@ __global__ void __launch_bounds__(kThreads, 2)
       const uint32_t n = sub_count(a.item_rows[item]);
       float m = -CUDART_INF_F, lsum = 0.f;
       for (uint32_t j = 0; j < n; ++j, ++it) {
-        const uint32_t st = it & 1;
-        if (!warp_wait(smem_u32(&sh->s_full[st]), (it >> 1) & 1, abort, a.status, 31, idx, j, it, 0)) { ok = false; break; }
-        if (!warp_wait(smem_u32(&sh->i_full[st]), (it >> 1) & 1, abort, a.status, 32, idx, j, it, 0)) { ok = false; break; }
+        const uint32_t st = it % NST, sb2 = it & 1;
+        if (!warp_wait(smem_u32(&sh->s_full[sb2]), (it >> 1) & 1, abort, a.status, 31, idx, j, it, 0)) { ok = false; break; }
+        if (!warp_wait(smem_u32(&sh->i_full[st]), (it / NST) & 1, abort, a.status, 32, idx, j, it, 0)) { ok = false; break; }
         tc_fence_after();
         const SubInfo& ti = sh->ti[st];
         uint32_t sr[32], sr2[32];
-        tmem_ld32(tmem + st * kSub + lane_off, sr);
-        tmem_ld32(tmem + st * kSub + 32 + lane_off, sr2);
+        tmem_ld32(tmem + sb2 * kSub + lane_off, sr);
+        tmem_ld32(tmem + sb2 * kSub + 32 + lane_off, sr2);
         float s[kSub];
 #pragma unroll
         for (int i = 0; i < 32; ++i) { s[i] = __uint_as_float(sr[i]); s[32 + i] = __uint_as_float(sr2[i]); }
@@ -522,10 +528,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         // sub-tiles with masked columns (p must be exactly 0 there) use the
         // special-function unit only
         lsum += fast_tile ? sub_probs<kPolyPairs>(s, sc, cb, mu, pk) : sub_probs<0>(s, sc, cb, mu, pk);
-        tmem_st32(tmem + st * kSub + lane_off, pk);
+        tmem_st32(tmem + sb2 * kSub + lane_off, pk);
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(smem_u32(&sh->p_full[st]));
+        mbar_arrive(smem_u32(&sh->p_full[sb2]));
       }
       if (!ok) break;
       // epilogue: O / l once the item's last PV is done (o_final completes
@@ -576,14 +582,25 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 }
 
+// Resident CTAs per SM and ring depth.  Measured on B200 (Wan2.1-14B-shaped
+// problem): two CTAs per SM with two-stage rings run 1.75x faster than one
+// CTA per SM with five-stage rings; each CTA's S -> softmax -> PV chain has a
+// fixed latency per sub-tile that only a second CTA hides.
+#ifndef PSA_ATTN_CTAS
+#define PSA_ATTN_CTAS 2
+#endif
+
 template <int D, bool F32>
 cudaError_t launch_one(const AttnMaps& maps, const AttnArgs& a, int num_sms, cudaStream_t s) {
-  const size_t smem = 1024 + static_cast<size_t>(D) * 256 + 4 * static_cast<size_t>(D) * 128 + sizeof(AttnShared);
-  cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, F32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  constexpr int CTAS = PSA_ATTN_CTAS;
+  constexpr int NST = CTAS == 1 ? (D == 128 ? 5 : 8) : 2;
+  const size_t smem = 1024 + static_cast<size_t>(D) * 256 + 2 * NST * static_cast<size_t>(D) * 128 +
+                      sizeof(AttnShared<NST>);
+  cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, F32, NST, CTAS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const int grid = a.n_items < 2 * num_sms ? a.n_items : 2 * num_sms;
-  attn_kernel<D, F32><<<grid, kThreads, smem, s>>>(maps, a);
+  const int grid = a.n_items < CTAS * num_sms ? a.n_items : CTAS * num_sms;
+  attn_kernel<D, F32, NST, CTAS><<<grid, kThreads, smem, s>>>(maps, a);
   return cudaGetLastError();
 }
 
