@@ -164,7 +164,7 @@ MaskLayout mask_layout(const psa_shape_t* s, const psa_mask_params_t* p) {
   size_t off = 256;
   L.status = 0;
   L.blocklse = off; off = align_up(off + BHq * nkb * L.rows * 4, 256);
-  L.rowlse = off;   off = align_up(off + BHq * L.rows * 4, 256);
+  L.rowlse = off;   off = align_up(off + 2 * BHq * L.rows * 4, 256);   // one partial per epilogue warpgroup
   if (s->dtype == PSA_DT_FP32) {
     L.q16 = off; off = align_up(off + BHq * s->N * s->d * 2, 256);
     L.k16 = off; off = align_up(off + static_cast<size_t>(s->B) * s->Hkv * s->N * s->d * 2, 256);

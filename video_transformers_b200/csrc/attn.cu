@@ -51,14 +51,17 @@ struct AttnMaps {
   CUtensorMap m[9];
 };
 
-// Record of one KV sub-tile, written by the producer for the softmax.
+// Record of one KV sub-tile, written by the producer for the softmax.  The
+// bias is kept per query half: with 64-token blocks a 128-row query tile
+// holds two query blocks, and a segment may serve only one of them (its
+// other half sees -inf).
 struct alignas(16) SubInfo {
-  float cb[4];          // level of each 16-column chunk (fast sub-tiles)
-  int fast;             // every column valid, no per-row check needed
-  int rowcheck;         // slow sub-tiles: some column needs the causal / half test
-  int pad[2];
-  float bias[kSub];     // slow sub-tiles: level, or -inf for padding / past-the-end rows
-  int info[kSub];       // slow sub-tiles: (last covered token << 2) | query-half mask
+  float cb[2][4];       // level (or -inf) of each 16-column chunk, per query half (fast sub-tiles)
+  int fast;             // every chunk uniform per half, no padding, no ragged block, no causal edge
+  int causal_check;     // slow sub-tiles: some column needs the causal test
+  int pad[6];
+  float bias[2][kSub];  // slow sub-tiles: level, or -inf, per query half
+  int info[kSub];       // slow sub-tiles: last token each column covers (causal test)
 };
 
 // NST: depth of the K, V and sub-tile-record rings
@@ -259,21 +262,29 @@ __global__ void __launch_bounds__(kThreads, CTAS)
         const int last_tok = (p_last << l) - 1;                // last token covered
         const bool seg_pad = mine && half == 0;
         const bool seg_ragged = mine && half != 0 && p_last > nl;
-        const bool seg_check = mine && half != 0 && (half != 3 || (a.causal && last_tok > q0));
-        const bool fast = !__any_sync(0xffffffffu, seg_pad || seg_ragged || seg_check);
-        const bool rowcheck = __any_sync(0xffffffffu, seg_check);
+        const bool seg_causal = mine && half != 0 && a.causal && last_tok > q0;
+        // an 8-row segment shares its 16-column chunk with the next one: the
+        // chunk is uniform only if both serve the same query halves
+        const int nxt_half = __shfl_down_sync(0xffffffffu, half, 1);
+        const bool nxt_mine = __shfl_down_sync(0xffffffffu, mine ? 1 : 0, 1) != 0;
+        const bool seg_split = mine && cnt < 16 && (dst & 15) == 0 && (!nxt_mine || lane + 1 >= nseg || nxt_half != half);
+        const bool fast = !__any_sync(0xffffffffu, seg_pad || seg_ragged || seg_causal || seg_split);
+        const bool causal_check = __any_sync(0xffffffffu, seg_causal);
         if (fast) {
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const unsigned bal = __ballot_sync(0xffffffffu, mine && dst <= 16 * k);
-            const int lev = __shfl_sync(0xffffffffu, l, bal ? 31 - __clz(bal) : 0);
-            if (lane == k) ti.cb[k] = static_cast<float>(lev);
+            const int src = bal ? 31 - __clz(bal) : 0;
+            const int lev = __shfl_sync(0xffffffffu, l, src);
+            const int hm = __shfl_sync(0xffffffffu, half, src);
+            if (lane == k) ti.cb[0][k] = (hm & 1) ? static_cast<float>(lev) : -CUDART_INF_F;
+            if (lane == 4 + k) ti.cb[1][k] = (hm & 2) ? static_cast<float>(lev) : -CUDART_INF_F;
           }
         } else {
 #pragma unroll
           for (int m = 0; m < 2; ++m) {
             const int c = lane + 32 * m;
-            float bias = -CUDART_INF_F;
+            float bias0 = -CUDART_INF_F, bias1 = -CUDART_INF_F;
             int inf = 0;
             for (int s = 0; s < nseg; ++s) {
               const int ms = __shfl_sync(0xffffffffu, mine ? 1 : 0, s);
@@ -285,15 +296,17 @@ __global__ void __launch_bounds__(kThreads, CTAS)
                 const int ls = seg_level(ws), hf = seg_half(ws), Js = seg_block(ws);
                 const int p = Js * (a.block >> ls) + los + (c - ds);
                 const bool valid = hf != 0 && p < (a.N >> ls);
-                bias = valid ? static_cast<float>(ls) : -CUDART_INF_F;
-                inf = ((((p + 1) << ls) - 1) << 2) | hf;
+                bias0 = valid && (hf & 1) ? static_cast<float>(ls) : -CUDART_INF_F;
+                bias1 = valid && (hf & 2) ? static_cast<float>(ls) : -CUDART_INF_F;
+                inf = ((p + 1) << ls) - 1;
               }
             }
-            ti.bias[c] = bias;
+            ti.bias[0][c] = bias0;
+            ti.bias[1][c] = bias1;
             ti.info[c] = inf;
           }
         }
-        if (lane == 0) { ti.fast = fast ? 1 : 0; ti.rowcheck = rowcheck ? 1 : 0; }
+        if (lane == 0) { ti.fast = fast ? 1 : 0; ti.causal_check = causal_check ? 1 : 0; }
         mbar_arrive(smem_u32(&sh->i_full[st]));
 
         // V of the previous sub-tile
@@ -405,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, CTAS)
     const int q = warp & 3;
     const int row = q * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-    const int my_half_bit = 1 << (row >> 6);
+    const int my_half = row >> 6;         // which query block of a 64-token-block tile
     uint32_t it = 0, icnt = 0;
     bool ok = true;
     for (int idx = blockIdx.x; idx < a.n_items && ok; idx += gridDim.x) {
@@ -447,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, CTAS)
         float mt;
         const bool fast_tile = ti.fast != 0;
         if (fast_tile) {
-          const float4 c4 = *reinterpret_cast<const float4*>(ti.cb);
+          const float4 c4 = *reinterpret_cast<const float4*>(ti.cb[my_half]);
           cb[0] = c4.x; cb[1] = c4.y; cb[2] = c4.z; cb[3] = c4.w;
           float cmax[4];
 #pragma unroll
@@ -463,22 +476,20 @@ __global__ void __launch_bounds__(kThreads, CTAS)
           // causal / query-half test; afterwards s holds the full argument
 #pragma unroll
           for (int c4 = 0; c4 < kSub / 4; ++c4) {
-            const float4 bv = *reinterpret_cast<const float4*>(&ti.bias[4 * c4]);
+            const float4 bv = *reinterpret_cast<const float4*>(&ti.bias[my_half][4 * c4]);
             s[4 * c4 + 0] = fmaf(s[4 * c4 + 0], sc, bv.x);
             s[4 * c4 + 1] = fmaf(s[4 * c4 + 1], sc, bv.y);
             s[4 * c4 + 2] = fmaf(s[4 * c4 + 2], sc, bv.z);
             s[4 * c4 + 3] = fmaf(s[4 * c4 + 3], sc, bv.w);
           }
-          if (ti.rowcheck) {
+          if (ti.causal_check) {
 #pragma unroll
             for (int c4 = 0; c4 < kSub / 4; ++c4) {
               const int4 iv = *reinterpret_cast<const int4*>(&ti.info[4 * c4]);
-              const int iw[4] = {iv.x, iv.y, iv.z, iv.w};
-#pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                const bool vis = (iw[u] & my_half_bit) && (!a.causal || (iw[u] >> 2) <= tok);
-                s[4 * c4 + u] = vis ? s[4 * c4 + u] : -CUDART_INF_F;
-              }
+              s[4 * c4 + 0] = iv.x <= tok ? s[4 * c4 + 0] : -CUDART_INF_F;
+              s[4 * c4 + 1] = iv.y <= tok ? s[4 * c4 + 1] : -CUDART_INF_F;
+              s[4 * c4 + 2] = iv.z <= tok ? s[4 * c4 + 2] : -CUDART_INF_F;
+              s[4 * c4 + 3] = iv.w <= tok ? s[4 * c4 + 3] : -CUDART_INF_F;
             }
           }
           sc = 1.0f;

@@ -34,7 +34,7 @@ struct ScoreArgs {
   int causal;
   float scale_log2;    // softmax scale * log2(e)
   float* blocklse;     // [BHq][nkb][rows]  log2-domain logsumexp of each block
-  float* rowlse;       // [BHq][rows]
+  float* rowlse;       // [2][BHq][rows]  partial row LSEs of the two epilogue warpgroups
   int* status;
 };
 cudaError_t launch_score(const CUtensorMap* mapA, const CUtensorMap* mapB, const ScoreArgs& a,
@@ -47,7 +47,7 @@ struct SelectArgs {
   float cos_min;
   int n_dense_prefix;
   const float* blocklse;
-  const float* rowlse;
+  const float* rowlse;      // [2][B*Hq][rows]
   const float* blockcos;
   uint8_t* mask;
   float* mass_out;

@@ -7,8 +7,10 @@
 // score_kernel   a tcgen05 GEMM of 128 score rows x 128 score columns per
 //                tile (rows: sampled queries, or antidiagonal query groups;
 //                columns: keys, or key groups), accumulated in TMEM, followed
-//                by a per-(row, KV block) log-sum-exp in the epilogue warps.
-//                Only the block LSEs and each row's total LSE leave the SM.
+//                by a per-(row, KV block) log-sum-exp in two epilogue
+//                warpgroups that take alternate column tiles.  Only the block
+//                LSEs and each row's LSE (one partial per warpgroup) leave
+//                the SM.
 // select_kernel  one CTA per (b, h, query block): block masses from the
 //                LSEs, a bitonic sort (mass descending, index ascending), an
 //                fp64 exclusive scan, thresholds, forced rules.
@@ -21,16 +23,20 @@
 namespace psa {
 namespace {
 
-constexpr int kStages = 4;
-constexpr int kChunkBytes = 128 * 128;        // 128 rows x 64 bf16
-constexpr int kStageBytes = 2 * kChunkBytes;  // A chunk + B chunk
-constexpr int kThreads = 192;                 // producer, MMA, 4 epilogue warps
+constexpr int kThreads = 320;                 // producer, MMA, two epilogue warpgroups
+constexpr int kChunk = 128 * 128;             // 128 rows x 64 bf16: one 128-byte-swizzled chunk
+constexpr int kRegionChunks = 8;              // 128 KB of staging
+// Sampling: A (the sampled query rows, <= 2 chunks) stays resident in chunks
+// [0, 2) for all column tiles of a row tile; K chunks stream through a ring
+// in chunks [2, 8).  Antidiagonal: A and B both stream, one (A, B) chunk
+// pair per stage, four stages.
+constexpr int kSampleStages = 6;
+constexpr int kAntiStages = 4;
 
 struct ScoreShared {
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
-  uint64_t s_full[2];
-  uint64_t s_empty[2];
+  uint64_t a_full, a_empty;
+  uint64_t full[kSampleStages], empty[kSampleStages];
+  uint64_t s_full[2], s_empty[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -41,23 +47,63 @@ __device__ __forceinline__ int kv_head_of(int bh, int Hq, int Hkv) {
   return b * Hkv + h / (Hq / Hkv);
 }
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// log2-domain log-sum-exp of CPB consecutive scores s[0..CPB) (already
+// masked to -inf where invalid when MASKED), scaled by sc.
+template <int CPB, bool MASKED>
+__device__ __forceinline__ float block_lse(const float* s, float sc) {
+  static_assert(CPB % 4 == 0 && CPB >= 8, "block width");
+  float x[4] = {s[0], s[1], s[2], s[3]};
+  constexpr int J8 = 4 + (CPB - 4) / 8 * 8;     // end of the 8-wide steps
+#pragma unroll
+  for (int j = 4; j < J8; j += 8) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) x[u] = fmax3(x[u], s[j + u], s[j + 4 + u]);
+  }
+#pragma unroll
+  for (int j = J8; j < CPB; j += 4) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) x[u] = fmaxf(x[u], s[j + u]);
+  }
+  const float mraw = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+  if (MASKED && mraw == -CUDART_INF_F) return -CUDART_INF_F;
+  const float mb = mraw * sc;
+  const float2 sc2 = make_float2(sc, sc), off = make_float2(-mb, -mb);
+  float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int j = 0; j < CPB; j += 2) {
+    const float2 z = __ffma2_rn(make_float2(s[j], s[j + 1]), sc2, off);
+    acc[(j >> 1) & 1] = __fadd2_rn(acc[(j >> 1) & 1], make_float2(fast_exp2(z.x), fast_exp2(z.y)));
+  }
+  const float2 t = __fadd2_rn(acc[0], acc[1]);
+  return mb + __log2f(t.x + t.y);
+}
+
 template <int CPB>
 __global__ void __launch_bounds__(kThreads, 1)
     score_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                  const ScoreArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  ScoreShared* sh = reinterpret_cast<ScoreShared*>(tiles + kStages * kStageBytes);
+  ScoreShared* sh = reinterpret_cast<ScoreShared*>(tiles + kRegionChunks * kChunk);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row_tiles = (a.rows + 127) / 128;
   const int col_tiles = (a.cols + 127) / 128;
   const int n_items = a.BHq * row_tiles;
-  const int nk = (a.mode == 0 ? a.d / 64 : a.S * a.d / 64);
+  const bool sampling = a.mode == 0;
+  const int nk = sampling ? a.d / 64 : a.S * a.d / 64;   // 64-channel chunks per column tile
   const int kc_per_s = a.d / 64;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) { mbar_init(smem_u32(&sh->full[i]), 1); mbar_init(smem_u32(&sh->empty[i]), 1); }
+    mbar_init(smem_u32(&sh->a_full), 1);
+    mbar_init(smem_u32(&sh->a_empty), 1);
+    for (int i = 0; i < kSampleStages; ++i) { mbar_init(smem_u32(&sh->full[i]), 1); mbar_init(smem_u32(&sh->empty[i]), 1); }
     for (int i = 0; i < 2; ++i) { mbar_init(smem_u32(&sh->s_full[i]), 1); mbar_init(smem_u32(&sh->s_empty[i]), 128); }
     mbar_init(smem_u32(&sh->drain), 1);
     sh->abort = 0;
@@ -74,141 +120,154 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto tiles_for = [&](int r0) {
     if (!a.causal) return col_tiles;
     const int rlast = min(r0 + 127, a.rows - 1);
-    const int pos = a.mode == 0 ? rlast * a.step : rlast;
+    const int pos = sampling ? rlast * a.step : rlast;
     return min(col_tiles, pos / 128 + 1);
   };
+  const int nst = sampling ? kSampleStages : kAntiStages;
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       tma_prefetch_desc(&mapA);
       tma_prefetch_desc(&mapB);
-      uint32_t it = 0;
+      uint32_t it = 0, icnt = 0;
       bool ok = true;
-      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++icnt) {
         const int bh = item / row_tiles, r0 = (item - bh * row_tiles) * 128;
         const int hkv = kv_head_of(bh, a.Hq, a.Hkv);
         const int nct = tiles_for(r0);
+        if (sampling) {
+          if (!bounded_wait(smem_u32(&sh->a_empty), (icnt & 1) ^ 1, abort, a.status, 45, item, 0, 0, icnt)) { ok = false; break; }
+          mbar_arrive_expect_tx(smem_u32(&sh->a_full), nk * kChunk);
+          for (int kc = 0; kc < nk; ++kc)
+            tma_load_4d(smem_u32(tiles + kc * kChunk), &mapA, smem_u32(&sh->a_full), kc * 64, 0, r0, bh);
+        }
         for (int ct = 0; ct < nct && ok; ++ct) {
           for (int kc = 0; kc < nk; ++kc, ++it) {
-            const int st = it % kStages;
-            if (!bounded_wait(smem_u32(&sh->empty[st]), ((it / kStages) & 1) ^ 1, abort, a.status, 41, item, ct, kc, it)) { ok = false; break; }
+            const int st = it % nst;
+            if (!bounded_wait(smem_u32(&sh->empty[st]), ((it / nst) & 1) ^ 1, abort, a.status, 41, item, ct, kc, it)) { ok = false; break; }
             const uint32_t bar = smem_u32(&sh->full[st]);
-            mbar_arrive_expect_tx(bar, kStageBytes);
-            const uint32_t dA = smem_u32(tiles + st * kStageBytes);
-            const uint32_t dB = dA + kChunkBytes;
-            const int s = kc / kc_per_s, half = kc - s * kc_per_s;
-            if (a.mode == 0) {
-              tma_load_4d(dA, &mapA, bar, kc * 64, 0, r0, bh);
-              tma_load_4d(dB, &mapB, bar, kc * 64, 0, ct * 128, hkv);
+            if (sampling) {
+              mbar_arrive_expect_tx(bar, kChunk);
+              tma_load_4d(smem_u32(tiles + (2 + st) * kChunk), &mapB, bar, kc * 64, 0, ct * 128, hkv);
             } else {
-              tma_load_4d(dA, &mapA, bar, half * 64, a.S - 1 - s, r0, bh);
-              tma_load_4d(dB, &mapB, bar, half * 64, s, ct * 128, hkv);
+              const int s = kc / kc_per_s, half = kc - s * kc_per_s;
+              mbar_arrive_expect_tx(bar, 2 * kChunk);
+              tma_load_4d(smem_u32(tiles + (2 * st) * kChunk), &mapA, bar, half * 64, a.S - 1 - s, r0, bh);
+              tma_load_4d(smem_u32(tiles + (2 * st + 1) * kChunk), &mapB, bar, half * 64, s, ct * 128, hkv);
             }
           }
         }
       }
       // drain: every armed stage must have landed before the CTA exits
-      for (uint32_t st = 0; st < static_cast<uint32_t>(kStages); ++st) {
-        if (it > st) drain_wait(smem_u32(&sh->full[st]), ((it - 1 - st) / kStages) & 1, a.status);
-      }
+      for (uint32_t st = 0; st < static_cast<uint32_t>(nst); ++st)
+        if (it > st) drain_wait(smem_u32(&sh->full[st]), ((it - 1 - st) / nst) & 1, a.status);
+      if (sampling && icnt > 0) drain_wait(smem_u32(&sh->a_full), (icnt - 1) & 1, a.status);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false);
-      uint32_t it = 0, t = 0;
+      const uint64_t d0 = sdesc_sw128(smem_u32(tiles), 16, 1024);
+      uint32_t it = 0, t = 0, icnt = 0;
       bool ok = true;
-      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++icnt) {
         const int bh = item / row_tiles, r0 = (item - bh * row_tiles) * 128;
         (void)bh;
         const int nct = tiles_for(r0);
+        if (sampling) {
+          if (!bounded_wait(smem_u32(&sh->a_full), icnt & 1, abort, a.status, 46, item, 0, 0, icnt)) { ok = false; break; }
+          tc_fence_after();
+        }
         for (int ct = 0; ct < nct && ok; ++ct, ++t) {
           const int buf = t & 1;
           if (!bounded_wait(smem_u32(&sh->s_empty[buf]), ((t >> 1) & 1) ^ 1, abort, a.status, 42, item, ct, t, it)) { ok = false; break; }
           tc_fence_after();
           const uint32_t dS = tmem + buf * 128;
           for (int kc = 0; kc < nk; ++kc, ++it) {
-            const int st = it % kStages;
-            if (!bounded_wait(smem_u32(&sh->full[st]), (it / kStages) & 1, abort, a.status, 43, item, ct, kc, it)) { ok = false; break; }
+            const int st = it % nst;
+            if (!bounded_wait(smem_u32(&sh->full[st]), (it / nst) & 1, abort, a.status, 43, item, ct, kc, it)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t sA = smem_u32(tiles + st * kStageBytes);
-            const uint32_t sB = sA + kChunkBytes;
+            const int ca = sampling ? kc : 2 * st;
+            const int cb = sampling ? 2 + st : 2 * st + 1;
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              umma_ss(dS, sdesc_sw128(sA + 32 * k, 16, 1024), sdesc_sw128(sB + 32 * k, 16, 1024), idesc,
-                      (kc | k) != 0);
-            }
+            for (int k = 0; k < 4; ++k)
+              umma_ss(dS, d0 + ((ca * kChunk + 32 * k) >> 4), d0 + ((cb * kChunk + 32 * k) >> 4), idesc, (kc | k) != 0);
             umma_commit(smem_u32(&sh->empty[st]));
           }
-          if (ok) umma_commit(smem_u32(&sh->s_full[buf]));
+          if (!ok) break;
+          umma_commit(smem_u32(&sh->s_full[buf]));
+          if (sampling && ct + 1 == nct) umma_commit(smem_u32(&sh->a_empty));
         }
       }
       umma_commit(smem_u32(&sh->drain));
       drain_wait(smem_u32(&sh->drain), 0, a.status);
     }
   } else {
-    // ---------------- epilogue: per (row, block) log-sum-exp ----------------
+    // ---------- epilogue: two warpgroups take alternate column tiles ----------
+    const int wg = (warp - 2) >> 2;         // 0 or 1: the S buffer this group reads
     const int q = warp & 3;                 // TMEM lane quarter of this warp
     const int lrow = q * 32 + lane;         // tile row owned by this thread
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     constexpr int BPT = 128 / CPB;          // KV blocks per column tile
     uint32_t t = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
       const int bh = item / row_tiles, r0 = (item - bh * row_tiles) * 128;
       const int r = r0 + lrow;
-      const int pos = a.mode == 0 ? r * a.step : r;     // token (sampling) or group index
+      const int pos = sampling ? r * a.step : r;     // token (sampling) or group index
       const int nct = tiles_for(r0);
+      const int climit = a.causal ? min(a.cols, pos + 1) : a.cols;   // valid columns: c < climit
       float M = -CUDART_INF_F, Ssum = 0.f;
+      float* bl = a.blocklse + static_cast<int64_t>(bh) * a.nkb * a.rows + r;
       for (int ct = 0; ct < nct; ++ct, ++t) {
-        const int buf = t & 1;
-        if (!warp_wait(smem_u32(&sh->s_full[buf]), (t >> 1) & 1, abort, a.status, 44, item, ct, t, 0)) { ok = false; break; }
+        if ((t & 1) != static_cast<uint32_t>(wg)) continue;
+        if (!warp_wait(smem_u32(&sh->s_full[wg]), (t >> 1) & 1, abort, a.status, 44, item, ct, t, wg)) { ok = false; break; }
         tc_fence_after();
-        float z[128];
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          uint32_t raw[32];
-          tmem_ld32(tmem + buf * 128 + c4 * 32 + (static_cast<uint32_t>(q * 32) << 16), raw);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) z[c4 * 32 + j] = __uint_as_float(raw[j]) * a.scale_log2;
-        }
+        uint32_t raw[128];
+        tmem_ld128(tmem + wg * 128 + lane_off, raw);
         tc_fence_before();
-        mbar_arrive(smem_u32(&sh->s_empty[buf]));
+        mbar_arrive(smem_u32(&sh->s_empty[wg]));
+        float* z = reinterpret_cast<float*>(raw);
         const int c0 = ct * 128;
-        const int climit = a.causal ? min(a.cols, pos + 1) : a.cols;   // valid columns: c < climit
+        float blse[BPT];
+        if (c0 + 128 <= climit) {
 #pragma unroll
-        for (int bb = 0; bb < BPT; ++bb) {
-          float m = -CUDART_INF_F;
+          for (int bb = 0; bb < BPT; ++bb) blse[bb] = block_lse<CPB, false>(z + bb * CPB, a.scale_log2);
+        } else {
 #pragma unroll
-          for (int j = 0; j < CPB; ++j) {
-            const int c = c0 + bb * CPB + j;
-            if (c < climit) m = fmaxf(m, z[bb * CPB + j]);
-          }
-          float s = 0.f;
-          if (m != -CUDART_INF_F) {
+          for (int c = 0; c < 128; ++c) z[c] = c0 + c < climit ? z[c] : -CUDART_INF_F;
 #pragma unroll
-            for (int j = 0; j < CPB; ++j) {
-              const int c = c0 + bb * CPB + j;
-              if (c < climit) s += fast_exp2(z[bb * CPB + j] - m);
-            }
-          }
-          const float blse = m == -CUDART_INF_F ? -CUDART_INF_F : m + __log2f(s);
-          const int J = (c0 / CPB) + bb;
-          if (r < a.rows && J < a.nkb) a.blocklse[(static_cast<int64_t>(bh) * a.nkb + J) * a.rows + r] = blse;
-          if (blse != -CUDART_INF_F) {
-            const float Mn = fmaxf(M, blse);
-            Ssum = Ssum * fast_exp2(M - Mn) + fast_exp2(blse - Mn);
-            M = Mn;
+          for (int bb = 0; bb < BPT; ++bb) blse[bb] = block_lse<CPB, true>(z + bb * CPB, a.scale_log2);
+        }
+        float mt = blse[0];
+#pragma unroll
+        for (int bb = 1; bb < BPT; ++bb) mt = fmaxf(mt, blse[bb]);
+        if (mt != -CUDART_INF_F) {
+          const float Mn = fmaxf(M, mt);
+          float add = 0.f;
+#pragma unroll
+          for (int bb = 0; bb < BPT; ++bb) add += fast_exp2(blse[bb] - Mn);
+          Ssum = Ssum * fast_exp2(M - Mn) + add;
+          M = Mn;
+        }
+        if (r < a.rows) {
+#pragma unroll
+          for (int bb = 0; bb < BPT; ++bb) {
+            const int J = ct * BPT + bb;
+            if (J < a.nkb) bl[static_cast<int64_t>(J) * a.rows] = blse[bb];
           }
         }
       }
       if (!ok) break;
-      // column tiles never visited (causal) hold no probability
-      if (a.causal) {
-        for (int J = nct * BPT; J < a.nkb; ++J)
-          if (r < a.rows) a.blocklse[(static_cast<int64_t>(bh) * a.nkb + J) * a.rows + r] = -CUDART_INF_F;
+      if (r < a.rows) {
+        // column tiles never visited (causal) hold no probability
+        if (wg == 0) {
+          for (int J = nct * BPT; J < a.nkb; ++J) bl[static_cast<int64_t>(J) * a.rows] = -CUDART_INF_F;
+        }
+        a.rowlse[(static_cast<int64_t>(wg) * a.BHq + bh) * a.rows + r] =
+            M == -CUDART_INF_F ? -CUDART_INF_F : M + __log2f(Ssum);
       }
-      if (r < a.rows) a.rowlse[static_cast<int64_t>(bh) * a.rows + r] = M == -CUDART_INF_F ? -CUDART_INF_F : M + __log2f(Ssum);
     }
   }
 
@@ -246,7 +305,16 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectArgs a)
   } else {
     nvalid = min(a.rows_per_block, a.rows - rbeg);
   }
-  const float* rl = a.rowlse + static_cast<int64_t>(bh) * a.rows + rbeg;
+  // row LSE: the two epilogue warpgroups of the score kernel each wrote the
+  // LSE of the column tiles they handled; combine them (log2 domain)
+  __shared__ double rlse[128];
+  for (int s = threadIdx.x; s < nvalid; s += blockDim.x) {
+    const double x = a.rowlse[static_cast<int64_t>(bh) * a.rows + rbeg + s];
+    const double y = a.rowlse[(static_cast<int64_t>(a.B) * a.Hq + bh) * a.rows + rbeg + s];
+    const double mx = fmax(x, y);
+    rlse[s] = mx == -CUDART_INF ? mx : mx + log2(exp2(x - mx) + exp2(y - mx));
+  }
+  __syncthreads();
 
   for (int J = threadIdx.x; J < P2; J += blockDim.x) {
     if (J < a.nkb) {
@@ -254,7 +322,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectArgs a)
       double m = 0.0;
       for (int s = 0; s < nvalid; ++s) {
         const float x = bl[s];
-        if (x != -CUDART_INF_F) m += exp2(static_cast<double>(x) - static_cast<double>(rl[s]));
+        if (x != -CUDART_INF_F) m += exp2(static_cast<double>(x) - rlse[s]);
       }
       const float mass = static_cast<float>(m / nvalid);
       if (a.mass_out) a.mass_out[static_cast<int64_t>(row) * a.nkb + J] = mass;
@@ -328,7 +396,7 @@ cudaError_t launch_score(const CUtensorMap* mapA, const CUtensorMap* mapB, const
   const int row_tiles = (a.rows + 127) / 128;
   const int n_items = a.BHq * row_tiles;
   const int grid = n_items < num_sms ? n_items : num_sms;
-  const size_t smem = 1024 + kStages * kStageBytes + sizeof(ScoreShared);
+  const size_t smem = 1024 + kRegionChunks * kChunk + sizeof(ScoreShared);
   switch (a.cols_per_block) {
 #define PSA_SCORE_CASE(CPB)                                                                       \
   case CPB: {                                                                                     \
