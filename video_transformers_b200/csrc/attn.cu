@@ -133,7 +133,10 @@ __device__ __forceinline__ float sub_probs(const float* s, float sc, const float
 // number of 64-row sub-tiles of an item with `rows` real KV rows
 __device__ __forceinline__ uint32_t sub_count(int rows) { return static_cast<uint32_t>((rows + kSub - 1) / kSub); }
 
-template <int D, bool OUT_F32, int NST, int CTAS>
+// H2: the query tile holds two 64-token query blocks whose segment lists
+// differ, so records are kept per query half (block 64); with 128-token
+// blocks both halves always agree and the per-half work is compiled out.
+template <int D, bool OUT_F32, int NST, int CTAS, bool H2>
 __global__ void __launch_bounds__(kThreads, CTAS)
     attn_kernel(const __grid_constant__ AttnMaps maps, const AttnArgs a) {
   constexpr int QB = D * 256;          // bytes of the 128-row Q tile
@@ -267,7 +270,8 @@ __global__ void __launch_bounds__(kThreads, CTAS)
         // chunk is uniform only if both serve the same query halves
         const int nxt_half = __shfl_down_sync(0xffffffffu, half, 1);
         const bool nxt_mine = __shfl_down_sync(0xffffffffu, mine ? 1 : 0, 1) != 0;
-        const bool seg_split = mine && cnt < 16 && (dst & 15) == 0 && (!nxt_mine || lane + 1 >= nseg || nxt_half != half);
+        const bool seg_split = H2 && mine && cnt < 16 && (dst & 15) == 0 &&
+                               (!nxt_mine || lane + 1 >= nseg || nxt_half != half);
         const bool fast = !__any_sync(0xffffffffu, seg_pad || seg_ragged || seg_causal || seg_split);
         const bool causal_check = __any_sync(0xffffffffu, seg_causal);
         if (fast) {
@@ -278,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, CTAS)
             const int lev = __shfl_sync(0xffffffffu, l, src);
             const int hm = __shfl_sync(0xffffffffu, half, src);
             if (lane == k) ti.cb[0][k] = (hm & 1) ? static_cast<float>(lev) : -CUDART_INF_F;
-            if (lane == 4 + k) ti.cb[1][k] = (hm & 2) ? static_cast<float>(lev) : -CUDART_INF_F;
+            if (H2 && lane == 4 + k) ti.cb[1][k] = (hm & 2) ? static_cast<float>(lev) : -CUDART_INF_F;
           }
         } else {
 #pragma unroll
@@ -302,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, CTAS)
               }
             }
             ti.bias[0][c] = bias0;
-            ti.bias[1][c] = bias1;
+            if (H2) ti.bias[1][c] = bias1;
             ti.info[c] = inf;
           }
         }
@@ -418,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, CTAS)
     const int q = warp & 3;
     const int row = q * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-    const int my_half = row >> 6;         // which query block of a 64-token-block tile
+    const int my_half = H2 ? (row >> 6) : 0;   // which query block of a 64-token-block tile
     uint32_t it = 0, icnt = 0;
     bool ok = true;
     for (int idx = blockIdx.x; idx < a.n_items && ok; idx += gridDim.x) {
@@ -607,11 +611,18 @@ cudaError_t launch_one(const AttnMaps& maps, const AttnArgs& a, int num_sms, cud
   constexpr int NST = CTAS == 1 ? (D == 128 ? 5 : 8) : 2;
   const size_t smem = 1024 + static_cast<size_t>(D) * 256 + 2 * NST * static_cast<size_t>(D) * 128 +
                       sizeof(AttnShared<NST>);
-  cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, F32, NST, CTAS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
   const int grid = a.n_items < CTAS * num_sms ? a.n_items : CTAS * num_sms;
-  attn_kernel<D, F32, NST, CTAS><<<grid, kThreads, smem, s>>>(maps, a);
+  if (a.block == 64) {
+    cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, F32, NST, CTAS, true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    attn_kernel<D, F32, NST, CTAS, true><<<grid, kThreads, smem, s>>>(maps, a);
+  } else {
+    cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, F32, NST, CTAS, false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    attn_kernel<D, F32, NST, CTAS, false><<<grid, kThreads, smem, s>>>(maps, a);
+  }
   return cudaGetLastError();
 }
 
