@@ -41,6 +41,12 @@ sys.path.insert(0, ROOT)
 import workloads as W  # noqa: E402
 
 METRIC = "PSA attn fwd ms/call & achieved TFLOP/s (executed FLOPs) vs B200 BF16 peak"
+# DRAM traffic of one attention launch (dram__bytes_read.sum + dram__bytes_write.sum), from an
+# ncu capture of the same workload at 4 heads scaled to the full head count (traffic grows with
+# the heads: the head-major queue keeps one head's KV in L2 at a time); valid only for the
+# attention source it was measured on (summary in profiles/attn_kernel_wan14b.md).
+ATTN_TRAFFIC = {"wan14b": {"bytes_per_launch": 10 * (743.809280e6 + 71.797504e6),
+                           "attn_cu_sha256": "b99157c006021851afeb671c24c57be7ee988983e6b850d20d79d5b3f8cc9f72"}}
 UNIT = "TFLOP/s"
 KERNELS_PER_STEP = {"pyramid": 1, "blockcos": 0, "score": 1, "select": 1, "plan": 3, "attention": 1}
 
@@ -109,6 +115,19 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- helpers
+
+def attn_traffic(w):
+    """Measured DRAM bytes per attention launch for this workload, or None when
+    there is no capture of it or the attention source changed since."""
+    import hashlib
+    rec = ATTN_TRAFFIC.get(w.name)
+    if rec is None:
+        return None
+    with open(os.path.join(ROOT, "video_transformers_b200", "csrc", "attn.cu"), "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest() != rec["attn_cu_sha256"]:
+            return None
+    return rec["bytes_per_launch"]
+
 
 def max_over_ranks(ms: float, world: int, device) -> float:
     """Device time of the timed region, max over ranks (every rank takes
@@ -301,7 +320,7 @@ def run_psa(args, rank, world, local_rank):
         "roofline": {"bound": "tensor", "kernel": "attn_kernel (psa_attention_fwd incl. its 3 planner kernels)",
                      "achieved": attn_tflops, "peak": bf16_sus, "unit": "TFLOP/s", "frac": attn_tflops / bf16_sus,
                      "peak_kind": "sustained bf16 (%s)" % src, "frac_of_burst": attn_tflops / bf16_burst,
-                     "traffic": None},
+                     "traffic": attn_traffic(w)},
         "pyramid_roofline": {"bound": "hbm", "achieved": pyr_bytes / (pyr_ms * 1e-3) / 1e9, "peak": hbm,
                              "unit": "GB/s", "frac": pyr_bytes / (pyr_ms * 1e-3) / 1e9 / hbm},
         "e2e": e2e,
