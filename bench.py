@@ -412,6 +412,9 @@ def cpu_threads():
         return os.cpu_count()
 
 
+REF_BLOCKS_TOTAL = 640
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return None
@@ -420,9 +423,12 @@ def run_reference(args, rank, world):
     mask = W.make_given_mask(w, gen, device=q.device) if w.mask_mode == "given" else None
     for _ in range(args.warmup):
         oracle_sample(w, q, k, v, 1, seed=99, mask_dev=mask)
+    # the whole timed run samples about REF_BLOCKS_TOTAL query blocks (about a
+    # minute of host time at Wan2.1-14B size), spread over the steps
+    per_step = max(1, min(args.cpu_blocks, REF_BLOCKS_TOTAL // max(1, args.steps)))
     secs, fl, desc = 0.0, 0.0, None
     for i in range(args.steps):
-        dt, f, desc = oracle_sample(w, q, k, v, args.cpu_blocks, seed=i, mask_dev=mask)
+        dt, f, desc = oracle_sample(w, q, k, v, per_step, seed=i, mask_dev=mask)
         secs += dt
         fl += f
     value = fl / secs / 1e12
@@ -453,11 +459,11 @@ def workload(args) -> W.Workload:
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--config", default="wan14b", choices=W.ORDER)
     ap.add_argument("--impl", default="psa", choices=["psa", "reference"])
-    ap.add_argument("--cpu-blocks", type=int, default=40, help="query blocks in the oracle sample")
+    ap.add_argument("--cpu-blocks", type=int, default=160, help="query blocks in the oracle sample (about 15 s of host time at Wan2.1-14B size)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
