@@ -48,6 +48,16 @@ reason in the design notes):
       J == I -> level 0.
   R9  block cosine = mean pairwise cosine over i != j of the block's valid
       keys; a zero key has unit vector 0; a one-key block scores 1.
+  R10 quantile (rank) level assignment, the alternative to R7 that the
+      [article] Results ablation compares with: rank as in R7; the block at
+      rank r gets level #{t_l <= r / n_vis}, SKIP when that count reaches L,
+      where n_vis is the number of key blocks the row can see (J <= I when
+      causal, else all).  With L = 1 and t_0 = k / n_vis this keeps exactly
+      the k heaviest blocks (a top-k binary mask).
+  R11 mean-key score ([skill] Core Technique, block importance as the
+      query against the mean of the block's keys): the query side is the
+      mean of the query block's valid queries as well; mass[I, J] =
+      softmax over visible J of sm_scale * mean_q(I) . mean_k(J).
 
 Pins: every function here is checked by ``tests/test_oracle_pins.py``
 against closed forms, invariants, brute force or an independent library
@@ -275,6 +285,56 @@ def exclusive_prefix(mass_row: Sequence[float]) -> np.ndarray:
     return C
 
 
+def assign_levels_quantile_row(mass_row: Sequence[float], thresholds: Sequence[float], levels: int,
+                               n_visible: Optional[int] = None) -> np.ndarray:
+    """Rank-based (quantile / top-k) level assignment for one query block,
+    the alternative the [article] Results ablation weighs against threshold
+    levels.  Reading R10: the block at rank r (mass descending, ties to the
+    lower index) gets level #{t_l <= r / n_visible}."""
+    mass_row = np.asarray(mass_row, dtype=np.float64)
+    n = mass_row.shape[0]
+    nv = n if n_visible is None else n_visible
+    order = sorted(range(n), key=lambda J: (-mass_row[J], J))
+    out = np.empty(n, dtype=np.int64)
+    for r, J in enumerate(order):
+        frac = r / nv
+        lev = sum(1 for t in thresholds if t <= frac)
+        out[J] = SKIP if lev >= levels else lev
+    return out
+
+
+def block_means(x, block: int) -> np.ndarray:
+    """[B, H, N, d] -> [B, H, nB, d]: the mean of each block's valid tokens
+    (the last block may be ragged)."""
+    x = _f64(x)
+    B, H, N, d = x.shape
+    nb = -(-N // block)
+    out = np.empty((B, H, nb, d))
+    for J in range(nb):
+        out[:, :, J] = x[:, :, J * block:min((J + 1) * block, N)].mean(axis=2)
+    return out
+
+
+def meankey_mass(q, k, block: int, sm_scale: float, causal: bool = False,
+                 rows: Optional[Iterable[Tuple[int, int, int]]] = None) -> np.ndarray:
+    """Block importance from block means ([skill] Core Technique, a block is
+    scored by the query against the mean of its keys).  Reading R11.
+    Returns mass [B, Hq, nQB, nKB]; rows not listed in ``rows`` stay NaN."""
+    qm = block_means(q, block)
+    km = block_means(k, block)
+    B, Hq, nb, d = qm.shape
+    grp = Hq // km.shape[1]
+    mass = np.full((B, Hq, nb, nb), np.nan)
+    if rows is None:
+        rows = [(b, h, I) for b in range(B) for h in range(Hq) for I in range(nb)]
+    for b, h, I in rows:
+        z = sm_scale * (km[b, h // grp] @ qm[b, h, I])             # [nKB]
+        if causal:
+            z = np.where(np.arange(nb) <= I, z, -np.inf)
+        mass[b, h, I] = _softmax_rows(z[None, :])[0]
+    return mass
+
+
 def apply_forced_rules(levels_row: np.ndarray, I: int, block: int, levels: int, causal: bool,
                        n_dense_prefix: int = 0, cos_row: Optional[np.ndarray] = None,
                        cos_min: float = -3.0) -> np.ndarray:
@@ -297,14 +357,19 @@ def apply_forced_rules(levels_row: np.ndarray, I: int, block: int, levels: int, 
 
 def make_mask(mass: np.ndarray, thresholds, levels: int, block: int, causal: bool,
               n_dense_prefix: int = 0, blockcos: Optional[np.ndarray] = None, cos_min: float = -3.0,
-              hq_per_kv: int = 1, rows=None) -> np.ndarray:
-    """mass [B,Hq,nQB,nKB] -> mask uint8 of the same shape (SKIP = 0xFF)."""
+              hq_per_kv: int = 1, rows=None, policy: str = "mass") -> np.ndarray:
+    """mass [B,Hq,nQB,nKB] -> mask uint8 of the same shape (SKIP = 0xFF).
+    policy "mass": levels by reading R7; "quantile": by reading R10."""
     B, Hq, nqb, nkb = mass.shape
     out = np.full((B, Hq, nqb, nkb), SKIP, dtype=np.int64)
     if rows is None:
         rows = [(b, h, I) for b in range(B) for h in range(Hq) for I in range(nqb)]
     for b, h, I in rows:
-        lev = assign_levels_row(mass[b, h, I], thresholds, levels)
+        if policy == "quantile":
+            lev = assign_levels_quantile_row(mass[b, h, I], thresholds, levels,
+                                             min(I + 1, nkb) if causal else nkb)
+        else:
+            lev = assign_levels_row(mass[b, h, I], thresholds, levels)
         cos_row = None if blockcos is None else blockcos[b, h // hq_per_kv]
         out[b, h, I] = apply_forced_rules(lev, I, block, levels, causal, n_dense_prefix, cos_row, cos_min)
     return out.astype(np.uint8)
@@ -330,6 +395,27 @@ def ambiguous_pairs(mass: np.ndarray, thresholds, eps: float = 1e-6, rows=None,
                 if lo - eps <= t <= hi + eps:
                     amb[b, h, I, J] = True
             if blockcos is not None and cos_min > -2.0 and abs(blockcos[b, h // hq_per_kv, J] - cos_min) <= eps:
+                amb[b, h, I, J] = True
+    return amb
+
+
+def ambiguous_pairs_quantile(mass: np.ndarray, thresholds, levels: int, causal: bool, eps: float = 1e-6,
+                             rows=None) -> np.ndarray:
+    """Pairs whose rank-based level (reading R10) may legitimately differ
+    between an fp32 and an fp64 evaluation: the ranks that near-equal masses
+    (relative eps) allow for block J span a level boundary."""
+    B, Hq, nqb, nkb = mass.shape
+    amb = np.zeros(mass.shape, dtype=bool)
+    if rows is None:
+        rows = [(b, h, I) for b in range(B) for h in range(Hq) for I in range(nqb)]
+    for b, h, I in rows:
+        m = mass[b, h, I]
+        nv = min(I + 1, nkb) if causal else nkb
+        for J in range(nkb):
+            r_lo = int((m > m[J] * (1 + eps)).sum())
+            r_hi = int((m >= m[J] * (1 - eps)).sum()) - 1
+            lev = {sum(1 for t in thresholds if t <= r / nv) for r in (r_lo, r_hi)}
+            if len(lev) > 1:
                 amb[b, h, I, J] = True
     return amb
 

@@ -15,13 +15,22 @@ something other than itself.
                         block-summed full softmax (torch); sum over J == 1
   assign_levels_row     hand-computed golden cases; monotone in rank; top = 0
   apply_forced_rules    hand-computed golden cases
+  assign_levels_quantile_row
+                        hand-computed golden cases; L = 1 with t_0 = k/n keeps
+                        exactly numpy's stable top-k; per-level counts n/L
+  block_means /         hand-computed golden case (ragged block, causal); torch
+  meankey_mass          avg_pool1d + torch.softmax (independent routines); sum
+                        over J == 1; token order inside a block and a common
+                        shift of every key change nothing
   attention             all-level-0 == torch SDPA (fp64); expanded-KV SDPA
                         equivalence; identical-group invariance; NaN in a
                         skipped block changes nothing; pure-Python brute force
                         over an exhaustive {0,1,2,3,SKIP} mask; empty rows
   mutation tests        planted mistakes (bias sign, dropped bias, sum instead of
                         mean, wrong block width, inclusive prefix, transposed
-                        antidiagonal) each make a pin fail
+                        antidiagonal, rank off by one, ragged mean over the
+                        full block, transposed mean-key logits) each make a pin
+                        fail
 """
 import json
 import math
@@ -523,3 +532,128 @@ def test_mutation_transposed_attention_operand(monkeypatch):
     monkeypatch.setattr(O, "gather_keys", bad)
     with pytest.raises(AssertionError):
         test_attention_level0_is_dense_sdpa(False)
+
+
+# --------------------------------------------------------------------------------------
+# rank-based (quantile / top-k) levels, reading R10
+# --------------------------------------------------------------------------------------
+
+def test_quantile_golden(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "quantile_hand.json")))
+    for c in g["cases"]:
+        got = O.assign_levels_quantile_row(c["mass"], c["thresholds"], c["levels"], c["n_visible"])
+        assert list(got) == c["expect"], (c, list(got))
+
+
+@pytest.mark.parametrize("n,k", [(16, 5), (32, 1), (8, 8), (64, 40)])
+def test_quantile_binary_is_topk(n, k):
+    """L = 1 and t_0 = k/n (exact in binary for these n) keep exactly the k
+    heaviest blocks: numpy's stable argsort of -mass is the independent
+    routine."""
+    m = RNG.random(n)
+    got = O.assign_levels_quantile_row(m, [k / n], 1, n)
+    keep = set(np.argsort(-m, kind="stable")[:k].tolist())
+    assert {J for J in range(n) if got[J] == 0} == keep
+    assert all(got[J] == SKIP for J in range(n) if J not in keep)
+
+
+def test_quantile_level_counts_and_monotone():
+    n, L = 32, 4
+    m = RNG.random(n)
+    got = O.assign_levels_quantile_row(m, [0.25, 0.5, 0.75, 1.0], L, n)
+    assert [int((got == l).sum()) for l in range(L)] == [8, 8, 8, 8]
+    order = np.argsort(-m, kind="stable")
+    assert all(got[order[i]] <= got[order[i + 1]] for i in range(n - 1))
+
+
+# --------------------------------------------------------------------------------------
+# mean-key scorer, reading R11
+# --------------------------------------------------------------------------------------
+
+def _meankey_golden_case(golden_dir, causal, mod=O):
+    g = json.load(open(os.path.join(golden_dir, "meankey_hand.json")))
+    q = torch.tensor(g["q"], dtype=torch.float64)[None, None]
+    k = torch.tensor(g["k"], dtype=torch.float64)[None, None]
+    got = mod.meankey_mass(q, k, g["block"], g["sm_scale"], causal)[0, 0]
+    want = np.array(g["expect_causal" if causal else "expect"])
+    return np.abs(got - want).max()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_meankey_golden(golden_dir, causal):
+    assert _meankey_golden_case(golden_dir, causal) <= 1e-15
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_meankey_vs_torch(causal):
+    """Block means from torch's avg_pool1d (ceil_mode, pad excluded from the
+    count), logits and softmax from torch: an independent path."""
+    B, Hq, Hkv, N, d, blk = 2, 4, 2, 77, 8, 16
+    q = torch.randn(B, Hq, N, d, dtype=torch.float64)
+    k = torch.randn(B, Hkv, N, d, dtype=torch.float64)
+    def pool(x):
+        y = x.reshape(-1, N, d).transpose(1, 2)                     # [*, d, N]
+        y = torch.nn.functional.avg_pool1d(y, blk, blk, ceil_mode=True, count_include_pad=False)
+        return y.transpose(1, 2).reshape(x.shape[0], x.shape[1], -1, d)
+    qm, km = pool(q), pool(k)
+    km = km.repeat_interleave(Hq // Hkv, dim=1)
+    z = 0.3 * qm @ km.transpose(-1, -2)
+    nb = z.shape[-1]
+    if causal:
+        z = z.masked_fill(torch.ones(nb, nb, dtype=torch.bool).triu(1), float("-inf"))
+    want = torch.softmax(z, dim=-1).numpy()
+    got = O.meankey_mass(q, k, blk, 0.3, causal)
+    assert np.abs(got - want).max() <= 1e-14
+
+
+def test_meankey_invariants():
+    B, H, N, d, blk = 1, 2, 100, 6, 20
+    q = torch.randn(B, H, N, d, dtype=torch.float64)
+    k = torch.randn(B, H, N, d, dtype=torch.float64)
+    base = O.meankey_mass(q, k, blk, 0.5, False)
+    assert np.allclose(base.sum(axis=-1), 1.0, atol=1e-14)
+    perm = torch.cat([torch.randperm(blk) + J * blk for J in range(N // blk)])
+    assert np.abs(O.meankey_mass(q[:, :, perm], k[:, :, perm], blk, 0.5, False) - base).max() <= 1e-13
+    shifted = O.meankey_mass(q, k + torch.randn(d, dtype=torch.float64), blk, 0.5, False)
+    assert np.abs(shifted - base).max() <= 1e-12
+    causal = O.meankey_mass(q, k, blk, 0.5, True)[0, 0]
+    assert np.all(causal[np.triu_indices(N // blk, 1)] == 0.0) and causal[0, 0] == 1.0
+
+
+def test_mutation_quantile_rank_off_by_one(monkeypatch, golden_dir):
+    orig = O.assign_levels_quantile_row
+
+    def planted(mass_row, thresholds, levels, n_visible=None):
+        n = len(mass_row)
+        nv = n if n_visible is None else n_visible
+        return orig(mass_row, [t - 1.0 / nv for t in thresholds], levels, nv)   # (r + 1) / n
+    monkeypatch.setattr(O, "assign_levels_quantile_row", planted)
+    with pytest.raises(AssertionError):
+        test_quantile_golden(golden_dir)
+
+
+def test_mutation_ragged_mean_over_full_block(monkeypatch, golden_dir):
+    def planted(x, block):
+        x = O._f64(x)
+        B, H, N, d = x.shape
+        nb = -(-N // block)
+        out = np.empty((B, H, nb, d))
+        for J in range(nb):
+            out[:, :, J] = x[:, :, J * block:min((J + 1) * block, N)].sum(axis=2) / block
+        return out
+    monkeypatch.setattr(O, "block_means", planted)
+    assert _meankey_golden_case(golden_dir, False) > 1e-3
+
+
+def test_mutation_meankey_transposed(monkeypatch, golden_dir):
+    orig = O.block_means
+
+    # transposed logits: score query block J against key block I
+    def planted(q, k, block, sm_scale, causal=False, rows=None):
+        qm, km = orig(q, block), orig(k, block)
+        z = sm_scale * (qm[0, 0] @ km[0, 0].T).T
+        if causal:
+            z = np.where(np.tril(np.ones_like(z)) > 0, z, -np.inf)
+        return O._softmax_rows(z)[None, None]
+    monkeypatch.setattr(O, "meankey_mass", planted)
+    assert _meankey_golden_case(golden_dir, False) > 1e-3
