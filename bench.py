@@ -172,9 +172,11 @@ class Path:
         dev = q.device
         self.shape = P.make_shape(w.B, w.Hq, w.Hkv, w.N, w.d, w.block, w.levels, w.causal,
                                   P.PSA_DT_FP32 if w.dtype == "fp32" else P.PSA_DT_BF16)
-        mode = P.PSA_MASK_SAMPLE if w.mask_mode == "sample" else P.PSA_MASK_ANTIDIAG
+        mode = {"sample": P.PSA_MASK_SAMPLE, "meankey": P.PSA_MASK_MEANKEY}.get(w.mask_mode, P.PSA_MASK_ANTIDIAG)
+        policy = P.PSA_POLICY_QUANTILE if w.policy == "quantile" else P.PSA_POLICY_MASS
         self.params = P.make_params(mode, w.thresholds or (0.6, 0.8, 0.9, 0.95)[:w.levels], w.sm_scale,
-                                    stride=w.stride, cos_min=w.cos_min, n_dense_prefix=w.n_dense_prefix)
+                                    stride=w.stride, cos_min=w.cos_min, n_dense_prefix=w.n_dense_prefix,
+                                    policy=policy)
         self.kp, self.vp = P.pyramid_buffers(self.shape, dev, q.dtype)
         nb = w.nqb
         self.bc = torch.empty(w.B, w.Hkv, nb, dtype=torch.float32, device=dev) if w.cos_min > -2 else None
@@ -305,7 +307,7 @@ def run_psa(args, rank, world, local_rank):
         "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "fp32 in, bf16 MMA",
         "data": "synthetic (smooth Gaussian field + noise, seeded)" if w.recipe == "field" else "synthetic iid N(0,1)",
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "block": w.block,
-                   "levels": w.levels, "causal": w.causal, "mask": w.mask_mode, "thresholds": list(w.thresholds),
+                   "levels": w.levels, "causal": w.causal, "mask": w.mask_mode, "policy": w.policy, "thresholds": list(w.thresholds),
                    "l2": "inputs (%.2f GB) larger than L2; no flush" % ((q.numel() + 2 * k.numel()) * q.element_size() / 1e9),
                    "step": "psa_build_pyramid + psa_make_mask + psa_attention_fwd",
                    "parallelism": "replicas, one workload instance per GPU" if world > 1 else "single GPU"},
@@ -381,11 +383,13 @@ def oracle_sample(w, q, k, v, n_blocks, seed=0, mask_dev=None):
     else:
         if w.mask_mode == "sample":
             mass = O.sampling_mass(qh, kh, w.block, w.sm_scale, w.causal, rows=rows)
+        elif w.mask_mode == "meankey":
+            mass = O.meankey_mass(qh, kh, w.block, w.sm_scale, w.causal, rows=rows)
         else:
             mass = O.antidiag_mass(qh, kh, w.block, w.stride, w.sm_scale, w.causal, rows=rows)
         cos = O.block_cosine(kh, w.block) if w.cos_min > -2 else None
         mask = O.make_mask(mass, w.thresholds, w.levels, w.block, w.causal, w.n_dense_prefix, cos, w.cos_min,
-                           1, rows=rows)
+                           1, rows=rows, policy=w.policy)
     O.attention(qh, kl, vl, mask, w.block, w.sm_scale, w.causal, rows=rows)
     dt = time.perf_counter() - t0
     sub = np.full_like(mask, 0xFF)
@@ -449,6 +453,10 @@ def workload(args) -> W.Workload:
     """The chosen preset; --heads shrinks it (same shape per head) for
     profiling captures that must stay a few GB on the device."""
     w = W.PRESETS[args.config]
+    mask_mode, policy = getattr(args, "mask_mode", "preset"), getattr(args, "policy", "mass")
+    if mask_mode != "preset" or policy != "mass":
+        mode = w.mask_mode if mask_mode == "preset" else mask_mode
+        w = w.replace(name="%s[mask=%s,%s]" % (w.name, mode, policy), mask_mode=mode, policy=policy)
     if args.heads:
         hq = args.heads
         hkv = max(1, hq * w.Hkv // w.Hq)
@@ -469,6 +477,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--verbose", action="store_true", help="progress and per-stage warm-up times on stderr")
     ap.add_argument("--heads", type=int, default=0, help="override the query head count (profiling captures)")
+    ap.add_argument("--mask-mode", default="preset", choices=["preset", "sample", "antidiag", "meankey"],
+                    help="block scorer of the mask stage (default: the preset's)")
+    ap.add_argument("--policy", default="mass", choices=["mass", "quantile"], help="level policy of the mask stage")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

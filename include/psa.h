@@ -66,8 +66,14 @@ typedef enum { PSA_DT_BF16 = 0, PSA_DT_FP32 = 1 } psa_dtype_t;
 
 typedef enum {
   PSA_MASK_SAMPLE = 0,       /* generation task: sampled-query scoring */
-  PSA_MASK_ANTIDIAG = 1      /* understanding task: antidiagonal scoring */
+  PSA_MASK_ANTIDIAG = 1,     /* understanding task: antidiagonal scoring */
+  PSA_MASK_MEANKEY = 2       /* cheap scorer: block-mean queries against block-mean keys */
 } psa_mask_mode_t;
+
+typedef enum {
+  PSA_POLICY_MASS = 0,       /* level = number of thresholds <= the exclusive prefix of the mass */
+  PSA_POLICY_QUANTILE = 1    /* level = number of thresholds <= rank / visible blocks */
+} psa_level_policy_t;
 
 #define PSA_SKIP 0xFF
 #define PSA_MAX_LEVELS 4
@@ -97,6 +103,7 @@ typedef struct {
   float cos_min;             /* cosine gate; <= -2 disables it */
   int32_t n_dense_prefix;    /* tokens [0, n) are text: their blocks stay level 0 */
   float sm_scale;            /* softmax scale of the score; usually 1/sqrt(d) */
+  int32_t policy;            /* psa_level_policy_t; 0 (the default when zeroed) = by mass */
 } psa_mask_params_t;
 
 /* ------------------------------------------------------------------------
@@ -132,11 +139,22 @@ PSA_API psa_status_t psa_build_pyramid(const psa_shape_t* shape, const void* k, 
  * sum_s q[a*S + S-1-s] . k[c*S + s]; softmax over key groups c (c <= a when
  * causal); mass[I, J] = mean over the query groups of I of the probability
  * in the key groups of J.  Requires N % S == 0.
- * Levels: per row (b, h, I) rank J by mass (descending, ties to lower J),
+ * Score, PSA_MASK_MEANKEY (skill page, Core Technique: a block scored by
+ * the query against the mean of its keys): qbar_I and kbar_J are the means
+ * of the valid tokens of query block I and key block J (fp64); mass[I, J] =
+ * softmax over J of sm_scale * qbar_I . kbar_J (J <= I when causal).  It
+ * reads Q and K once and needs no N alignment.
+ * Levels, policy PSA_POLICY_MASS (summary article, Results: threshold-based
+ * levels): per row (b, h, I) rank J by mass (descending, ties to lower J),
  * take the exclusive prefix C_J, level = #{t_l <= C_J}, SKIP when that count
- * reaches L; then blocks holding a token < n_dense_prefix (as query or key
- * block) -> 0; if cos_min > -2 and level >= 1 and blockcos[b, h_kv, J] <
- * cos_min -> 0; if causal, J > I -> SKIP and J == I -> 0.
+ * reaches L.  Policy PSA_POLICY_QUANTILE (the rank-based alternative of the
+ * same ablation): the block at rank r gets level #{t_l <= r / n_vis}, n_vis
+ * = I + 1 when causal, else nKB; with L = 1 and t_0 = k / n_vis this keeps
+ * the k heaviest blocks (a binary top-k mask).  Either policy with L = 1
+ * gives a binary {0, SKIP} mask.  Then blocks holding a token <
+ * n_dense_prefix (as query or key block) -> 0; if cos_min > -2 and level >=
+ * 1 and blockcos[b, h_kv, J] < cos_min -> 0; if causal, J > I -> SKIP and
+ * J == I -> 0.
  *
  * mask: uint8 [B, Hq, nQB, nKB] (PSA_SKIP = 0xFF).  mass_out (optional):
  * fp32 [B, Hq, nQB, nKB].  blockcos is required iff cos_min > -2.

@@ -54,10 +54,12 @@ def run_attention(shape, q, k, v, kp, vp, mask, sm_scale, want_lse=True, ws=None
     return out, lse, ws
 
 
-def params_for(w: W.Workload):
-    mode = P.PSA_MASK_SAMPLE if w.mask_mode == "sample" else P.PSA_MASK_ANTIDIAG
-    return P.make_params(mode, w.thresholds, w.sm_scale, stride=w.stride, cos_min=w.cos_min,
-                         n_dense_prefix=w.n_dense_prefix)
+MODES = {"sample": P.PSA_MASK_SAMPLE, "antidiag": P.PSA_MASK_ANTIDIAG, "meankey": P.PSA_MASK_MEANKEY}
+
+
+def params_for(w: W.Workload, policy: int = P.PSA_POLICY_MASS):
+    return P.make_params(MODES[w.mask_mode], w.thresholds, w.sm_scale, stride=w.stride, cos_min=w.cos_min,
+                         n_dense_prefix=w.n_dense_prefix, policy=policy)
 
 
 def shape_for(w: W.Workload):

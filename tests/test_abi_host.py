@@ -133,6 +133,43 @@ def test_mask_rejects_bad_params():
     assert call(P.make_params(P.PSA_MASK_SAMPLE, (0.6, 0.8, 0.9, 0.95), 0.125, cos_min=0.8)) == P.PSA_ERR_INVALID_ARG
     assert call(good, mask=None) == P.PSA_ERR_INVALID_ARG
     assert call(good, ws_bytes=16) == P.PSA_ERR_WORKSPACE
+    assert call(P.make_params(P.PSA_MASK_SAMPLE, (0.6, 0.8, 0.9, 0.95), 0.125, policy=2)) == P.PSA_ERR_INVALID_ARG
+    assert call(P.make_params(3, (0.6, 0.8, 0.9, 0.95), 0.125)) == P.PSA_ERR_INVALID_ARG
+    mk = P.make_params(P.PSA_MASK_MEANKEY, (0.6, 0.8, 0.9, 0.95), 0.125, policy=P.PSA_POLICY_QUANTILE)
+    assert call(mk, ws_bytes=16) == P.PSA_ERR_WORKSPACE
+
+
+def test_meankey_workspace_needs_no_alignment():
+    """The mean-key scorer takes any N (sampling needs N % (block/8) == 0);
+    its workspace holds the score rows and the fp64 block means."""
+    s = P.make_shape(2, 4, 2, 1001, 128, 64, 1)       # one level: a binary mask, any N
+    nb = -(-1001 // 64)
+    samp = P.make_params(P.PSA_MASK_SAMPLE, (0.9,), 0.1)
+    mk = P.make_params(P.PSA_MASK_MEANKEY, (0.9,), 0.1)
+    assert P.psa_mask_workspace_bytes(s, samp) == 0
+    need = P.psa_mask_workspace_bytes(s, mk)
+    floor = 2 * 4 * nb * nb * 4 + 2 * 2 * 4 * nb * 4 + 2 * 4 * nb * 128 * 8 + 2 * 2 * nb * 128 * 8
+    assert floor <= need <= floor + 8 * 256 + 256
+
+
+def test_struct_layouts_match_the_header(tmp_path):
+    """sizeof / offsetof of the two parameter structs, from gcc compiling the
+    public header, against the ctypes binding."""
+    prog = tmp_path / "layout.c"
+    fields_s = [f for f, _ in P.Shape._fields_]
+    fields_m = [f for f, _ in P.MaskParams._fields_]
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "psa.h"', 'int main(void) {',
+             '  printf("%zu\\n", sizeof(psa_shape_t));', '  printf("%zu\\n", sizeof(psa_mask_params_t));']
+    lines += ['  printf("%%zu\\n", offsetof(psa_shape_t, %s));' % f for f in fields_s]
+    lines += ['  printf("%%zu\\n", offsetof(psa_mask_params_t, %s));' % f for f in fields_m]
+    lines += ['  return 0;', '}']
+    prog.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(prog), "-o", str(exe)], check=True)
+    got = [int(x) for x in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
+    want = [ctypes.sizeof(P.Shape), ctypes.sizeof(P.MaskParams)]
+    want += [getattr(P.Shape, f).offset for f in fields_s] + [getattr(P.MaskParams, f).offset for f in fields_m]
+    assert got == want
 
 
 def test_binding_refuses_cpu_tensors():

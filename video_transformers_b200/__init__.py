@@ -21,7 +21,8 @@ LIB_PATH = os.path.join(_HERE, "libpsa.so")
 
 PSA_OK, PSA_ERR_INVALID_ARG, PSA_ERR_UNSUPPORTED, PSA_ERR_WORKSPACE, PSA_ERR_CUDA, PSA_ERR_TIMEOUT = range(6)
 PSA_DT_BF16, PSA_DT_FP32 = 0, 1
-PSA_MASK_SAMPLE, PSA_MASK_ANTIDIAG = 0, 1
+PSA_MASK_SAMPLE, PSA_MASK_ANTIDIAG, PSA_MASK_MEANKEY = 0, 1, 2
+PSA_POLICY_MASS, PSA_POLICY_QUANTILE = 0, 1
 PSA_SKIP = 0xFF
 
 EXPORTS = [
@@ -48,7 +49,7 @@ class MaskParams(ctypes.Structure):
     _fields_ = [("mode", ctypes.c_int32), ("n_samples", ctypes.c_int32), ("stride", ctypes.c_int32),
                 ("thresholds", ctypes.c_float * 8), ("n_thresholds", ctypes.c_int32),
                 ("cos_min", ctypes.c_float), ("n_dense_prefix", ctypes.c_int32),
-                ("sm_scale", ctypes.c_float)]
+                ("sm_scale", ctypes.c_float), ("policy", ctypes.c_int32)]
 
 
 def _load(path: str = LIB_PATH):
@@ -125,9 +126,10 @@ def shape_of(q: torch.Tensor, k: torch.Tensor, block: int, levels: int, causal: 
 
 
 def make_params(mode: int, thresholds: Sequence[float], sm_scale: float, stride: int = 8,
-                cos_min: float = -3.0, n_dense_prefix: int = 0, n_samples: int = 8) -> MaskParams:
+                cos_min: float = -3.0, n_dense_prefix: int = 0, n_samples: int = 8,
+                policy: int = PSA_POLICY_MASS) -> MaskParams:
     th = (ctypes.c_float * 8)(*([float(t) for t in thresholds] + [0.0] * (8 - len(thresholds))))
-    return MaskParams(mode, n_samples, stride, th, len(thresholds), cos_min, n_dense_prefix, sm_scale)
+    return MaskParams(mode, n_samples, stride, th, len(thresholds), cos_min, n_dense_prefix, sm_scale, policy)
 
 
 def psa_version() -> int:

@@ -18,7 +18,7 @@ OBJ = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libpsa.so")
 ROOT = os.path.dirname(HERE)
 
-SOURCES = ["api.cu", "pyramid.cu", "mask.cu", "plan.cu", "attn.cu"]
+SOURCES = ["api.cu", "pyramid.cu", "mask.cu", "meankey.cu", "plan.cu", "attn.cu"]
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-lineinfo", "-O3", "-std=c++17",

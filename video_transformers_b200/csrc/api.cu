@@ -140,7 +140,7 @@ size_t pyr_bytes(const psa_shape_t* s, size_t esize) { return pyr_level_offset(s
 
 // ------------------------------------------------------------------ mask workspace
 struct MaskLayout {
-  size_t status, blocklse, rowlse, q16, k16, total;
+  size_t status, blocklse, rowlse, q16, k16, qmean, kmean, total;
   int rows, step, rpb, cols, cpb;
 };
 MaskLayout mask_layout(const psa_shape_t* s, const psa_mask_params_t* p) {
@@ -153,6 +153,12 @@ MaskLayout mask_layout(const psa_shape_t* s, const psa_mask_params_t* p) {
     L.rows = nqb * 8;
     L.cols = s->N;
     L.cpb = s->block;
+  } else if (p->mode == PSA_MASK_MEANKEY) {
+    L.step = s->block;
+    L.rpb = 1;
+    L.rows = nqb;
+    L.cols = nkb;
+    L.cpb = 1;
   } else {
     L.step = p->stride;
     L.rpb = s->block / p->stride;
@@ -165,7 +171,11 @@ MaskLayout mask_layout(const psa_shape_t* s, const psa_mask_params_t* p) {
   L.status = 0;
   L.blocklse = off; off = align_up(off + BHq * nkb * L.rows * 4, 256);
   L.rowlse = off;   off = align_up(off + 2 * BHq * L.rows * 4, 256);   // one partial per epilogue warpgroup
-  if (s->dtype == PSA_DT_FP32) {
+  if (p->mode == PSA_MASK_MEANKEY) {
+    // block means in fp64; the mean-key scorer reads the inputs directly
+    L.qmean = off; off = align_up(off + BHq * nqb * s->d * 8, 256);
+    L.kmean = off; off = align_up(off + static_cast<size_t>(s->B) * s->Hkv * nkb * s->d * 8, 256);
+  } else if (s->dtype == PSA_DT_FP32) {
     L.q16 = off; off = align_up(off + BHq * s->N * s->d * 2, 256);
     L.k16 = off; off = align_up(off + static_cast<size_t>(s->B) * s->Hkv * s->N * s->d * 2, 256);
   }
@@ -175,7 +185,10 @@ MaskLayout mask_layout(const psa_shape_t* s, const psa_mask_params_t* p) {
 
 psa_status_t check_mask_params(const psa_shape_t* s, const psa_mask_params_t* p) {
   if (!p) return fail(PSA_ERR_INVALID_ARG, "params is NULL");
-  if (p->mode != PSA_MASK_SAMPLE && p->mode != PSA_MASK_ANTIDIAG) return fail(PSA_ERR_INVALID_ARG, "unknown mask mode %d", p->mode);
+  if (p->mode != PSA_MASK_SAMPLE && p->mode != PSA_MASK_ANTIDIAG && p->mode != PSA_MASK_MEANKEY)
+    return fail(PSA_ERR_INVALID_ARG, "unknown mask mode %d", p->mode);
+  if (p->policy != PSA_POLICY_MASS && p->policy != PSA_POLICY_QUANTILE)
+    return fail(PSA_ERR_INVALID_ARG, "unknown level policy %d", p->policy);
   if (p->n_thresholds != s->levels) return fail(PSA_ERR_INVALID_ARG, "n_thresholds %d != levels %d", p->n_thresholds, s->levels);
   for (int i = 0; i < p->n_thresholds; ++i)
     if (!(p->thresholds[i] == p->thresholds[i])) return fail(PSA_ERR_INVALID_ARG, "threshold %d is NaN", i);
@@ -184,6 +197,8 @@ psa_status_t check_mask_params(const psa_shape_t* s, const psa_mask_params_t* p)
   if (p->mode == PSA_MASK_SAMPLE) {
     if (p->n_samples != 8) return fail(PSA_ERR_UNSUPPORTED, "n_samples must be 8");
     if (s->N % (s->block / 8)) return fail(PSA_ERR_UNSUPPORTED, "sampling needs N %% (block/8) == 0");
+  } else if (p->mode == PSA_MASK_MEANKEY) {
+    // no alignment needed: the block means read every token once
   } else {
     const int S = p->stride;
     if (S != 1 && S != 2 && S != 4 && S != 8 && S != 16) return fail(PSA_ERR_UNSUPPORTED, "stride %d not in {1,2,4,8,16}", S);
@@ -295,6 +310,38 @@ psa_status_t psa_make_mask(const psa_shape_t* s, const psa_mask_params_t* p, con
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* w = static_cast<char*>(ws);
   const int64_t BHq = static_cast<int64_t>(s->B) * s->Hq, BHkv = static_cast<int64_t>(s->B) * s->Hkv;
+  const int nkb = static_cast<int>(ceil_div(s->N, s->block));
+  psa::SelectArgs se{};
+  se.B = s->B; se.Hq = s->Hq; se.Hkv = s->Hkv; se.N = s->N; se.block = s->block;
+  se.nqb = nkb; se.nkb = nkb; se.levels = s->levels; se.causal = s->causal != 0;
+  se.mode = p->mode; se.rows = L.rows; se.rows_per_block = L.rpb; se.step = L.step;
+  se.policy = p->policy;
+  for (int i = 0; i < 8; ++i) se.thresholds[i] = i < p->n_thresholds ? p->thresholds[i] : 3.0e38f;
+  se.cos_min = p->cos_min;
+  se.n_dense_prefix = p->n_dense_prefix;
+  se.blockcos = p->cos_min > -2.f ? blockcos : nullptr;
+  se.mask = mask;
+  se.mass_out = mass_out;
+  se.blocklse = reinterpret_cast<float*>(w + L.blocklse);
+  se.rowlse = reinterpret_cast<float*>(w + L.rowlse);
+  if (p->mode == PSA_MASK_MEANKEY) {
+    const int es = static_cast<int>(elem_size(s->dtype));
+    double* qm = reinterpret_cast<double*>(w + L.qmean);
+    double* km = reinterpret_cast<double*>(w + L.kmean);
+    PSA_CUDA(psa::launch_blockmean(q, qm, BHq, s->N, s->d, s->block, es, false, st), "query block means");
+    PSA_CUDA(psa::launch_blockmean(k, km, BHkv, s->N, s->d, s->block, es, true, st), "key block means");
+    psa::MeanKeyArgs ma{};
+    ma.BHq = static_cast<int>(BHq); ma.Hq = s->Hq; ma.Hkv = s->Hkv; ma.d = s->d;
+    ma.nqb = nkb; ma.nkb = nkb; ma.causal = s->causal != 0;
+    ma.scale_log2 = static_cast<double>(p->sm_scale) * 1.4426950408889634;
+    ma.qmean = qm; ma.kmeanT = km;
+    ma.blocklse = reinterpret_cast<float*>(w + L.blocklse);
+    ma.rowlse = reinterpret_cast<float*>(w + L.rowlse);
+    PSA_CUDA(psa::launch_meankey_score(ma, st), "mean-key score launch");
+    se.S = 1;
+    PSA_CUDA(psa::launch_select(se, st), "select launch");
+    return PSA_OK;
+  }
   const void* q16 = q;
   const void* k16 = k;
   if (s->dtype == PSA_DT_FP32) {
@@ -307,7 +354,6 @@ psa_status_t psa_make_mask(const psa_shape_t* s, const psa_mask_params_t* p, con
   PSA_TRY(map4(&mA, q16, BHq, s->N, s->d, L.step));
   PSA_TRY(map4(&mB, k16, BHkv, s->N, s->d, p->mode == PSA_MASK_SAMPLE ? 1 : p->stride));
   psa::ScoreArgs sa{};
-  const int nkb = static_cast<int>(ceil_div(s->N, s->block));
   sa.BHq = static_cast<int>(BHq); sa.Hq = s->Hq; sa.Hkv = s->Hkv; sa.N = s->N; sa.d = s->d;
   sa.block = s->block; sa.nkb = nkb; sa.mode = p->mode; sa.step = L.step;
   sa.S = p->mode == PSA_MASK_SAMPLE ? 1 : p->stride;
@@ -319,18 +365,7 @@ psa_status_t psa_make_mask(const psa_shape_t* s, const psa_mask_params_t* p, con
   sa.rowlse = reinterpret_cast<float*>(w + L.rowlse);
   sa.status = reinterpret_cast<int*>(w + L.status);
   PSA_CUDA(psa::launch_score(&mA, &mB, sa, num_sms(), st), "score launch");
-  psa::SelectArgs se{};
-  se.B = s->B; se.Hq = s->Hq; se.Hkv = s->Hkv; se.N = s->N; se.block = s->block;
-  se.nqb = nkb; se.nkb = nkb; se.levels = s->levels; se.causal = s->causal != 0;
-  se.mode = p->mode; se.S = sa.S; se.rows = L.rows; se.rows_per_block = L.rpb; se.step = L.step;
-  for (int i = 0; i < 8; ++i) se.thresholds[i] = i < p->n_thresholds ? p->thresholds[i] : 3.0e38f;
-  se.cos_min = p->cos_min;
-  se.n_dense_prefix = p->n_dense_prefix;
-  se.blocklse = sa.blocklse;
-  se.rowlse = sa.rowlse;
-  se.blockcos = p->cos_min > -2.f ? blockcos : nullptr;
-  se.mask = mask;
-  se.mass_out = mass_out;
+  se.S = sa.S;
   PSA_CUDA(psa::launch_select(se, st), "select launch");
   return PSA_OK;
 }

@@ -40,9 +40,25 @@ struct ScoreArgs {
 cudaError_t launch_score(const CUtensorMap* mapA, const CUtensorMap* mapB, const ScoreArgs& a,
                          int num_sms, cudaStream_t s);
 
+// Mean-key scorer (mode 2): block means of Q and K in fp64, then one score
+// row per query block written in the same [BHq][nkb][rows] / [2][BHq][rows]
+// log2-domain layout the score kernel uses (rows = nqb, one row per block).
+cudaError_t launch_blockmean(const void* x, double* out, int64_t BH, int N, int d, int block, int elem,
+                             bool transpose, cudaStream_t s);
+struct MeanKeyArgs {
+  int BHq, Hq, Hkv, d, nqb, nkb, causal;
+  double scale_log2;        // sm_scale * log2(e)
+  const double* qmean;      // [BHq][nqb][d]
+  const double* kmeanT;     // [BHkv][d][nkb]
+  float* blocklse;          // [BHq][nkb][nqb]
+  float* rowlse;            // [2][BHq][nqb]
+};
+cudaError_t launch_meankey_score(const MeanKeyArgs& a, cudaStream_t s);
+
 struct SelectArgs {
   int B, Hq, Hkv, N, block, nqb, nkb, levels, causal;
   int mode, S, rows, rows_per_block, step;
+  int policy;               // 0 levels by exclusive prefix of mass, 1 by rank / visible blocks
   float thresholds[8];
   float cos_min;
   int n_dense_prefix;

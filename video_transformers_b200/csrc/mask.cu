@@ -13,7 +13,8 @@
 //                the SM.
 // select_kernel  one CTA per (b, h, query block): block masses from the
 //                LSEs, a bitonic sort (mass descending, index ascending), an
-//                fp64 exclusive scan, thresholds, forced rules.
+//                fp64 exclusive scan, levels by that prefix (or by rank for
+//                the quantile policy), forced rules.
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
@@ -368,11 +369,15 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectArgs a)
   for (int w = 0; w < wid; ++w) wbase += warp_tot[w];
   double C = wbase + incl - local;
   __syncthreads();
+  // rank policy: the visible blocks are the first n_vis ranks (blocks past
+  // the diagonal have mass exactly 0 and lose ties to lower indices)
+  const int n_vis = a.causal ? min(I + 1, a.nkb) : a.nkb;
   for (int i = k0; i < min(k0 + per, a.nkb); ++i) {
     const int J = static_cast<int>(key[i] & 0xFFFFFFFFu);
     const double mJ = scan[J];
+    const double x = a.policy == 1 ? static_cast<double>(i) / static_cast<double>(n_vis) : C;
     int lev = 0;
-    for (int l = 0; l < a.levels; ++l) lev += (static_cast<double>(a.thresholds[l]) <= C);
+    for (int l = 0; l < a.levels; ++l) lev += (static_cast<double>(a.thresholds[l]) <= x);
     int out = lev >= a.levels ? PSA_SKIP : lev;
     if (a.n_dense_prefix > 0 &&
         (static_cast<int64_t>(I) * a.block < a.n_dense_prefix || static_cast<int64_t>(J) * a.block < a.n_dense_prefix))

@@ -48,8 +48,9 @@ class Workload:
     grid: Tuple[int, int, int] = (0, 0, 0)   # (T, H, W) of the video latent
     n_text: int = 0                 # iid text tokens placed before the video tokens
     n_iid: int = 0                  # total tokens for the iid recipe
-    mask_mode: str = "given"        # "given" (drawn here), "sample" or "antidiag"
+    mask_mode: str = "given"        # "given" (drawn here), "sample", "antidiag" or "meankey"
     thresholds: Tuple[float, ...] = ()
+    policy: str = "mass"            # level policy: "mass" (thresholds on the mass prefix) or "quantile"
     n_samples: int = 8
     stride: int = 8
     cos_min: float = -3.0           # <= -2 disables the cosine gate
