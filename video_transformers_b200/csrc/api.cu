@@ -328,7 +328,7 @@ psa_status_t psa_make_mask(const psa_shape_t* s, const psa_mask_params_t* p, con
     const int es = static_cast<int>(elem_size(s->dtype));
     double* qm = reinterpret_cast<double*>(w + L.qmean);
     double* km = reinterpret_cast<double*>(w + L.kmean);
-    PSA_CUDA(psa::launch_blockmean(q, qm, BHq, s->N, s->d, s->block, es, false, st), "query block means");
+    PSA_CUDA(psa::launch_blockmean(q, qm, BHq, s->N, s->d, s->block, es, true, st), "query block means");
     PSA_CUDA(psa::launch_blockmean(k, km, BHkv, s->N, s->d, s->block, es, true, st), "key block means");
     psa::MeanKeyArgs ma{};
     ma.BHq = static_cast<int>(BHq); ma.Hq = s->Hq; ma.Hkv = s->Hkv; ma.d = s->d;

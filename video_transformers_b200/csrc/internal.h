@@ -11,6 +11,18 @@
 
 namespace psa {
 
+// 2^x for x <= 0 (a difference of log-sum-exps, log2 domain) with relative
+// error about 2.5e-7: x = n + f with n = floor(x) in fp64, 2^f of the
+// fraction rounded to fp32 from the special-function unit, 2^n applied to
+// the exponent exactly.  Arguments below -1000 give 0.
+__device__ __forceinline__ double exp2_split(double x) {
+  if (x < -1000.0) return 0.0;
+  const double n = floor(x);
+  float p;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(p) : "f"(static_cast<float>(x - n)));
+  return ldexp(static_cast<double>(p), static_cast<int>(n));
+}
+
 // ---- stage 1 -------------------------------------------------------------
 // Pools K and V ([BH, N, d], elem = 2 (bf16) or 4 (fp32)) into levels
 // 1..L-1 written at the given byte offsets of k_pyr / v_pyr.
@@ -48,7 +60,7 @@ cudaError_t launch_blockmean(const void* x, double* out, int64_t BH, int N, int 
 struct MeanKeyArgs {
   int BHq, Hq, Hkv, d, nqb, nkb, causal;
   double scale_log2;        // sm_scale * log2(e)
-  const double* qmean;      // [BHq][nqb][d]
+  const double* qmean;      // [BHq][d][nqb]
   const double* kmeanT;     // [BHkv][d][nkb]
   float* blocklse;          // [BHq][nkb][nqb]
   float* rowlse;            // [2][BHq][nqb]

@@ -394,6 +394,128 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectArgs a)
   }
 }
 
+// ----------------------------------------------------------------------------
+// select, one warp per (b, h, I), for up to 1024 key blocks: lane l holds the
+// elements l + 32k (k < KPL) in registers; the bitonic network's exchanges
+// across lanes go through shuffles and those across k are register swaps.
+// Same results as select_kernel: keys (descending float mass, ascending J),
+// fp64 exclusive prefix of the float masses in rank order.
+// ----------------------------------------------------------------------------
+constexpr int kSelWarps = 4;
+
+template <int KPL>
+__global__ void __launch_bounds__(32 * kSelWarps, 1) select_warp_kernel(const SelectArgs a) {
+  __shared__ double rlse_s[kSelWarps][128];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int row = blockIdx.x * kSelWarps + wid;                 // (b*Hq + h)*nqb + I
+  if (row >= a.B * a.Hq * a.nqb) return;
+  const int bh = row / a.nqb, I = row - bh * a.nqb;
+  const int b = bh / a.Hq, h = bh - b * a.Hq;
+  const int hkv = b * a.Hkv + h / (a.Hq / a.Hkv);
+  constexpr int P2 = 32 * KPL;
+
+  const int rbeg = I * a.rows_per_block;
+  int nvalid;
+  if (a.mode == 0) {
+    nvalid = 0;
+    for (int s = 0; s < a.rows_per_block; ++s) nvalid += (static_cast<int64_t>(rbeg + s) * a.step < a.N);
+  } else {
+    nvalid = min(a.rows_per_block, a.rows - rbeg);
+  }
+  double* rlse = rlse_s[wid];
+  for (int s = lane; s < nvalid; s += 32) {
+    const double x = a.rowlse[static_cast<int64_t>(bh) * a.rows + rbeg + s];
+    const double y = a.rowlse[(static_cast<int64_t>(a.B) * a.Hq + bh) * a.rows + rbeg + s];
+    const double mx = fmax(x, y);
+    rlse[s] = mx == -CUDART_INF ? mx : mx + log2(exp2(x - mx) + exp2(y - mx));
+  }
+  __syncwarp();
+
+  unsigned long long key[KPL];
+#pragma unroll
+  for (int k = 0; k < KPL; ++k) {
+    const int J = lane + 32 * k;
+    if (J < a.nkb) {
+      const float* bl = a.blocklse + (static_cast<int64_t>(bh) * a.nkb + J) * a.rows + rbeg;
+      double m = 0.0;
+      for (int s = 0; s < nvalid; ++s) {
+        const float x = bl[s];
+        if (x != -CUDART_INF_F) m += exp2_split(static_cast<double>(x) - rlse[s]);
+      }
+      const float mass = static_cast<float>(m / nvalid);
+      if (a.mass_out) a.mass_out[static_cast<int64_t>(row) * a.nkb + J] = mass;
+      key[k] = (static_cast<unsigned long long>(0xFFFFFFFFu - __float_as_uint(mass)) << 32) | static_cast<unsigned>(J);
+    } else {
+      key[k] = ~0ull;
+    }
+  }
+  // bitonic sort, ascending, element e = lane + 32k
+#pragma unroll
+  for (int size = 2; size <= P2; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      if (stride >= 32) {
+        const int ks = stride >> 5;
+#pragma unroll
+        for (int k = 0; k < KPL; ++k) {
+          if ((k & ks) == 0) {
+            const int e = lane + 32 * k;
+            const bool up = (e & size) == 0;
+            const unsigned long long x = key[k], y = key[k | ks];
+            if ((x > y) == up) { key[k] = y; key[k | ks] = x; }
+          }
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < KPL; ++k) {
+          const int e = lane + 32 * k;
+          const unsigned long long y = __shfl_xor_sync(0xffffffffu, key[k], stride);
+          const bool up = (e & size) == 0;
+          const bool lower = (lane & stride) == 0;
+          // the lower element of an ascending pair keeps the minimum
+          const bool keep_min = up == lower;
+          key[k] = keep_min ? (key[k] < y ? key[k] : y) : (key[k] < y ? y : key[k]);
+        }
+      }
+    }
+  }
+  // exclusive prefix in rank order (rank r = lane + 32k), then levels
+  const int n_vis = a.causal ? min(I + 1, a.nkb) : a.nkb;
+  double carry = 0.0;
+#pragma unroll
+  for (int k = 0; k < KPL; ++k) {
+    const int r = lane + 32 * k;
+    const bool real = r < a.nkb;
+    const double v = real ? static_cast<double>(__uint_as_float(0xFFFFFFFFu - static_cast<unsigned>(key[k] >> 32))) : 0.0;
+    double incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const double y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const double C = carry + incl - v;
+    carry += __shfl_sync(0xffffffffu, incl, 31);
+    if (real) {
+      const int J = static_cast<int>(key[k] & 0xFFFFFFFFu);
+      const double x = a.policy == 1 ? static_cast<double>(r) / static_cast<double>(n_vis) : C;
+      int lev = 0;
+      for (int l = 0; l < a.levels; ++l) lev += (static_cast<double>(a.thresholds[l]) <= x);
+      int out = lev >= a.levels ? PSA_SKIP : lev;
+      if (a.n_dense_prefix > 0 &&
+          (static_cast<int64_t>(I) * a.block < a.n_dense_prefix || static_cast<int64_t>(J) * a.block < a.n_dense_prefix))
+        out = 0;
+      if (a.blockcos && a.cos_min > -2.f && out != PSA_SKIP && out >= 1 &&
+          a.blockcos[static_cast<int64_t>(hkv) * a.nkb + J] < a.cos_min)
+        out = 0;
+      if (a.causal) {
+        if (J > I) out = PSA_SKIP;
+        else if (J == I) out = 0;
+      }
+      a.mask[static_cast<int64_t>(row) * a.nkb + J] = static_cast<uint8_t>(out);
+    }
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_score(const CUtensorMap* mapA, const CUtensorMap* mapB, const ScoreArgs& a, int num_sms,
@@ -424,7 +546,24 @@ cudaError_t launch_score(const CUtensorMap* mapA, const CUtensorMap* mapB, const
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t s) {
   const int rows = a.B * a.Hq * a.nqb;
-  select_kernel<<<rows, kSelThreads, 0, s>>>(a);
+  const int wgrid = (rows + kSelWarps - 1) / kSelWarps;
+  if (a.rows_per_block > 128) {
+    select_kernel<<<rows, kSelThreads, 0, s>>>(a);
+  } else if (a.nkb <= 32) {
+    select_warp_kernel<1><<<wgrid, 32 * kSelWarps, 0, s>>>(a);
+  } else if (a.nkb <= 64) {
+    select_warp_kernel<2><<<wgrid, 32 * kSelWarps, 0, s>>>(a);
+  } else if (a.nkb <= 128) {
+    select_warp_kernel<4><<<wgrid, 32 * kSelWarps, 0, s>>>(a);
+  } else if (a.nkb <= 256) {
+    select_warp_kernel<8><<<wgrid, 32 * kSelWarps, 0, s>>>(a);
+  } else if (a.nkb <= 512) {
+    select_warp_kernel<16><<<wgrid, 32 * kSelWarps, 0, s>>>(a);
+  } else if (a.nkb <= 1024) {
+    select_warp_kernel<32><<<wgrid, 32 * kSelWarps, 0, s>>>(a);
+  } else {
+    select_kernel<<<rows, kSelThreads, 0, s>>>(a);
+  }
   return cudaGetLastError();
 }
 

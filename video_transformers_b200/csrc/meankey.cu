@@ -4,13 +4,14 @@
 // query block's mean as well).  It reads Q and K once and does
 // nQB * nKB * d multiply-adds per head, so it is bound by HBM bandwidth, not
 // by the tensor cores.
-//   blockmean_kernel      one CTA per (bh, block): fp64 mean of the block's
-//                         valid tokens, one thread per channel.
-//   meankey_score_kernel  one CTA per (bh, 8 query blocks): fp64 dot
-//                         products of the query-block means against every
-//                         key-block mean, written as log2-domain scores in
-//                         the layout the select kernel reads, then the
-//                         row's log-sum-exp over the visible key blocks.
+//   blockmean_kernel       one CTA per (bh, block): fp64 mean of the block's
+//                          valid tokens, one thread per channel, written
+//                          channel-major.
+//   meankey_logits_kernel  a 64 x 64 tile of (query block, key block) pairs
+//                          per CTA: fp64 dot products of the means, written
+//                          as log2-domain scores in the layout the select
+//                          kernel reads.
+//   meankey_lse_kernel     the row log-sum-exp over the visible key blocks.
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
@@ -18,9 +19,6 @@
 
 namespace psa {
 namespace {
-
-constexpr int kRowsPerCta = 8;
-constexpr int kScoreThreads = 256;
 
 __device__ __forceinline__ double to_f64(float x) { return static_cast<double>(x); }
 __device__ __forceinline__ double to_f64(__nv_bfloat16 x) { return static_cast<double>(__bfloat162float(x)); }
@@ -44,99 +42,81 @@ __global__ void blockmean_kernel(const T* __restrict__ x, double* __restrict__ o
   }
 }
 
-__device__ __forceinline__ double warp_max(double v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-__device__ __forceinline__ double warp_sum(double v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
+// Logits of a 64 x 64 tile of (query block I, key block J) pairs of one head
+// (fp64, 256 threads, 4 x 4 pairs per thread): thread (ty, tx) owns
+// I = I0 + tx + 16u and J = J0 + ty + 16v, so stores of one J are
+// contiguous in I.  The means arrive channel-major ([bh][c][block]).
+constexpr int kTile = 64;
+constexpr int kChan = 32;
 
-__global__ void __launch_bounds__(kScoreThreads) meankey_score_kernel(const MeanKeyArgs a) {
-  extern __shared__ double qs[];                       // [kRowsPerCta][d]
-  __shared__ double red[kScoreThreads / 32][kRowsPerCta];
-  __shared__ double rmax[kRowsPerCta], rsum[kRowsPerCta];
-  const int groups = (a.nqb + kRowsPerCta - 1) / kRowsPerCta;
-  const int bh = blockIdx.x / groups;
-  const int I0 = (blockIdx.x - bh * groups) * kRowsPerCta;
+__global__ void __launch_bounds__(256) meankey_logits_kernel(const MeanKeyArgs a) {
+  __shared__ double qt[kChan][kTile];
+  __shared__ double kt[kChan][kTile];
+  const int bh = blockIdx.y;
+  const int tiles_i = (a.nqb + kTile - 1) / kTile;
+  const int I0 = (blockIdx.x % tiles_i) * kTile, J0 = (blockIdx.x / tiles_i) * kTile;
   const int b = bh / a.Hq, h = bh - b * a.Hq;
   const int hkv = b * a.Hkv + h / (a.Hq / a.Hkv);
-  const int nr = min(kRowsPerCta, a.nqb - I0);
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  for (int i = threadIdx.x; i < kRowsPerCta * a.d; i += blockDim.x) {
-    const int r = i / a.d, c = i - r * a.d;
-    qs[i] = r < nr ? a.qmean[(static_cast<int64_t>(bh) * a.nqb + I0 + r) * a.d + c] : 0.0;
-  }
-  __syncthreads();
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const double* qm = a.qmean + static_cast<int64_t>(bh) * a.d * a.nqb;
   const double* km = a.kmeanT + static_cast<int64_t>(hkv) * a.d * a.nkb;
+  double acc[4][4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) acc[u][v] = 0.0;
+  for (int c0 = 0; c0 < a.d; c0 += kChan) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < kChan * kTile; i += 256) {
+      const int c = i / kTile, x = i - c * kTile;
+      const bool cin = c0 + c < a.d;
+      qt[c][x] = cin && I0 + x < a.nqb ? qm[static_cast<int64_t>(c0 + c) * a.nqb + I0 + x] : 0.0;
+      kt[c][x] = cin && J0 + x < a.nkb ? km[static_cast<int64_t>(c0 + c) * a.nkb + J0 + x] : 0.0;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int c = 0; c < kChan; ++c) {
+      double qv[4], kv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) qv[u] = qt[c][tx + 16 * u];
+#pragma unroll
+      for (int v = 0; v < 4; ++v) kv[v] = kt[c][ty + 16 * v];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[u][v] = fma(qv[u], kv[v], acc[u][v]);
+    }
+  }
   float* bl = a.blocklse + static_cast<int64_t>(bh) * a.nkb * a.nqb;
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    const int J = J0 + ty + 16 * v;
+    if (J >= a.nkb) continue;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int I = I0 + tx + 16 * u;
+      if (I >= a.nqb) continue;
+      const bool vis = !a.causal || J <= I;
+      bl[static_cast<int64_t>(J) * a.nqb + I] = vis ? static_cast<float>(acc[u][v] * a.scale_log2) : -CUDART_INF_F;
+    }
+  }
+}
 
-  // pass 1: scores (log2 domain) of every visible key block, row maxima
-  double mx[kRowsPerCta];
-#pragma unroll
-  for (int r = 0; r < kRowsPerCta; ++r) mx[r] = -CUDART_INF;
-  for (int J = threadIdx.x; J < a.nkb; J += blockDim.x) {
-    double acc[kRowsPerCta];
-#pragma unroll
-    for (int r = 0; r < kRowsPerCta; ++r) acc[r] = 0.0;
-    for (int c = 0; c < a.d; ++c) {
-      const double kv = km[static_cast<int64_t>(c) * a.nkb + J];
-#pragma unroll
-      for (int r = 0; r < kRowsPerCta; ++r) acc[r] = fma(qs[r * a.d + c], kv, acc[r]);
-    }
-#pragma unroll
-    for (int r = 0; r < kRowsPerCta; ++r) {
-      if (r < nr) {
-        const int I = I0 + r;
-        const bool vis = !a.causal || J <= I;
-        const float z = vis ? static_cast<float>(acc[r] * a.scale_log2) : -CUDART_INF_F;
-        bl[static_cast<int64_t>(J) * a.nqb + I] = z;
-        if (vis) mx[r] = fmax(mx[r], static_cast<double>(z));
-      }
-    }
-  }
-#pragma unroll
-  for (int r = 0; r < kRowsPerCta; ++r) {
-    const double v = warp_max(mx[r]);
-    if (lane == 0) red[wid][r] = v;
-  }
-  __syncthreads();
-  if (threadIdx.x < kRowsPerCta) {
-    double v = -CUDART_INF;
-    for (int w = 0; w < kScoreThreads / 32; ++w) v = fmax(v, red[w][threadIdx.x]);
-    rmax[threadIdx.x] = v;
-  }
-  __syncthreads();
-
-  // pass 2: sum of 2^(z - max) over the scores this thread wrote
-  double sm[kRowsPerCta];
-#pragma unroll
-  for (int r = 0; r < kRowsPerCta; ++r) sm[r] = 0.0;
-  for (int J = threadIdx.x; J < a.nkb; J += blockDim.x) {
-#pragma unroll
-    for (int r = 0; r < kRowsPerCta; ++r) {
-      if (r < nr) {
-        const float z = bl[static_cast<int64_t>(J) * a.nqb + I0 + r];
-        if (z != -CUDART_INF_F) sm[r] += exp2(static_cast<double>(z) - rmax[r]);
-      }
-    }
-  }
-#pragma unroll
-  for (int r = 0; r < kRowsPerCta; ++r) {
-    const double v = warp_sum(sm[r]);
-    if (lane == 0) red[wid][r] = v;
-  }
-  __syncthreads();
-  if (threadIdx.x < nr) {
-    double v = 0.0;
-    for (int w = 0; w < kScoreThreads / 32; ++w) v += red[w][threadIdx.x];
-    const int64_t o = static_cast<int64_t>(bh) * a.nqb + I0 + threadIdx.x;
-    a.rowlse[o] = static_cast<float>(rmax[threadIdx.x] + log2(v));
-    a.rowlse[static_cast<int64_t>(a.BHq) * a.nqb + o] = -CUDART_INF_F;
-  }
+// Row log-sum-exp (log2 domain, fp64) over the visible key blocks, one
+// thread per (bh, I); a warp reads one J of 32 consecutive rows at a time.
+__global__ void __launch_bounds__(256) meankey_lse_kernel(const MeanKeyArgs a) {
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= static_cast<int64_t>(a.BHq) * a.nqb) return;
+  const int64_t bh = t / a.nqb;
+  const int I = static_cast<int>(t - bh * a.nqb);
+  const float* bl = a.blocklse + bh * a.nkb * a.nqb + I;
+  const int nj = a.causal ? min(I + 1, a.nkb) : a.nkb;
+  double mx = -CUDART_INF;
+  for (int J = 0; J < nj; ++J) mx = fmax(mx, static_cast<double>(bl[static_cast<int64_t>(J) * a.nqb]));
+  double sm = 0.0;
+  for (int J = 0; J < nj; ++J) sm += exp2(static_cast<double>(bl[static_cast<int64_t>(J) * a.nqb]) - mx);
+  a.rowlse[t] = static_cast<float>(mx + log2(sm));
+  a.rowlse[static_cast<int64_t>(a.BHq) * a.nqb + t] = -CUDART_INF_F;
 }
 
 }  // namespace
@@ -156,9 +136,10 @@ cudaError_t launch_blockmean(const void* x, double* out, int64_t BH, int N, int 
 }
 
 cudaError_t launch_meankey_score(const MeanKeyArgs& a, cudaStream_t s) {
-  const int groups = (a.nqb + kRowsPerCta - 1) / kRowsPerCta;
-  const size_t smem = static_cast<size_t>(kRowsPerCta) * a.d * sizeof(double);
-  meankey_score_kernel<<<static_cast<unsigned>(a.BHq) * groups, kScoreThreads, smem, s>>>(a);
+  const int tiles = ((a.nqb + kTile - 1) / kTile) * ((a.nkb + kTile - 1) / kTile);
+  meankey_logits_kernel<<<dim3(tiles, a.BHq), 256, 0, s>>>(a);
+  const int64_t rows = static_cast<int64_t>(a.BHq) * a.nqb;
+  meankey_lse_kernel<<<static_cast<unsigned>((rows + 255) / 256), 256, 0, s>>>(a);
   return cudaGetLastError();
 }
 
