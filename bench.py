@@ -49,6 +49,35 @@ ATTN_TRAFFIC = {"wan14b": {"bytes_per_launch": 10 * (743.809280e6 + 71.797504e6)
                            "attn_cu_sha256": "b99157c006021851afeb671c24c57be7ee988983e6b850d20d79d5b3f8cc9f72"}}
 UNIT = "TFLOP/s"
 KERNELS_PER_STEP = {"pyramid": 1, "blockcos": 0, "score": 1, "select": 1, "plan": 3, "attention": 1}
+# kernels of psa_make_mask per scorer: score + select, or block means (Q, K),
+# logits, row LSE + select; a given mask is a device copy, none of ours
+MASK_KERNELS = {"sample": 2, "antidiag": 2, "meankey": 5, "given": 0}
+MUFU_PER_CLK_SM = 16       # ex2.approx.ftz.f32 per clock per SM (measured on B200)
+
+
+def mask_roofline(w, mask_ms, hbm, clocks, elem):
+    """Roofline of the whole mask stage (scorer + select): the sampling and
+    antidiagonal scorers are bound by one exp2 per score element on the
+    special-function unit; the mean-key scorer by reading Q and K once."""
+    if w.mask_mode == "meankey":
+        byts = w.B * (w.Hq + w.Hkv) * w.N * w.d * elem
+        ach = byts / (mask_ms * 1e-3) / 1e9
+        return {"bound": "hbm", "stage": "psa_make_mask", "achieved": ach, "peak": hbm, "unit": "GB/s",
+                "frac": ach / hbm, "work": "Q and K read once, %.3f GB" % (byts / 1e9)}
+    if w.mask_mode not in ("sample", "antidiag"):
+        return None
+    if w.mask_mode == "sample":
+        rows, cols = -(-w.N // w.block) * 8, w.N
+    else:
+        rows = cols = w.N // w.stride
+    exps = rows * cols * w.B * w.Hq * (0.5 if w.causal else 1.0)
+    mhz = (clocks or {}).get("sm_mhz") or 1965.0
+    peak = MUFU_PER_CLK_SM * 148 * mhz * 1e6 / 1e9
+    ach = exps / (mask_ms * 1e-3) / 1e9
+    return {"bound": "alu", "unit_kind": "special-function unit (exp2)", "stage": "psa_make_mask",
+            "achieved": ach, "peak": peak, "unit": "Gexp2/s", "frac": ach / peak,
+            "work": "%.3g exp2 (one per score element); peak = %d/clk/SM x 148 SMs x %.0f MHz (sampled clock)"
+                    % (exps, MUFU_PER_CLK_SM, mhz)}
 
 
 def peaks():
@@ -298,6 +327,7 @@ def run_psa(args, rank, world, local_rank):
     e2e = run_e2e(path, w, flops, args, stream) if not args.no_e2e else None
 
     bf16_burst, bf16_sus, hbm, src = peaks()
+    clocks = clk.summary()
     attn_tflops = flops / (attn_ms * 1e-3) / 1e12
     pyr_bytes = 2 * w.B * w.Hkv * w.N * w.d * q.element_size() * (1 + sum(2.0 ** -l for l in range(1, w.levels)))
     hist = torch.bincount(path.mask.flatten().long(), minlength=256).cpu()
@@ -326,9 +356,13 @@ def run_psa(args, rank, world, local_rank):
         "pyramid_roofline": {"bound": "hbm", "achieved": pyr_bytes / (pyr_ms * 1e-3) / 1e9, "peak": hbm,
                              "unit": "GB/s", "frac": pyr_bytes / (pyr_ms * 1e-3) / 1e9 / hbm},
         "e2e": e2e,
-        "gpu_launches": sum(KERNELS_PER_STEP.values()) * args.steps + (1 if w.cos_min > -2 else 0) * args.steps,
-        "clocks": clk.summary(),
+        "gpu_launches": (sum(KERNELS_PER_STEP.values()) - KERNELS_PER_STEP["score"] - KERNELS_PER_STEP["select"]
+                         + MASK_KERNELS.get(w.mask_mode, 2) + (1 if w.cos_min > -2 else 0)) * args.steps,
+        "clocks": clocks,
     }
+    mr = mask_roofline(w, mask_ms, hbm, clocks, q.element_size())
+    if mr is not None:
+        line["mask_roofline"] = mr
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(w, q, k, v, path, args)
     return line

@@ -117,3 +117,18 @@ def test_attention_on_variant_masks(mode, policy, levels):
     o, l = O.attention(q, kl, vl, mask.cpu(), w.block, w.sm_scale, w.causal)
     mx, mean, _ = attn_errors(out, o)
     assert mx <= 2e-2 and mean <= 2e-3, (mx, mean)
+
+
+def test_meankey_quantile_text_prefix_causal_fp32():
+    """Every forced rule on top of the new scorer and policy: a text prefix
+    (its blocks stay level 0), causal masking (J > I skipped, J == I level
+    0), fp32 inputs, GQA 2:1 and a ragged last block."""
+    w = W.reduced("cogvideox5b", grid=(3, 10, 15), heads=(4, 2), n_text=30).replace(
+        mask_mode="meankey", causal=True, dtype="fp32", thresholds=(0.25, 0.5, 0.75, 0.875), cos_min=-3.0)
+    q, k, v, _ = W.make_qkv(w, device="cpu")
+    mask = check_variant(w, q.to(DEV), k.to(DEV), P.PSA_POLICY_QUANTILE)
+    nb = mask.shape[-1]
+    iu = np.triu_indices(nb, 1)
+    assert np.all(mask[..., iu[0], iu[1]] == SKIP)
+    assert np.all(mask[..., np.arange(nb), np.arange(nb)] == 0)
+    assert np.all(mask[..., 0, 0] == 0) and np.all(mask[..., :, 0] == 0)     # block 0 holds text

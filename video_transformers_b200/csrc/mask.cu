@@ -18,6 +18,7 @@
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
+#include "exp2_poly.h"
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -54,6 +55,35 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
+// Of every 8 column pairs of a block, this many take their exponential on
+// the FMA pipe (exp2_fma2_d5) instead of the special-function unit.
+#ifndef PSA_SCORE_POLY
+#define PSA_SCORE_POLY 0
+#endif
+constexpr int kScorePoly = PSA_SCORE_POLY;
+
+// 2^x for two lanes at once on the FMA pipe, x <= 20, relative error about
+// 2.4e-7: Cody-Waite split x = n + f with n = round(x) (adding 1.5 * 2^23
+// rounds to an integer in the low mantissa bits) and f in [-1/2, 1/2]; 2^f
+// from the degree-5 Remez polynomial of exp2_poly.h; 2^n added to the
+// exponent field as an integer.  Inputs below -126 are clamped there (the
+// result is then about 2^-126 instead of 0, far below one part in 10^30 of
+// a block sum, whose largest term is 1).
+__device__ __forceinline__ float2 exp2_fma2_d5(float2 x) {
+  x.x = fmaxf(x.x, -126.0f);
+  x.y = fmaxf(x.y, -126.0f);
+  const float2 t = __fadd2_rn(x, make_float2(12582912.0f, 12582912.0f));
+  const float2 n = __fadd2_rn(t, make_float2(-12582912.0f, -12582912.0f));
+  const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), x);
+  float2 p = __ffma2_rn(make_float2(kExp2Poly5_5, kExp2Poly5_5), f, make_float2(kExp2Poly5_4, kExp2Poly5_4));
+  p = __ffma2_rn(p, f, make_float2(kExp2Poly5_3, kExp2Poly5_3));
+  p = __ffma2_rn(p, f, make_float2(kExp2Poly5_2, kExp2Poly5_2));
+  p = __ffma2_rn(p, f, make_float2(kExp2Poly5_1, kExp2Poly5_1));
+  p = __ffma2_rn(p, f, make_float2(kExp2Poly5_0, kExp2Poly5_0));
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
 // log2-domain log-sum-exp of CPB consecutive scores s[0..CPB) (already
 // masked to -inf where invalid when MASKED), scaled by sc.
 template <int CPB, bool MASKED>
@@ -79,7 +109,8 @@ __device__ __forceinline__ float block_lse(const float* s, float sc) {
 #pragma unroll
   for (int j = 0; j < CPB; j += 2) {
     const float2 z = __ffma2_rn(make_float2(s[j], s[j + 1]), sc2, off);
-    acc[(j >> 1) & 1] = __fadd2_rn(acc[(j >> 1) & 1], make_float2(fast_exp2(z.x), fast_exp2(z.y)));
+    const float2 e = ((j >> 1) & 7) < kScorePoly ? exp2_fma2_d5(z) : make_float2(fast_exp2(z.x), fast_exp2(z.y));
+    acc[(j >> 1) & 1] = __fadd2_rn(acc[(j >> 1) & 1], e);
   }
   const float2 t = __fadd2_rn(acc[0], acc[1]);
   return mb + __log2f(t.x + t.y);
