@@ -435,7 +435,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectArgs a)
 constexpr int kSelWarps = 4;
 
 template <int KPL>
-__global__ void __launch_bounds__(32 * kSelWarps, 1) select_warp_kernel(const SelectArgs a) {
+__global__ void __launch_bounds__(32 * kSelWarps, 4) select_warp_kernel(const SelectArgs a) {
   __shared__ double rlse_s[kSelWarps][128];
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int row = blockIdx.x * kSelWarps + wid;                 // (b*Hq + h)*nqb + I
