@@ -68,3 +68,46 @@ def test_fullsize_sampled_parity(name):
         assert mx <= 2e-2 and mean <= 2e-3, (name, h, I, mx, mean)
     assert P.psa_get_device_status(ws) == P.PSA_OK
     print("%s: %d ambiguous of %d sampled pairs" % (name, n_amb, n_pairs))
+
+
+@pytest.mark.parametrize("mode,policy", [("meankey", "mass"), ("sample", "quantile")])
+def test_fullsize_mask_variants_sampled(mode, policy):
+    """The mask variants at the Wan2.1-14B shape, as `bench.py --mask-mode
+    meankey` and `--policy quantile` run them: sampled query-block rows of
+    the mask (bit-exact outside the ambiguity band) and their masses, then
+    the attention rows of those blocks on the GPU mask."""
+    w = W.PRESETS["wan14b"].replace(mask_mode=mode, policy=policy)
+    q, k, v, _ = W.make_qkv(w, device=DEV)
+    shape = shape_for(w)
+    pol = P.PSA_POLICY_QUANTILE if policy == "quantile" else P.PSA_POLICY_MASS
+    kp, vp, _ = run_pyramid(shape, k, v)
+    mask, mass = run_mask(shape, params_for(w, pol), q, k)
+    out, lse, ws = run_attention(shape, q, k, v, kp, vp, mask, w.sm_scale)
+    torch.cuda.synchronize()
+    th = [float(np.float32(t)) for t in w.thresholds]
+    for b, h, I in sample_rows(w, 4, seed=7 + len(mode)):
+        qh, kh, vh = q[b:b + 1, h:h + 1].cpu(), k[b:b + 1, h:h + 1].cpu(), v[b:b + 1, h:h + 1].cpu()
+        row = [(0, 0, I)]
+        if mode == "meankey":
+            om = O.meankey_mass(qh, kh, w.block, w.sm_scale, w.causal, rows=row)
+        else:
+            om = O.sampling_mass(qh, kh, w.block, w.sm_scale, w.causal, rows=row)
+        omask = O.make_mask(om, th, w.levels, w.block, w.causal, w.n_dense_prefix, None, -3.0, 1, rows=row,
+                            policy=policy)[0, 0, I]
+        if policy == "quantile":
+            amb = O.ambiguous_pairs_quantile(om, th, w.levels, w.causal, 1e-6, rows=row)[0, 0, I]
+        else:
+            amb = O.ambiguous_pairs(om, th, 1e-6, row)[0, 0, I]
+        gm = mask[b, h, I].cpu().numpy()
+        gmass = mass[b, h, I].cpu().numpy().astype(np.float64)
+        big = om[0, 0, I] > 1e-6
+        assert (np.abs(gmass[big] - om[0, 0, I][big]) / om[0, 0, I][big]).max() <= 1e-4
+        assert np.all((gm == omask) | amb), (mode, policy, h, I, int(((gm != omask) & ~amb).sum()))
+        kl = [kh.double().numpy()] + [P.pyramid_level(shape, kp, l)[b:b + 1, h:h + 1].double().cpu().numpy()
+                                      for l in range(1, w.levels)]
+        vl = [vh.double().numpy()] + [P.pyramid_level(shape, vp, l)[b:b + 1, h:h + 1].double().cpu().numpy()
+                                      for l in range(1, w.levels)]
+        o, l = O.attention(qh, kl, vl, mask[b:b + 1, h:h + 1].cpu(), w.block, w.sm_scale, w.causal, rows=row)
+        mx, mean, _ = attn_errors(out[b:b + 1, h:h + 1], o)
+        assert mx <= 2e-2 and mean <= 2e-3, (mode, policy, h, I, mx, mean)
+    assert P.psa_get_device_status(ws) == P.PSA_OK

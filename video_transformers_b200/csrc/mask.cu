@@ -62,6 +62,7 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 #endif
 constexpr int kScorePoly = PSA_SCORE_POLY;
 
+
 // 2^x for two lanes at once on the FMA pipe, x <= 20, relative error about
 // 2.4e-7: Cody-Waite split x = n + f with n = round(x) (adding 1.5 * 2^23
 // rounds to an integer in the low mantissa bits) and f in [-1/2, 1/2]; 2^f
@@ -313,6 +314,223 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ----------------------------------------------------------------------------
+// score2_kernel: the sampling score with two row tiles per work item, so
+// every K tile brought into shared memory serves 256 sampled rows instead of
+// 128 (half the K traffic per flop).  The two sampled-query tiles stay
+// resident; TMEM holds two S buffers per row tile (512 columns); epilogue
+// warpgroup x owns row tile x for every column tile and writes both row-LSE
+// partials (even and odd column tiles).  Used for d = 128, where it halves
+// the K traffic that bounds the one-row-tile kernel; at d = 64 (half the
+// MMA work per tile) it measured slower.
+// ----------------------------------------------------------------------------
+constexpr int kRegion2 = 12;        // 192 KB: 2 * (d/64) resident A chunks + the K ring
+constexpr int kMaxStages2 = 10;
+
+struct Score2Shared {
+  uint64_t a_full, a_empty;
+  uint64_t full[kMaxStages2], empty[kMaxStages2];
+  uint64_t s_full[2], s_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <int CPB>
+__global__ void __launch_bounds__(kThreads, 1)
+    score2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+                  const ScoreArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Score2Shared* sh = reinterpret_cast<Score2Shared*>(tiles + kRegion2 * kChunk);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row_tiles = (a.rows + 127) / 128;
+  const int pairs = (row_tiles + 1) / 2;
+  const int col_tiles = (a.cols + 127) / 128;
+  const int n_items = a.BHq * pairs;
+  const int nk = a.d / 64;                 // 64-channel chunks per tile
+  const int nst = kRegion2 - 2 * nk;       // K ring stages (8 for d = 128, 10 for d = 64)
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&sh->a_full), 1);
+    mbar_init(smem_u32(&sh->a_empty), 1);
+    for (int i = 0; i < kMaxStages2; ++i) { mbar_init(smem_u32(&sh->full[i]), 1); mbar_init(smem_u32(&sh->empty[i]), 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(smem_u32(&sh->s_full[i]), 1); mbar_init(smem_u32(&sh->s_empty[i]), 256); }
+    mbar_init(smem_u32(&sh->drain), 1);
+    sh->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) { tmem_alloc(smem_u32(&sh->tmem_base), 512); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh->tmem_base;
+  volatile int* abort = &sh->abort;
+
+  // row tiles of a pair that exist, and the column tiles the pair visits
+  // (causal: up to the last row of its last tile)
+  auto n_rt = [&](int p) { return 2 * p + 1 < row_tiles ? 2 : 1; };
+  auto tiles_for = [&](int p) {
+    if (!a.causal) return col_tiles;
+    const int rlast = min((2 * p + n_rt(p)) * 128 - 1, a.rows - 1);
+    return min(col_tiles, rlast * a.step / 128 + 1);
+  };
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      tma_prefetch_desc(&mapA);
+      tma_prefetch_desc(&mapB);
+      uint32_t it = 0, icnt = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++icnt) {
+        const int bh = item / pairs, p = item - bh * pairs;
+        const int hkv = kv_head_of(bh, a.Hq, a.Hkv);
+        const int nrt = n_rt(p), nct = tiles_for(p);
+        if (!bounded_wait(smem_u32(&sh->a_empty), (icnt & 1) ^ 1, abort, a.status, 45, item, 0, 0, icnt)) { ok = false; break; }
+        mbar_arrive_expect_tx(smem_u32(&sh->a_full), nrt * nk * kChunk);
+        for (int x = 0; x < nrt; ++x)
+          for (int kc = 0; kc < nk; ++kc)
+            tma_load_4d(smem_u32(tiles + (x * nk + kc) * kChunk), &mapA, smem_u32(&sh->a_full), kc * 64, 0,
+                        (2 * p + x) * 128, bh);
+        for (int ct = 0; ct < nct && ok; ++ct) {
+          for (int kc = 0; kc < nk; ++kc, ++it) {
+            const int st = it % nst;
+            if (!bounded_wait(smem_u32(&sh->empty[st]), ((it / nst) & 1) ^ 1, abort, a.status, 41, item, ct, kc, it)) { ok = false; break; }
+            const uint32_t bar = smem_u32(&sh->full[st]);
+            mbar_arrive_expect_tx(bar, kChunk);
+            tma_load_4d(smem_u32(tiles + (2 * nk + st) * kChunk), &mapB, bar, kc * 64, 0, ct * 128, hkv);
+          }
+        }
+      }
+      for (uint32_t st = 0; st < static_cast<uint32_t>(nst); ++st)
+        if (it > st) drain_wait(smem_u32(&sh->full[st]), ((it - 1 - st) / nst) & 1, a.status);
+      if (icnt > 0) drain_wait(smem_u32(&sh->a_full), (icnt - 1) & 1, a.status);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false);
+      const uint64_t d0 = sdesc_sw128(smem_u32(tiles), 16, 1024);
+      uint32_t it = 0, t = 0, icnt = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++icnt) {
+        const int bh = item / pairs, p = item - bh * pairs;
+        (void)bh;
+        const int nrt = n_rt(p), nct = tiles_for(p);
+        if (!bounded_wait(smem_u32(&sh->a_full), icnt & 1, abort, a.status, 46, item, 0, 0, icnt)) { ok = false; break; }
+        tc_fence_after();
+        for (int ct = 0; ct < nct && ok; ++ct, ++t) {
+          const int b = t & 1;
+          if (!bounded_wait(smem_u32(&sh->s_empty[b]), ((t >> 1) & 1) ^ 1, abort, a.status, 42, item, ct, t, it)) { ok = false; break; }
+          tc_fence_after();
+          for (int kc = 0; kc < nk; ++kc, ++it) {
+            const int st = it % nst;
+            if (!bounded_wait(smem_u32(&sh->full[st]), (it / nst) & 1, abort, a.status, 43, item, ct, kc, it)) { ok = false; break; }
+            tc_fence_after();
+            for (int x = 0; x < nrt; ++x) {
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                umma_ss(tmem + x * 256 + b * 128, d0 + (((x * nk + kc) * kChunk + 32 * k) >> 4),
+                        d0 + (((2 * nk + st) * kChunk + 32 * k) >> 4), idesc, (kc | k) != 0);
+            }
+            umma_commit(smem_u32(&sh->empty[st]));
+          }
+          if (!ok) break;
+          umma_commit(smem_u32(&sh->s_full[b]));
+          if (ct + 1 == nct) umma_commit(smem_u32(&sh->a_empty));
+        }
+      }
+      umma_commit(smem_u32(&sh->drain));
+      drain_wait(smem_u32(&sh->drain), 0, a.status);
+    }
+  } else {
+    // ---------------- epilogue: warpgroup x owns row tile x ----------------
+    const int x = (warp - 2) >> 2;
+    const int q = warp & 3;                 // TMEM lane quarter of this warp
+    const int lrow = q * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    constexpr int BPT = 128 / CPB;          // KV blocks per column tile
+    uint32_t t = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+      const int bh = item / pairs, p = item - bh * pairs;
+      const bool mine = x < n_rt(p);
+      const int nct = tiles_for(p);
+      const int r = (2 * p + x) * 128 + lrow;
+      const int pos = r * a.step;
+      const int climit = a.causal ? min(a.cols, pos + 1) : a.cols;
+      // two running LSEs, even and odd column tiles (the select kernel
+      // combines them in fp64, as for the one-row-tile kernel)
+      float M[2] = {-CUDART_INF_F, -CUDART_INF_F}, Ssum[2] = {0.f, 0.f};
+      float* bl = a.blocklse + static_cast<int64_t>(bh) * a.nkb * a.rows + r;
+      for (int ct = 0; ct < nct; ++ct, ++t) {
+        const int b = t & 1;
+        if (!warp_wait(smem_u32(&sh->s_full[b]), (t >> 1) & 1, abort, a.status, 44, item, ct, t, x)) { ok = false; break; }
+        tc_fence_after();
+        if (!mine) {
+          tc_fence_before();
+          mbar_arrive(smem_u32(&sh->s_empty[b]));
+          continue;
+        }
+        uint32_t raw[128];
+        tmem_ld128(tmem + x * 256 + b * 128 + lane_off, raw);
+        tc_fence_before();
+        mbar_arrive(smem_u32(&sh->s_empty[b]));
+        float* z = reinterpret_cast<float*>(raw);
+        const int c0 = ct * 128;
+        float blse[BPT];
+        if (c0 + 128 <= climit) {
+#pragma unroll
+          for (int bb = 0; bb < BPT; ++bb) blse[bb] = block_lse<CPB, false>(z + bb * CPB, a.scale_log2);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 128; ++c) z[c] = c0 + c < climit ? z[c] : -CUDART_INF_F;
+#pragma unroll
+          for (int bb = 0; bb < BPT; ++bb) blse[bb] = block_lse<CPB, true>(z + bb * CPB, a.scale_log2);
+        }
+        float mt = blse[0];
+#pragma unroll
+        for (int bb = 1; bb < BPT; ++bb) mt = fmaxf(mt, blse[bb]);
+        if (mt != -CUDART_INF_F) {
+          const int e = ct & 1;
+          const float Mn = fmaxf(M[e], mt);
+          float add = 0.f;
+#pragma unroll
+          for (int bb = 0; bb < BPT; ++bb) add += fast_exp2(blse[bb] - Mn);
+          Ssum[e] = Ssum[e] * fast_exp2(M[e] - Mn) + add;
+          M[e] = Mn;
+        }
+        if (r < a.rows) {
+#pragma unroll
+          for (int bb = 0; bb < BPT; ++bb) {
+            const int J = ct * BPT + bb;
+            if (J < a.nkb) bl[static_cast<int64_t>(J) * a.rows] = blse[bb];
+          }
+        }
+      }
+      if (!ok) break;
+      if (mine && r < a.rows) {
+        // column tiles never visited (causal) hold no probability
+        for (int J = nct * BPT; J < a.nkb; ++J) bl[static_cast<int64_t>(J) * a.rows] = -CUDART_INF_F;
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+          a.rowlse[(static_cast<int64_t>(e) * a.BHq + bh) * a.rows + r] =
+              M[e] == -CUDART_INF_F ? -CUDART_INF_F : M[e] + __log2f(Ssum[e]);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ----------------------------------------------------------------------------
 // select: one CTA of 512 threads per (b, h, I)
 // ----------------------------------------------------------------------------
 constexpr int kSelThreads = 512;
@@ -552,6 +770,26 @@ __global__ void __launch_bounds__(32 * kSelWarps, 4) select_warp_kernel(const Se
 cudaError_t launch_score(const CUtensorMap* mapA, const CUtensorMap* mapB, const ScoreArgs& a, int num_sms,
                          cudaStream_t s) {
   const int row_tiles = (a.rows + 127) / 128;
+  if (a.mode == 0 && a.d == 128) {
+    // sampling: two row tiles per item share each K tile
+    const int n2 = a.BHq * ((row_tiles + 1) / 2);
+    const int grid2 = n2 < num_sms ? n2 : num_sms;
+    const size_t smem2 = 1024 + kRegion2 * kChunk + sizeof(Score2Shared);
+    switch (a.cols_per_block) {
+#define PSA_SCORE2_CASE(CPB)                                                                       \
+  case CPB: {                                                                                      \
+    cudaError_t e = cudaFuncSetAttribute(score2_kernel<CPB>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                                         static_cast<int>(smem2));                                 \
+    if (e != cudaSuccess) return e;                                                                \
+    score2_kernel<CPB><<<grid2, kThreads, smem2, s>>>(*mapA, *mapB, a);                            \
+    return cudaGetLastError();                                                                     \
+  }
+      PSA_SCORE2_CASE(64)
+      PSA_SCORE2_CASE(128)
+#undef PSA_SCORE2_CASE
+      default: break;
+    }
+  }
   const int n_items = a.BHq * row_tiles;
   const int grid = n_items < num_sms ? n_items : num_sms;
   const size_t smem = 1024 + kRegionChunks * kChunk + sizeof(ScoreShared);
