@@ -316,12 +316,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ----------------------------------------------------------------------------
 // score2_kernel: the sampling score with two row tiles per work item, so
 // every K tile brought into shared memory serves 256 sampled rows instead of
-// 128 (half the K traffic per flop).  The two sampled-query tiles stay
-// resident; TMEM holds two S buffers per row tile (512 columns); epilogue
-// warpgroup x owns row tile x for every column tile and writes both row-LSE
-// partials (even and odd column tiles).  Used for d = 128, where it halves
-// the K traffic that bounds the one-row-tile kernel; at d = 64 (half the
-// MMA work per tile) it measured slower.
+// 128 (half the K traffic per flop).  A work item is (head, row-tile pair,
+// half of the column tiles); the two sampled-query tiles stay resident;
+// TMEM holds two S buffers per row tile (512 columns); epilogue warpgroup x
+// owns row tile x and writes row-LSE partial e for column half e.  Used for
+// d = 128, where it halves the K traffic that bounds the one-row-tile
+// kernel; at d = 64 (half the MMA work per tile) it measured slower.
 // ----------------------------------------------------------------------------
 constexpr int kRegion2 = 12;        // 192 KB: 2 * (d/64) resident A chunks + the K ring
 constexpr int kMaxStages2 = 10;
@@ -347,7 +347,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int row_tiles = (a.rows + 127) / 128;
   const int pairs = (row_tiles + 1) / 2;
   const int col_tiles = (a.cols + 127) / 128;
-  const int n_items = a.BHq * pairs;
+  // item = (bh, row-tile pair, column half): the two halves of a pair's
+  // column sweep are separate items (finer work for the persistent grid);
+  // half e writes row-LSE partial e
+  const int n_items = a.BHq * pairs * 2;
   const int nk = a.d / 64;                 // 64-channel chunks per tile
   const int nst = kRegion2 - 2 * nk;       // K ring stages (8 for d = 128, 10 for d = 64)
 
@@ -375,6 +378,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int rlast = min((2 * p + n_rt(p)) * 128 - 1, a.rows - 1);
     return min(col_tiles, rlast * a.step / 128 + 1);
   };
+  // column tiles [lo, hi) of item half e
+  auto range_of = [&](int p, int e, int& lo, int& hi) {
+    const int nct = tiles_for(p), h = (nct + 1) / 2;
+    lo = e == 0 ? 0 : h;
+    hi = e == 0 ? h : nct;
+  };
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -383,17 +392,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&mapB);
       uint32_t it = 0, icnt = 0;
       bool ok = true;
-      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++icnt) {
-        const int bh = item / pairs, p = item - bh * pairs;
+      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+        const int e = item & 1, bh = (item >> 1) / pairs, p = (item >> 1) - bh * pairs;
         const int hkv = kv_head_of(bh, a.Hq, a.Hkv);
-        const int nrt = n_rt(p), nct = tiles_for(p);
+        const int nrt = n_rt(p);
+        int lo, hi;
+        range_of(p, e, lo, hi);
+        if (hi == lo) continue;
         if (!bounded_wait(smem_u32(&sh->a_empty), (icnt & 1) ^ 1, abort, a.status, 45, item, 0, 0, icnt)) { ok = false; break; }
+        ++icnt;
         mbar_arrive_expect_tx(smem_u32(&sh->a_full), nrt * nk * kChunk);
         for (int x = 0; x < nrt; ++x)
           for (int kc = 0; kc < nk; ++kc)
             tma_load_4d(smem_u32(tiles + (x * nk + kc) * kChunk), &mapA, smem_u32(&sh->a_full), kc * 64, 0,
                         (2 * p + x) * 128, bh);
-        for (int ct = 0; ct < nct && ok; ++ct) {
+        for (int ct = lo; ct < hi && ok; ++ct) {
           for (int kc = 0; kc < nk; ++kc, ++it) {
             const int st = it % nst;
             if (!bounded_wait(smem_u32(&sh->empty[st]), ((it / nst) & 1) ^ 1, abort, a.status, 41, item, ct, kc, it)) { ok = false; break; }
@@ -414,13 +427,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t d0 = sdesc_sw128(smem_u32(tiles), 16, 1024);
       uint32_t it = 0, t = 0, icnt = 0;
       bool ok = true;
-      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++icnt) {
-        const int bh = item / pairs, p = item - bh * pairs;
+      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+        const int e = item & 1, bh = (item >> 1) / pairs, p = (item >> 1) - bh * pairs;
         (void)bh;
-        const int nrt = n_rt(p), nct = tiles_for(p);
+        const int nrt = n_rt(p);
+        int lo, hi;
+        range_of(p, e, lo, hi);
+        if (hi == lo) continue;
         if (!bounded_wait(smem_u32(&sh->a_full), icnt & 1, abort, a.status, 46, item, 0, 0, icnt)) { ok = false; break; }
+        ++icnt;
         tc_fence_after();
-        for (int ct = 0; ct < nct && ok; ++ct, ++t) {
+        for (int ct = lo; ct < hi && ok; ++ct, ++t) {
           const int b = t & 1;
           if (!bounded_wait(smem_u32(&sh->s_empty[b]), ((t >> 1) & 1) ^ 1, abort, a.status, 42, item, ct, t, it)) { ok = false; break; }
           tc_fence_after();
@@ -438,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (!ok) break;
           umma_commit(smem_u32(&sh->s_full[b]));
-          if (ct + 1 == nct) umma_commit(smem_u32(&sh->a_empty));
+          if (ct + 1 == hi) umma_commit(smem_u32(&sh->a_empty));
         }
       }
       umma_commit(smem_u32(&sh->drain));
@@ -454,17 +471,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t t = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-      const int bh = item / pairs, p = item - bh * pairs;
+      const int e = item & 1, bh = (item >> 1) / pairs, p = (item >> 1) - bh * pairs;
       const bool mine = x < n_rt(p);
       const int nct = tiles_for(p);
+      int lo, hi;
+      range_of(p, e, lo, hi);
       const int r = (2 * p + x) * 128 + lrow;
       const int pos = r * a.step;
       const int climit = a.causal ? min(a.cols, pos + 1) : a.cols;
-      // two running LSEs, even and odd column tiles (the select kernel
-      // combines them in fp64, as for the one-row-tile kernel)
-      float M[2] = {-CUDART_INF_F, -CUDART_INF_F}, Ssum[2] = {0.f, 0.f};
+      // this half's running LSE: row-LSE partial e (the select kernel
+      // combines the two in fp64)
+      float M = -CUDART_INF_F, Ssum = 0.f;
       float* bl = a.blocklse + static_cast<int64_t>(bh) * a.nkb * a.rows + r;
-      for (int ct = 0; ct < nct; ++ct, ++t) {
+      for (int ct = lo; ct < hi; ++ct, ++t) {
         const int b = t & 1;
         if (!warp_wait(smem_u32(&sh->s_full[b]), (t >> 1) & 1, abort, a.status, 44, item, ct, t, x)) { ok = false; break; }
         tc_fence_after();
@@ -493,13 +512,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int bb = 1; bb < BPT; ++bb) mt = fmaxf(mt, blse[bb]);
         if (mt != -CUDART_INF_F) {
-          const int e = ct & 1;
-          const float Mn = fmaxf(M[e], mt);
+          const float Mn = fmaxf(M, mt);
           float add = 0.f;
 #pragma unroll
           for (int bb = 0; bb < BPT; ++bb) add += fast_exp2(blse[bb] - Mn);
-          Ssum[e] = Ssum[e] * fast_exp2(M[e] - Mn) + add;
-          M[e] = Mn;
+          Ssum = Ssum * fast_exp2(M - Mn) + add;
+          M = Mn;
         }
         if (r < a.rows) {
 #pragma unroll
@@ -512,11 +530,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       if (mine && r < a.rows) {
         // column tiles never visited (causal) hold no probability
-        for (int J = nct * BPT; J < a.nkb; ++J) bl[static_cast<int64_t>(J) * a.rows] = -CUDART_INF_F;
-#pragma unroll
-        for (int e = 0; e < 2; ++e)
-          a.rowlse[(static_cast<int64_t>(e) * a.BHq + bh) * a.rows + r] =
-              M[e] == -CUDART_INF_F ? -CUDART_INF_F : M[e] + __log2f(Ssum[e]);
+        if (e == 1)
+          for (int J = nct * BPT; J < a.nkb; ++J) bl[static_cast<int64_t>(J) * a.rows] = -CUDART_INF_F;
+        a.rowlse[(static_cast<int64_t>(e) * a.BHq + bh) * a.rows + r] =
+            M == -CUDART_INF_F ? -CUDART_INF_F : M + __log2f(Ssum);
       }
     }
   }
@@ -772,7 +789,7 @@ cudaError_t launch_score(const CUtensorMap* mapA, const CUtensorMap* mapB, const
   const int row_tiles = (a.rows + 127) / 128;
   if (a.mode == 0 && a.d == 128) {
     // sampling: two row tiles per item share each K tile
-    const int n2 = a.BHq * ((row_tiles + 1) / 2);
+    const int n2 = a.BHq * ((row_tiles + 1) / 2) * 2;
     const int grid2 = n2 < num_sms ? n2 : num_sms;
     const size_t smem2 = 1024 + kRegion2 * kChunk + sizeof(Score2Shared);
     switch (a.cols_per_block) {
