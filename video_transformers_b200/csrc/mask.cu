@@ -10,7 +10,13 @@
 //                by a per-(row, KV block) log-sum-exp in two epilogue
 //                warpgroups that take alternate column tiles.  Only the block
 //                LSEs and each row's LSE (one partial per warpgroup) leave
-//                the SM.
+//                the SM.  Used for the antidiagonal score and for sampling at
+//                d = 64.
+// score2_kernel  the sampling score at d = 128: two row tiles share every K
+//                tile, epilogue warpgroup x owns row tile x, and a work item
+//                covers half of the column tiles (row-LSE partial = half).
+// select_warp_kernel  one warp per (b, h, query block), up to 1024 key
+//                blocks: the same levels as select_kernel, keys in registers.
 // select_kernel  one CTA per (b, h, query block): block masses from the
 //                LSEs, a bitonic sort (mass descending, index ascending), an
 //                fp64 exclusive scan, levels by that prefix (or by rank for
