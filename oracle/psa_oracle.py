@@ -58,6 +58,9 @@ reason in the design notes):
       query against the mean of the block's keys): the query side is the
       mean of the query block's valid queries as well; mass[I, J] =
       softmax over visible J of sm_scale * mean_q(I) . mean_k(J).
+  R12 backward pass: the mask (the levels) is a fixed selection and is not
+      differentiated; gradients flow through the pooling of each level as a
+      mean (1/2^l to each averaged token).
 
 Pins: every function here is checked by ``tests/test_oracle_pins.py``
 against closed forms, invariants, brute force or an independent library
@@ -495,6 +498,83 @@ def attention(q, kp, vp, mask, block: int, sm_scale: float, causal: bool,
         o[b, h, i0:i1] = np.where(empty[:, None], 0.0, (e @ vals) / np.where(empty, 1.0, s)[:, None])
         lse[b, h, i0:i1] = np.where(empty, -np.inf, m[:, 0] + np.log(np.where(empty, 1.0, s)))
     return o, lse
+
+
+def attention_backward(q, k, v, mask, block: int, sm_scale: float, causal: bool, levels: int, dout):
+    """Gradients of adaptive pyramid attention with respect to Q, K and V
+    (not on the pages' hot path: the news review claims end-to-end
+    training, the summary article pairs PSA with distillation).  The mask
+    is a fixed selection.  For query i of block I, with P = softmax(z) over
+    the key set of I (as in :func:`attention`) and upstream gradient dO_i:
+
+        dV^l[p] += P_ip dO_i,      dP_ip = dO_i . V^l[p],
+        D_i = sum_p P_ip dP_ip,    dZ_ip = P_ip (dP_ip - D_i),
+        dQ_i = sm_scale sum_p dZ_ip K^l[p],
+        dK^l[p] += sm_scale dZ_ip q_i,
+
+    then through the pooling of level l (a mean of 2^l consecutive tokens):
+    dK[t] += dK^l[t >> l] / 2^l, and the same for V.  Rows with no visible
+    key contribute nothing.  q: [B, Hq, N, d]; k, v: [B, Hkv, N, d];
+    dout: [B, Hq, N, d].  Returns (dq, dk, dv) in float64."""
+    q = _f64(q)
+    k = _f64(k)
+    v = _f64(v)
+    dout = _f64(dout)
+    kp, vp = build_pyramid(k, v, levels)
+    mask = np.asarray(mask.cpu() if hasattr(mask, "cpu") else mask).astype(np.int64)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    grp = Hq // Hkv
+    nb = -(-N // block)
+    dq = np.zeros_like(q)
+    dkp = [np.zeros_like(x) for x in kp]
+    dvp = [np.zeros_like(x) for x in vp]
+    for b in range(B):
+        for h in range(Hq):
+            hk = h // grp
+            for I in range(nb):
+                i0, i1 = I * block, min((I + 1) * block, N)
+                # the key set of I, remembering where each key came from
+                src = []
+                for J, l in enumerate(mask[b, h, I]):
+                    l = int(l)
+                    if l == SKIP:
+                        continue
+                    g = 1 << l
+                    for pp in range((J * block) // g, min((J + 1) * block, N) // g):
+                        src.append((l, pp))
+                if not src:
+                    continue
+                keys = np.stack([kp[l][b, hk, pp] for l, pp in src])
+                vals = np.stack([vp[l][b, hk, pp] for l, pp in src])
+                bias = np.array([level_bias(l) for l, _ in src])
+                last = np.array([(pp + 1) * (1 << l) - 1 for l, pp in src])
+                z = sm_scale * (q[b, h, i0:i1] @ keys.T) + bias[None, :]
+                if causal:
+                    z = np.where(last[None, :] <= np.arange(i0, i1)[:, None], z, -np.inf)
+                P = _softmax_rows(z)                                        # [rows, n]
+                dO = dout[b, h, i0:i1]
+                dP = dO @ vals.T
+                D = (P * dP).sum(axis=1, keepdims=True)
+                dZ = P * (dP - D)
+                dq[b, h, i0:i1] += sm_scale * (dZ @ keys)
+                gk = sm_scale * (dZ.T @ q[b, h, i0:i1])                     # [n, d]
+                gv = P.T @ dO
+                for n_, (l, pp) in enumerate(src):
+                    dkp[l][b, hk, pp] += gk[n_]
+                    dvp[l][b, hk, pp] += gv[n_]
+    return dq, pool_backward(dkp, N), pool_backward(dvp, N)
+
+
+def pool_backward(grads: List[np.ndarray], N: int) -> np.ndarray:
+    """Gradient through the pyramid: level l token t is the mean of input
+    tokens t*2^l .. t*2^l + 2^l - 1, so each of them receives 1/2^l of its
+    gradient; level 0 is the input itself."""
+    out = grads[0].copy()
+    for l in range(1, len(grads)):
+        g = 1 << l
+        out += np.repeat(grads[l], g, axis=2)[:, :, :N] / g
+    return out
 
 
 def executed_flops(mask, N: int, block: int, d: int, causal: bool = False) -> float:

@@ -26,11 +26,16 @@ something other than itself.
                         equivalence; identical-group invariance; NaN in a
                         skipped block changes nothing; pure-Python brute force
                         over an exhaustive {0,1,2,3,SKIP} mask; empty rows
+  attention_backward /  torch autograd through torch avg_pool1d and softmax
+  pool_backward         (independent routines), with and without causal
+                        masking and GQA; central finite differences; all level
+                        0 == torch SDPA autograd; sum of dK over tokens is 0;
+                        sum of dV is the sum of dO over rows that see a key
   mutation tests        planted mistakes (bias sign, dropped bias, sum instead of
                         mean, wrong block width, inclusive prefix, transposed
                         antidiagonal, rank off by one, ragged mean over the
-                        full block, transposed mean-key logits) each make a pin
-                        fail
+                        full block, transposed mean-key logits, pooling
+                        gradient without 1/2^l) each make a pin fail
 """
 import json
 import math
@@ -657,3 +662,139 @@ def test_mutation_meankey_transposed(monkeypatch, golden_dir):
         return O._softmax_rows(z)[None, None]
     monkeypatch.setattr(O, "meankey_mass", planted)
     assert _meankey_golden_case(golden_dir, False) > 1e-3
+
+
+# --------------------------------------------------------------------------------------
+# backward pass (next row of the scope table): dQ, dK, dV through the levels
+# --------------------------------------------------------------------------------------
+
+def torch_psa_grads(q, k, v, mask, block, sm_scale, causal, levels, dout):
+    """The forward written again with torch ops (avg_pool1d pyramid, gather,
+    softmax), differentiated by torch autograd."""
+    q = q.clone().requires_grad_(True)
+    k = k.clone().requires_grad_(True)
+    v = v.clone().requires_grad_(True)
+    B, Hq, N, d = q.shape
+    grp = Hq // k.shape[1]
+    nb = -(-N // block)
+
+    def pool(x, l):
+        if l == 0:
+            return x
+        g = 1 << l
+        y = x.reshape(-1, N, d).transpose(1, 2)
+        y = torch.nn.functional.avg_pool1d(y, g, g)
+        return y.transpose(1, 2).reshape(x.shape[0], x.shape[1], -1, d)
+    kl = [pool(k, l) for l in range(levels)]
+    vl = [pool(v, l) for l in range(levels)]
+    loss = q.new_zeros(())
+    for b in range(B):
+        for h in range(Hq):
+            for I in range(nb):
+                i0, i1 = I * block, min((I + 1) * block, N)
+                ks, vs, bs, lastt = [], [], [], []
+                for J in range(nb):
+                    l = int(mask[b, h, I, J])
+                    if l == SKIP:
+                        continue
+                    g = 1 << l
+                    p0, p1 = (J * block) // g, min((J + 1) * block, N) // g
+                    ks.append(kl[l][b, h // grp, p0:p1])
+                    vs.append(vl[l][b, h // grp, p0:p1])
+                    bs += [l * math.log(2.0)] * (p1 - p0)
+                    lastt += [(p + 1) * g - 1 for p in range(p0, p1)]
+                if not ks:
+                    continue
+                z = sm_scale * q[b, h, i0:i1] @ torch.cat(ks).T + torch.tensor(bs, dtype=q.dtype)
+                if causal:
+                    vis = torch.tensor(lastt)[None, :] <= torch.arange(i0, i1)[:, None]
+                    z = z.masked_fill(~vis, float("-inf"))
+                    keep = vis.any(dim=1)
+                else:
+                    keep = torch.ones(i1 - i0, dtype=torch.bool)
+                p_ = torch.softmax(z[keep], dim=-1)
+                loss = loss + (p_ @ torch.cat(vs) * dout[b, h, i0:i1][keep]).sum()
+    loss.backward()
+    return q.grad.numpy(), k.grad.numpy(), v.grad.numpy()
+
+
+def _bwd_case(causal, seed=5):
+    g = torch.Generator().manual_seed(seed)
+    B, Hq, Hkv, N, d, blk, L = 1, 4, 2, 96, 8, 16, 4
+    q = torch.randn(B, Hq, N, d, generator=g, dtype=torch.float64)
+    k = torch.randn(B, Hkv, N, d, generator=g, dtype=torch.float64)
+    v = torch.randn(B, Hkv, N, d, generator=g, dtype=torch.float64)
+    do = torch.randn(B, Hq, N, d, generator=g, dtype=torch.float64)
+    nb = N // blk
+    m = torch.randint(0, L + 1, (B, Hq, nb, nb), generator=g)
+    m = torch.where(m == L, torch.full_like(m, SKIP), m)
+    return q, k, v, m, blk, 0.35, causal, L, do
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_vs_torch_autograd(causal):
+    args = _bwd_case(causal)
+    got = O.attention_backward(*args)
+    want = torch_psa_grads(*args)
+    for a_, b_ in zip(got, want):
+        assert np.abs(a_ - b_).max() <= 1e-12
+
+
+def test_backward_finite_differences():
+    q, k, v, m, blk, sc, causal, L, do = _bwd_case(True, seed=9)
+    dq, dk, dv = O.attention_backward(q, k, v, m, blk, sc, causal, L, do)
+
+    def loss(q_, k_, v_):
+        kl, vl = O.build_pyramid(k_, v_, L)
+        o, _ = O.attention(q_, kl, vl, m, blk, sc, causal)
+        return float((np.nan_to_num(o) * do.numpy()).sum())
+    eps = 1e-6
+    rng = np.random.default_rng(0)
+    for which, grad, t in (("q", dq, q), ("k", dk, k), ("v", dv, v)):
+        for _ in range(4):
+            idx = tuple(int(rng.integers(n)) for n in t.shape)
+            tp, tm = t.clone(), t.clone()
+            tp[idx] += eps
+            tm[idx] -= eps
+            args_p = {"q": (tp, k, v), "k": (q, tp, v), "v": (q, k, tp)}[which]
+            args_m = {"q": (tm, k, v), "k": (q, tm, v), "v": (q, k, tm)}[which]
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+            assert abs(fd - grad[idx]) <= 1e-6 * max(1.0, abs(fd)), (which, idx, fd, grad[idx])
+
+
+def test_backward_level0_is_dense_sdpa():
+    g = torch.Generator().manual_seed(3)
+    q = torch.randn(1, 1, 48, 8, generator=g, dtype=torch.float64)
+    k = torch.randn(1, 1, 48, 8, generator=g, dtype=torch.float64)
+    v = torch.randn(1, 1, 48, 8, generator=g, dtype=torch.float64)
+    do = torch.randn(1, 1, 48, 8, generator=g, dtype=torch.float64)
+    mask = torch.zeros(1, 1, 3, 3, dtype=torch.int64)
+    dq, dk, dv = O.attention_backward(q, k, v, mask, 16, 0.4, False, 4, do)
+    qt, kt, vt = (x.clone().requires_grad_(True) for x in (q, k, v))
+    o = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, scale=0.4)
+    (o * do).sum().backward()
+    for a_, b_ in ((dq, qt.grad), (dk, kt.grad), (dv, vt.grad)):
+        assert np.abs(a_ - b_.numpy()).max() <= 1e-12
+
+
+def test_backward_sum_invariants():
+    q, k, v, m, blk, sc, causal, L, do = _bwd_case(True, seed=11)
+    dq, dk, dv = O.attention_backward(q, k, v, m, blk, sc, causal, L, do)
+    kl, vl = O.build_pyramid(k, v, L)
+    _, lse = O.attention(q, kl, vl, m, blk, sc, causal)
+    seen = np.isfinite(lse)                                    # rows with a visible key
+    assert np.abs(dk.sum(axis=2)).max() <= 1e-12
+    grp = q.shape[1] // k.shape[1]
+    want = (do.numpy() * seen[..., None]).reshape(1, k.shape[1], grp, -1, q.shape[-1]).sum(axis=(2, 3))
+    assert np.abs(dv.sum(axis=2) - want).max() <= 1e-12
+
+
+def test_mutation_pool_backward_without_scale(monkeypatch):
+    def planted(grads, N):
+        out = grads[0].copy()
+        for l in range(1, len(grads)):
+            out += np.repeat(grads[l], 1 << l, axis=2)[:, :, :N]
+        return out
+    monkeypatch.setattr(O, "pool_backward", planted)
+    with pytest.raises(AssertionError):
+        test_backward_vs_torch_autograd(False)
