@@ -12,7 +12,14 @@ something other than itself.
   sampling_mass         sum over J == 1; pure-Python brute force; torch.softmax
                         (an independent library routine); one-hot alignment
   antidiag_logits/mass  element-wise brute force; stride 1 reduces to the
-                        block-summed full softmax (torch); sum over J == 1
+                        block-summed full softmax (torch); sum over J == 1;
+                        pure-Python brute force of the group -> block
+                        aggregation at strides 2 and 4 (causal, ragged, GQA)
+  ambiguous_pairs /     hand-derived dyadic goldens (threshold at C_J, at
+  ambiguous_pairs_      C_J +- 2 eps and +- eps/2, exact ties, near-ties within
+  quantile              and outside relative eps, relative vs absolute eps,
+                        cosine at cos_min +- eps); every level flip under a
+                        1e-7 relative perturbation lies in the band
   assign_levels_row     hand-computed golden cases; monotone in rank; top = 0
   apply_forced_rules    hand-computed golden cases
   assign_levels_quantile_row
@@ -35,7 +42,11 @@ something other than itself.
                         mean, wrong block width, inclusive prefix, transposed
                         antidiagonal, rank off by one, ragged mean over the
                         full block, transposed mean-key logits, pooling
-                        gradient without 1/2^l) each make a pin fail
+                        gradient without 1/2^l, band edges that keep the
+                        block itself / use an absolute eps / flip a sign,
+                        rank range off by one, n_vis ignoring causality,
+                        antidiagonal key groups summed at the wrong width)
+                        each make a pin fail
 """
 import json
 import math
@@ -798,3 +809,185 @@ def test_mutation_pool_backward_without_scale(monkeypatch):
     monkeypatch.setattr(O, "pool_backward", planted)
     with pytest.raises(AssertionError):
         test_backward_vs_torch_autograd(False)
+
+
+# --------------------------------------------------------------------------------------
+# the parity band: ambiguous_pairs / ambiguous_pairs_quantile
+# --------------------------------------------------------------------------------------
+
+def _row(mass):
+    return np.asarray(mass, dtype=np.float64)[None, None, None, :]
+
+
+def pin_ambiguous_golden(golden_dir, mod=O):
+    """Number of hand-derived band cases the oracle gets wrong (0 = pinned)."""
+    g = json.load(open(os.path.join(golden_dir, "ambiguous_hand.json")))
+    eps = g["eps"]
+    wrong = 0
+    for case in g["mass_cases"]:
+        got = mod.ambiguous_pairs(_row(case["mass"]), case["thresholds"], eps)[0, 0, 0]
+        wrong += int(got.tolist() != case["expect"])
+    c = g["cos_case"]
+    cos = np.asarray(c["blockcos"], dtype=np.float64)[None, None, :]
+    got = mod.ambiguous_pairs(_row(c["mass"]), c["thresholds"], eps, blockcos=cos, cos_min=c["cos_min"])[0, 0, 0]
+    wrong += int(got.tolist() != c["expect"])
+    off = mod.ambiguous_pairs(_row(c["mass"]), c["thresholds"], eps, blockcos=cos, cos_min=-3.0)[0, 0, 0]
+    wrong += int(off.any())
+    for case in g["quantile_cases"]:
+        n = len(case["mass"])
+        mass = np.zeros((1, 1, n, n))
+        mass[0, 0, case["I"]] = case["mass"]
+        got = mod.ambiguous_pairs_quantile(mass, case["thresholds"], len(case["thresholds"]), case["causal"], eps,
+                                           rows=[(0, 0, case["I"])])[0, 0, case["I"]]
+        wrong += int(got.tolist() != case["expect"])
+    return wrong
+
+
+def test_ambiguous_golden(golden_dir):
+    assert pin_ambiguous_golden(golden_dir) == 0
+
+
+def test_ambiguous_band_brackets_every_fp32_flip():
+    """Every pair whose level changes when the masses are perturbed by a
+    relative 1e-7 (the size of fp32 rounding of an fp64 mass) must lie in
+    the band.  The rows are random, with a planted near-tie and thresholds
+    placed on (or within 5e-7 of) exact prefixes so that flips do happen;
+    the band stays a small fraction of the pairs."""
+    rng = np.random.default_rng(7)
+    flips = flagged = total = 0
+    for _ in range(200):
+        n = int(rng.integers(6, 40))
+        m = rng.dirichlet(np.ones(n))
+        m[rng.integers(0, n)] = m[rng.integers(0, n)] * (1 + 3e-8)        # plant a near-tie
+        m = m / m.sum()
+        C = np.sort(O.exclusive_prefix(m))
+        k1, k2, k3 = rng.choice(np.arange(1, n), size=3, replace=False)
+        th = tuple(sorted((C[k1], C[k2] + 5e-7, C[k3] + 3e-6, 2.0)))
+        amb = O.ambiguous_pairs(m[None, None, None, :], th, 1e-6)[0, 0, 0]
+        base = O.assign_levels_row(m, th, 4)
+        for _ in range(20):
+            p = m * (1 + 1e-7 * rng.standard_normal(n))
+            moved = O.assign_levels_row(p, th, 4) != base
+            flips += int(moved.sum())
+            assert not np.any(moved & ~amb)
+        flagged += int(amb.sum())
+        total += n
+    assert flips > 100, flips
+    assert flagged <= 0.25 * total, (flagged, total)
+
+
+def _bad_ambiguous(variant):
+    """ambiguous_pairs with one planted mistake (mutation tests)."""
+    def bad(mass, thresholds, eps=1e-6, rows=None, blockcos=None, cos_min=-3.0, hq_per_kv=1):
+        B, Hq, nqb, nkb = mass.shape
+        amb = np.zeros(mass.shape, dtype=bool)
+        if rows is None:
+            rows = [(b, h, I) for b in range(B) for h in range(Hq) for I in range(nqb)]
+        for b, h, I in rows:
+            m = mass[b, h, I]
+            for J in range(nkb):
+                if variant == "absolute_eps":
+                    lo = m[m > m[J] + eps].sum()
+                    hi = m[m >= m[J] - eps].sum() - m[J]
+                else:
+                    lo = m[m > m[J] * (1 + eps)].sum()
+                    hi = m[m >= m[J] * (1 - eps)].sum() - (0.0 if variant == "hi_keeps_self" else m[J])
+                lo_edge = lo + eps if variant == "lo_sign" else lo - eps
+                for t in thresholds:
+                    if lo_edge <= t <= hi + eps:
+                        amb[b, h, I, J] = True
+                if blockcos is not None and cos_min > -2.0 and abs(blockcos[b, h // hq_per_kv, J] - cos_min) <= eps:
+                    amb[b, h, I, J] = True
+        return amb
+    return bad
+
+
+@pytest.mark.parametrize("variant", ["hi_keeps_self", "absolute_eps", "lo_sign"])
+def test_mutation_ambiguous_band(monkeypatch, golden_dir, variant):
+    monkeypatch.setattr(O, "ambiguous_pairs", _bad_ambiguous(variant))
+    assert pin_ambiguous_golden(golden_dir, O) > 0
+
+
+def test_mutation_ambiguous_quantile_rank_range(monkeypatch, golden_dir):
+    """r_hi counted without excluding the block itself widens every rank
+    range by one and flags isolated blocks next to a level boundary."""
+    def bad(mass, thresholds, levels, causal, eps=1e-6, rows=None):
+        B, Hq, nqb, nkb = mass.shape
+        amb = np.zeros(mass.shape, dtype=bool)
+        for b, h, I in rows:
+            m = mass[b, h, I]
+            nv = min(I + 1, nkb) if causal else nkb
+            for J in range(nkb):
+                r_lo = int((m > m[J] * (1 + eps)).sum())
+                r_hi = int((m >= m[J] * (1 - eps)).sum())
+                lev = {sum(1 for t in thresholds if t <= r / nv) for r in (r_lo, r_hi)}
+                amb[b, h, I, J] = len(lev) > 1
+        return amb
+    monkeypatch.setattr(O, "ambiguous_pairs_quantile", bad)
+    assert pin_ambiguous_golden(golden_dir, O) > 0
+
+
+def test_mutation_ambiguous_quantile_ignores_causal(monkeypatch, golden_dir):
+    orig = O.ambiguous_pairs_quantile
+    monkeypatch.setattr(O, "ambiguous_pairs_quantile",
+                        lambda mass, th, levels, causal, eps=1e-6, rows=None: orig(mass, th, levels, False, eps, rows))
+    assert pin_ambiguous_golden(golden_dir, O) > 0
+
+
+# --------------------------------------------------------------------------------------
+# antidiagonal block masses at stride S > 1: pure-Python brute force
+# --------------------------------------------------------------------------------------
+
+def brute_antidiag_mass(q, k, block, S, scale, causal):
+    """Reading R6 with loops only: the antidiagonal logit of every (query
+    group a, key group c), a softmax over the visible key groups, each
+    group probability added to the key block holding the group's tokens,
+    and the mean over the query groups of each query block."""
+    N, d = len(q), len(q[0])
+    G = N // S
+    nb = -(-N // block)
+    mass = [[0.0] * nb for _ in range(nb)]
+    groups_in = [0] * nb
+    for a in range(G):
+        z = {}
+        for c in range(G):
+            if causal and c > a:
+                continue
+            acc = 0.0
+            for s in range(S):
+                i, j = a * S + S - 1 - s, c * S + s
+                acc += sum(q[i][x] * k[j][x] for x in range(d))
+            z[c] = scale * acc / S
+        mx = max(z.values())
+        e = {c: math.exp(v - mx) for c, v in z.items()}
+        tot = sum(e.values())
+        I = (a * S) // block
+        groups_in[I] += 1
+        for c, v in e.items():
+            mass[I][(c * S) // block] += v / tot
+    return [[x / groups_in[I] for x in row] for I, row in enumerate(mass)]
+
+
+@pytest.mark.parametrize("S,causal", [(2, False), (2, True), (4, True), (4, False)])
+def test_antidiag_mass_bruteforce_strided(S, causal):
+    """N = 40 tokens, block 16 (a ragged last block of 8 tokens), block / S
+    = 8 or 4 groups per block, GQA 2:1."""
+    N, d, blk, scale = 40, 3, 16, 0.8
+    q, k = rand(1, 2, N, d), rand(1, 1, N, d)
+    got = O.antidiag_mass(q, k, blk, S, scale, causal)
+    for h in range(2):
+        want = np.array(brute_antidiag_mass(q[0, h].tolist(), k[0, 0].tolist(), blk, S, scale, causal))
+        assert np.abs(got[0, h] - want).max() < 1e-12
+
+
+def test_mutation_antidiag_group_width(monkeypatch):
+    """Summing key groups in runs of the wrong width (tokens per block
+    instead of groups per block, here twice the groups) must fail the
+    strided brute force, although the masses still sum to one."""
+    orig = O._block_sum
+    monkeypatch.setattr(O, "_block_sum", lambda p, w, n: orig(p, 2 * w, n))
+    q, k = rand(1, 1, 256, 8), rand(1, 1, 256, 8)
+    m = O.antidiag_mass(q, k, 64, 8, 0.3, causal=True)
+    assert np.abs(m.sum(axis=-1) - 1).max() < 1e-12          # the invariant alone cannot see it
+    with pytest.raises(AssertionError):
+        test_antidiag_mass_bruteforce_strided(4, True)
