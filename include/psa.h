@@ -201,19 +201,26 @@ PSA_API psa_status_t psa_attention_fwd(const psa_shape_t* shape, const void* q, 
  * the process exits.  Shapes whose psa_attention_workspace_bytes exceeds it
  * are rejected with PSA_ERR_WORKSPACE before anything is launched (it covers,
  * for example, the Qwen2.5-VL- and Wan2.1-1.3B-shaped problems, not the
- * Wan2.1-14B-shaped one).  The first call on each device looks up the
- * array's device address (cudaGetSymbolAddress, with that device current),
- * so make that first call before any stream capture.  No device memory is
- * allocated or freed.  All calls share the one array and it keeps the last
- * call's contents; each call clears the 36-byte status header it needs at
- * zero, and calls that overlap on the GPU (other streams, other threads)
- * race on the array.  Time-out reports from the kernel stay inside the
- * array and are not readable through psa_get_device_status. */
+ * Wan2.1-14B-shaped one).  The first call on each device (of this function or
+ * of psa_get_static_device_status) looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current) and zero-fills its
+ * 256-byte header with a synchronous cudaMemset, so make that first call
+ * before any stream capture.  No device memory is allocated or freed.  All
+ * calls share the one array and it keeps the last call's contents; calls
+ * that overlap on the GPU (other streams, other threads) race on the array.
+ * A bounded-wait time-out in the kernel is recorded in the array's status
+ * word and stays there, across later calls, until
+ * psa_get_static_device_status reads and clears it. */
 #define PSA_STATIC_WORKSPACE_BYTES (32u << 20)
 PSA_API psa_status_t psa_attention_fwd_static(const psa_shape_t* shape, const void* q, const void* k,
                                               const void* v, const void* k_pyr, const void* v_pyr,
                                               const uint8_t* mask, float sm_scale, void* out, float* lse,
                                               void* stream);
+
+/* psa_get_device_status for the static workspace of
+ * psa_attention_fwd_static on the current device: reads (synchronising on
+ * `stream`) and clears its status word and time-out record. */
+PSA_API psa_status_t psa_get_static_device_status(void* stream);
 
 /* Executed work of the last plan built in `workspace` by psa_attention_fwd:
  * fills (synchronising on `stream`) the number of 128-row KV tiles and the
@@ -228,6 +235,18 @@ PSA_API psa_status_t psa_attention_plan_stats(const psa_shape_t* shape, const vo
  * thread and progress counters).  The status word and that record occupy
  * the first 36 bytes of every workspace. */
 PSA_API psa_status_t psa_get_device_status(void* workspace, void* stream);
+
+/* Debug and test aid: sets the limit, in nanoseconds, of the protocol waits
+ * (the waits between the producer, MMA and softmax roles) of the attention
+ * kernel when it runs on `workspace`; 0 restores the built-in limit (2 s).
+ * The value sits at bytes 40..47 of the workspace header; it outlives
+ * psa_get_device_status, which clears only the first 36 bytes.  A limit
+ * shorter than the work makes the kernel give up early: the call's outputs
+ * are then incomplete and psa_get_device_status returns PSA_ERR_TIMEOUT
+ * with the site of the first wait that gave up.  The waits that drain a
+ * CTA's in-flight copies and MMAs before it exits keep the built-in limit.
+ * Synchronises on `stream`.  `workspace` must be 8-byte aligned. */
+PSA_API psa_status_t psa_debug_set_wait_limit(void* workspace, uint64_t limit_ns, void* stream);
 
 /* Message of the last failed call on this thread ("" if none). */
 PSA_API const char* psa_last_error(void);

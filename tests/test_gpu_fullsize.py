@@ -2,7 +2,9 @@
 benchmark runs it (inputs generated on the GPU, the whole path through the
 C ABI, the persistent kernels at full grid), checked on sampled query
 blocks that the oracle recomputes one by one: the mask rows (bit-exact
-outside the ambiguity band), the block masses, and the attention rows."""
+outside the ambiguity band), the block masses, and the attention rows.
+At least 64 (head, query block) rows per preset: every head of the first,
+a middle and the ragged last block, plus random rows."""
 import numpy as np
 import pytest
 import torch
@@ -10,6 +12,7 @@ import torch
 import oracle.psa_oracle as O
 import video_transformers_b200 as P
 import workloads as W
+from amb_report import check_band
 from psa_run import SKIP, attn_errors, params_for, run_attention, run_mask, run_pyramid, shape_for
 
 pytestmark = pytest.mark.gpu
@@ -24,6 +27,28 @@ def sample_rows(w, n, seed):
     return [(0, int(h), int(I)) for h, I in zip(hs, Is)]
 
 
+def fullsize_rows(w, n_min=64, seed=0):
+    """Every head of the first, a middle and the (ragged) last query block,
+    topped up with random (head, block) rows to at least n_min."""
+    rows = {(0, h, I) for h in range(w.Hq) for I in (0, w.nqb // 2, w.nqb - 1)}
+    rng = np.random.default_rng(seed)
+    while len(rows) < n_min:
+        rows.add((0, int(rng.integers(0, w.Hq)), int(rng.integers(0, w.nqb))))
+    return sorted(rows)
+
+
+def by_head(rows):
+    out = {}
+    for b, h, I in rows:
+        out.setdefault((b, h), []).append(I)
+    return out
+
+
+def head_levels(shape, base, pyr, b, hk, levels):
+    return [base[b:b + 1, hk:hk + 1].double().cpu().numpy()] + \
+        [P.pyramid_level(shape, pyr, l)[b:b + 1, hk:hk + 1].double().cpu().numpy() for l in range(1, levels)]
+
+
 @pytest.mark.parametrize("name", ["wan1.3b", "cogvideox5b", "qwen2.5vl", "wan14b"])
 def test_fullsize_sampled_parity(name):
     w = W.PRESETS[name]
@@ -34,40 +59,69 @@ def test_fullsize_sampled_parity(name):
     out, lse, ws = run_attention(shape, q, k, v, kp, vp, mask, w.sm_scale)
     torch.cuda.synchronize()
     grp = w.Hq // w.Hkv
+    rows = fullsize_rows(w, seed=len(name))
+    assert len(rows) >= 64
     n_amb = n_pairs = 0
-    for b, h, I in sample_rows(w, 6, seed=len(name)):
+    cos_cache = {}
+    for (b, h), Is in by_head(rows).items():
         hk = h // grp
         qh, kh, vh = q[b:b + 1, h:h + 1].cpu(), k[b:b + 1, hk:hk + 1].cpu(), v[b:b + 1, hk:hk + 1].cpu()
-        row = [(0, 0, I)]
+        hrows = [(0, 0, I) for I in Is]
         if w.mask_mode == "sample":
-            om = O.sampling_mass(qh, kh, w.block, w.sm_scale, w.causal, rows=row)
+            om = O.sampling_mass(qh, kh, w.block, w.sm_scale, w.causal, rows=hrows)
         else:
-            om = O.antidiag_mass(qh, kh, w.block, w.stride, w.sm_scale, w.causal, rows=row)
+            om = O.antidiag_mass(qh, kh, w.block, w.stride, w.sm_scale, w.causal, rows=hrows)
         cos = None
         if bc is not None:
             cos = bc[b:b + 1, hk:hk + 1].cpu().numpy().astype(np.float64)
-            ocos = O.block_cosine(kh, w.block)
-            assert np.abs(cos - ocos).max() <= 1e-5
+            if hk not in cos_cache:
+                cos_cache[hk] = O.block_cosine(kh, w.block)
+                assert np.abs(cos - cos_cache[hk]).max() <= 1e-5
         omask = O.make_mask(om, w.thresholds, w.levels, w.block, w.causal, w.n_dense_prefix, cos, w.cos_min,
-                            1, rows=row)[0, 0, I]
-        amb = O.ambiguous_pairs(om, w.thresholds, 1e-6, row, cos, w.cos_min, 1)[0, 0, I]
-        gm = mask[b, h, I].cpu().numpy()
-        gmass = mass[b, h, I].cpu().numpy().astype(np.float64)
-        big = om[0, 0, I] > 1e-6
-        assert (np.abs(gmass[big] - om[0, 0, I][big]) / om[0, 0, I][big]).max() <= 1e-4
-        assert np.all((gm == omask) | amb), (name, h, I, int(((gm != omask) & ~amb).sum()))
-        n_amb += int(amb.sum())
-        n_pairs += amb.size
-        # attention rows of this query block, from the GPU pyramid and mask
-        kl = [kh.double().numpy()] + [P.pyramid_level(shape, kp, l)[b:b + 1, hk:hk + 1].double().cpu().numpy()
-                                      for l in range(1, w.levels)]
-        vl = [vh.double().numpy()] + [P.pyramid_level(shape, vp, l)[b:b + 1, hk:hk + 1].double().cpu().numpy()
-                                      for l in range(1, w.levels)]
-        o, l = O.attention(qh, kl, vl, mask[b:b + 1, h:h + 1].cpu(), w.block, w.sm_scale, w.causal, rows=row)
+                            1, rows=hrows)[0, 0]
+        amb = O.ambiguous_pairs(om, w.thresholds, 1e-6, hrows, cos, w.cos_min, 1)[0, 0]
+        gm = mask[b, h].cpu().numpy()
+        gmass = mass[b, h].cpu().numpy().astype(np.float64)
+        for I in Is:
+            big = om[0, 0, I] > 1e-6
+            assert (np.abs(gmass[I][big] - om[0, 0, I][big]) / om[0, 0, I][big]).max() <= 1e-4
+            assert np.all((gm[I] == omask[I]) | amb[I]), (name, h, I, int(((gm[I] != omask[I]) & ~amb[I]).sum()))
+            n_amb += int(amb[I].sum())
+            n_pairs += amb[I].size
+        # attention rows of these query blocks, from the GPU pyramid and mask
+        kl = head_levels(shape, k, kp, b, hk, w.levels)
+        vl = head_levels(shape, v, vp, b, hk, w.levels)
+        o, l = O.attention(qh, kl, vl, mask[b:b + 1, h:h + 1].cpu(), w.block, w.sm_scale, w.causal, rows=hrows)
         mx, mean, _ = attn_errors(out[b:b + 1, h:h + 1], o)
-        assert mx <= 2e-2 and mean <= 2e-3, (name, h, I, mx, mean)
+        assert mx <= 2e-2 and mean <= 2e-3, (name, h, Is, mx, mean)
+        lg = lse[b, h].cpu().numpy().astype(np.float64)
+        sel = ~np.isnan(l[0, 0])
+        assert np.abs(lg[sel] - l[0, 0][sel]).max() <= 2e-2
     assert P.psa_get_device_status(ws) == P.PSA_OK
-    print("%s: %d ambiguous of %d sampled pairs" % (name, n_amb, n_pairs))
+    check_band("%s full size, %d rows" % (name, len(rows)), n_amb, n_pairs)
+
+
+def test_fullsize_dense_wan14b():
+    """The dense reference point the benchmark times: the Wan2.1-14B shape
+    with every pair at level 0, checked on sampled query-block rows against
+    the oracle's plain softmax attention over all 75,600 keys."""
+    w = W.PRESETS["wan14b"]
+    q, k, v, _ = W.make_qkv(w, device=DEV)
+    shape = shape_for(w)
+    kp, vp, _ = run_pyramid(shape, k, v)
+    mask = torch.zeros(w.B, w.Hq, w.nqb, w.nqb, dtype=torch.uint8, device=DEV)
+    out, lse, ws = run_attention(shape, q, k, v, kp, vp, mask, w.sm_scale)
+    torch.cuda.synchronize()
+    for b, h, I in sample_rows(w, 12, seed=99):
+        row = [(0, 0, I)]
+        o, l = O.attention(q[b:b + 1, h:h + 1].cpu(), [k[b:b + 1, h:h + 1].cpu().double().numpy()],
+                           [v[b:b + 1, h:h + 1].cpu().double().numpy()], mask[b:b + 1, h:h + 1, :, :].cpu(),
+                           w.block, w.sm_scale, False, rows=row)
+        mx, mean, _ = attn_errors(out[b:b + 1, h:h + 1], o)
+        assert mx <= 2e-2 and mean <= 2e-3, (h, I, mx, mean)
+    nt, nr = P.psa_attention_plan_stats(shape, ws)
+    assert nr == w.Hq * w.nqb * w.N and nt == w.Hq * w.nqb * w.nqb
+    assert P.psa_get_device_status(ws) == P.PSA_OK
 
 
 @pytest.mark.parametrize("mode,policy", [("meankey", "mass"), ("sample", "quantile")])
@@ -85,6 +139,7 @@ def test_fullsize_mask_variants_sampled(mode, policy):
     out, lse, ws = run_attention(shape, q, k, v, kp, vp, mask, w.sm_scale)
     torch.cuda.synchronize()
     th = [float(np.float32(t)) for t in w.thresholds]
+    n_amb = n_pairs = 0
     for b, h, I in sample_rows(w, 4, seed=7 + len(mode)):
         qh, kh, vh = q[b:b + 1, h:h + 1].cpu(), k[b:b + 1, h:h + 1].cpu(), v[b:b + 1, h:h + 1].cpu()
         row = [(0, 0, I)]
@@ -103,6 +158,8 @@ def test_fullsize_mask_variants_sampled(mode, policy):
         big = om[0, 0, I] > 1e-6
         assert (np.abs(gmass[big] - om[0, 0, I][big]) / om[0, 0, I][big]).max() <= 1e-4
         assert np.all((gm == omask) | amb), (mode, policy, h, I, int(((gm != omask) & ~amb).sum()))
+        n_amb += int(amb.sum())
+        n_pairs += amb.size
         kl = [kh.double().numpy()] + [P.pyramid_level(shape, kp, l)[b:b + 1, h:h + 1].double().cpu().numpy()
                                       for l in range(1, w.levels)]
         vl = [vh.double().numpy()] + [P.pyramid_level(shape, vp, l)[b:b + 1, h:h + 1].double().cpu().numpy()
@@ -111,3 +168,4 @@ def test_fullsize_mask_variants_sampled(mode, policy):
         mx, mean, _ = attn_errors(out[b:b + 1, h:h + 1], o)
         assert mx <= 2e-2 and mean <= 2e-3, (mode, policy, h, I, mx, mean)
     assert P.psa_get_device_status(ws) == P.PSA_OK
+    check_band("wan14b full size, %s/%s" % (mode, policy), n_amb, n_pairs)

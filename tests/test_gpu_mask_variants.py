@@ -17,6 +17,7 @@ import torch
 import oracle.psa_oracle as O
 import video_transformers_b200 as P
 import workloads as W
+from amb_report import check_band
 from psa_run import SKIP, attn_errors, levels_of, params_for, run_attention, run_mask, run_pyramid, shape_for
 
 pytestmark = pytest.mark.gpu
@@ -49,6 +50,7 @@ def check_variant(w, q, k, policy):
     assert rel.max() <= 1e-4, rel.max()
     bad = ~amb & (mask != omask)
     assert bad.sum() == 0, "mask mismatches outside the ambiguity band: %d (ambiguous %d)" % (bad.sum(), amb.sum())
+    check_band("%s %s/%s L=%d N=%d" % (w.name, w.mask_mode, pol, w.levels, w.N), int(amb.sum()), int(amb.size))
     return mask
 
 

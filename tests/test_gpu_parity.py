@@ -16,6 +16,7 @@ import torch
 import oracle.psa_oracle as O
 import video_transformers_b200 as P
 import workloads as W
+from amb_report import check_band
 from psa_run import (SKIP, attn_errors, bf16_ulp, levels_of, params_for, run_attention, run_mask,
                      run_pyramid, shape_for)
 
@@ -102,6 +103,7 @@ def check_mask(w, q, k, rows=None):
     assert rel.max() <= 1e-4, rel.max()
     bad = sel & ~amb & (mask != omask)
     assert bad.sum() == 0, "mask mismatches outside the ambiguity band: %d (ambiguous %d)" % (bad.sum(), (amb & sel).sum())
+    check_band("%s %s N=%d" % (w.name, w.mask_mode, w.N), int((amb & sel).sum()), int(sel.sum()))
     return mask, int((amb & sel).sum()), int(sel.sum())
 
 

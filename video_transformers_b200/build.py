@@ -37,7 +37,7 @@ def nvcc() -> str:
 
 def _deps(src: str):
     deps = [src]
-    for h in ("internal.h", "sm100.cuh"):
+    for h in ("internal.h", "sm100.cuh", "exp2_poly.h"):
         deps.append(os.path.join(CSRC, h))
     deps.append(os.path.join(ROOT, "include", "psa.h"))
     return deps

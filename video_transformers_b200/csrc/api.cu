@@ -7,9 +7,43 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
+#include <vector>
 
 #include "internal.h"
+
+namespace psa {
+
+int device_sm_count() {
+  constexpr int kDevs = 64;
+  static std::atomic<int> cache[kDevs] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevs) return 148;
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n > 0) return n;
+  n = 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) n = 148;
+  cache[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+cudaError_t set_smem_limit(const void* fn, int bytes) {
+  struct Entry { const void* fn; int dev; int bytes; };
+  static std::mutex mu;
+  static std::vector<Entry> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const Entry& x : done)
+    if (x.fn == fn && x.dev == dev && x.bytes >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.push_back({fn, dev, bytes});
+  return e;
+}
+
+}  // namespace psa
 
 namespace {
 
@@ -85,12 +119,7 @@ psa_status_t map4(CUtensorMap* m, const void* base, int64_t BH, int64_t N, int d
   return encode_bf16(m, base, 4, dims, str, box);
 }
 
-int num_sms() {
-  int dev = 0, n = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n;
-}
+int num_sms() { return psa::device_sm_count(); }
 
 // ------------------------------------------------------------------ validation
 psa_status_t check_shape(const psa_shape_t* s) {
@@ -247,6 +276,25 @@ AttnLayout attn_layout(const psa_shape_t* s) {
   }
   L.total = off;
   return L;
+}
+
+// Byte offset, inside every workspace header, of the 64-bit protocol wait
+// limit read by the attention kernel (0 = the built-in limit).
+constexpr size_t kWaitLimitOffset = 40;
+
+// Reads the status word and time-out record at the start of a workspace
+// header, clears them (36 bytes: the wait limit after them is kept), and
+// turns them into a status and message.
+psa_status_t read_status(void* hdr, void* stream) {
+  int w[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
+  cudaStream_t str = static_cast<cudaStream_t>(stream);
+  PSA_CUDA(cudaMemcpyAsync(w, hdr, sizeof(w), cudaMemcpyDeviceToHost, str), "status copy");
+  PSA_CUDA(cudaMemsetAsync(hdr, 0, sizeof(w), str), "status clear");
+  PSA_CUDA(cudaStreamSynchronize(str), "status sync");
+  if (w[0] == 0) return PSA_OK;
+  return fail(static_cast<psa_status_t>(w[0]),
+              "device status %d: a bounded wait ran out (site %d, block %d, thread %d, counters %d %d %d %d)",
+              w[0], w[2], w[3], w[4], w[5], w[6], w[7], w[8]);
 }
 
 }  // namespace
@@ -479,15 +527,18 @@ psa_status_t psa_attention_plan_stats(const psa_shape_t* s, const void* ws, int6
 psa_status_t psa_get_device_status(void* ws, void* stream) {
   g_err[0] = 0;
   if (!ws) return fail(PSA_ERR_INVALID_ARG, "workspace is NULL");
-  int w[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
+  return read_status(ws, stream);
+}
+
+psa_status_t psa_debug_set_wait_limit(void* ws, uint64_t limit_ns, void* stream) {
+  g_err[0] = 0;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 7u)) return fail(PSA_ERR_INVALID_ARG, "workspace is NULL or misaligned");
   cudaStream_t str = static_cast<cudaStream_t>(stream);
-  PSA_CUDA(cudaMemcpyAsync(w, ws, sizeof(w), cudaMemcpyDeviceToHost, str), "status copy");
-  PSA_CUDA(cudaMemsetAsync(ws, 0, sizeof(w), str), "status clear");
-  PSA_CUDA(cudaStreamSynchronize(str), "status sync");
-  if (w[0] == 0) return PSA_OK;
-  return fail(static_cast<psa_status_t>(w[0]),
-              "device status %d: a bounded wait ran out (site %d, block %d, thread %d, counters %d %d %d %d)",
-              w[0], w[2], w[3], w[4], w[5], w[6], w[7], w[8]);
+  const unsigned long long v = limit_ns;
+  PSA_CUDA(cudaMemcpyAsync(static_cast<char*>(ws) + kWaitLimitOffset, &v, sizeof(v), cudaMemcpyHostToDevice, str),
+           "wait limit copy");
+  PSA_CUDA(cudaStreamSynchronize(str), "wait limit sync");
+  return PSA_OK;
 }
 
 }  // extern "C"
@@ -514,12 +565,23 @@ psa_status_t static_workspace(void** out) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_static_workspace);
     if (e != cudaSuccess || !p) return cuda_fail(e, "cudaGetSymbolAddress of the static workspace");
+    // the header (status word, time-out record, wait limit) starts at zero;
+    // afterwards only psa_get_static_device_status clears the status part
+    e = cudaMemset(p, 0, 256);
+    if (e != cudaSuccess) return cuda_fail(e, "static workspace header clear");
     g_static_ptr[dev] = p;
   }
   *out = g_static_ptr[dev];
   return PSA_OK;
 }
 }  // namespace
+
+extern "C" psa_status_t psa_get_static_device_status(void* stream) {
+  g_err[0] = 0;
+  void* ws = nullptr;
+  PSA_TRY(static_workspace(&ws));
+  return read_status(ws, stream);
+}
 
 extern "C" psa_status_t psa_attention_fwd_static(const psa_shape_t* s, const void* q, const void* k, const void* v,
                                                  const void* k_pyr, const void* v_pyr, const uint8_t* mask,
@@ -545,8 +607,9 @@ extern "C" psa_status_t psa_attention_fwd_static(const psa_shape_t* s, const voi
   if (!(sm_scale > 0.f) || sm_scale != sm_scale) return fail(PSA_ERR_INVALID_ARG, "sm_scale must be > 0");
   void* ws = nullptr;
   PSA_TRY(static_workspace(&ws));
-  // the status header must start at zero; everything else is rewritten by the plan
-  PSA_CUDA(cudaMemsetAsync(ws, 0, 256, static_cast<cudaStream_t>(stream)), "static workspace header clear");
+  // the header was cleared once at set-up; a time-out stays recorded there
+  // until psa_get_static_device_status reads it, and everything after the
+  // header is rewritten by the plan of each call
   return psa_attention_fwd(s, q, k, v, k_pyr, v_pyr, mask, sm_scale, out, lse, ws, PSA_STATIC_WORKSPACE_BYTES,
                            stream);
 }

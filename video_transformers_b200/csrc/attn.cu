@@ -184,6 +184,7 @@ __global__ void __launch_bounds__(kThreads, CTAS)
   const uint32_t tmem = sh->tmem_base;
   const uint32_t tO = tmem + 128;
   volatile int* abort = &sh->abort;
+  const uint64_t wlim = protocol_wait_limit(a.status);
 
   if (warp == 0) {
     // =============================== producer ===============================
@@ -191,6 +192,7 @@ __global__ void __launch_bounds__(kThreads, CTAS)
       for (int i = 0; i < 1 + 2 * L; ++i) tma_prefetch_desc(&maps.m[i]);
     }
     uint32_t it = 0, qcnt = 0;       // it: sub-tiles loaded so far
+    uint32_t kiss = 0, viss = 0;     // K and V sub-tile loads issued (the drain waits for exactly these)
     bool ok = true;
     for (int idx = blockIdx.x; idx < a.n_items && ok; idx += gridDim.x) {
       const int item = a.queue[idx];
@@ -201,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, CTAS)
       const int b = bh / a.Hq, h = bh - b * a.Hq;
       const int hkv = b * a.Hkv + h / (a.Hq / a.Hkv);
       const int q0 = tq * 128;
-      if (!warp_wait(smem_u32(&sh->q_empty), (qcnt & 1) ^ 1, abort, a.status, 11, idx, qcnt, it, 0)) { ok = false; break; }
+      if (!warp_wait(smem_u32(&sh->q_empty), (qcnt & 1) ^ 1, abort, a.status, 11, idx, qcnt, it, 0, wlim)) { ok = false; break; }
       if (lane == 0) {
         const uint32_t bar = smem_u32(&sh->q_full);
         mbar_arrive_expect_tx(bar, QB);
@@ -248,7 +250,7 @@ __global__ void __launch_bounds__(kThreads, CTAS)
         const uint32_t ph = (it / NST) & 1;
 
         // K
-        if (!warp_wait(smem_u32(&sh->k_empty[st]), ph ^ 1, abort, a.status, 12, idx, j, it, 0)) { ok = false; break; }
+        if (!warp_wait(smem_u32(&sh->k_empty[st]), ph ^ 1, abort, a.status, 12, idx, j, it, 0, wlim)) { ok = false; break; }
         if (lane == 0) mbar_arrive_expect_tx(smem_u32(&sh->k_full[st]), SB);
         __syncwarp();
         if (mine) {
@@ -257,9 +259,10 @@ __global__ void __launch_bounds__(kThreads, CTAS)
             tma_load_3d(smem_u32(sK + st * SB + kc * 8192 + dst * 128), &maps.m[1 + l], smem_u32(&sh->k_full[st]),
                         kc * 64, prow, hkv);
         }
+        ++kiss;
 
         // sub-tile record
-        if (!warp_wait(smem_u32(&sh->i_empty[st]), ph ^ 1, abort, a.status, 13, idx, j, it, 0)) { ok = false; break; }
+        if (!warp_wait(smem_u32(&sh->i_empty[st]), ph ^ 1, abort, a.status, 13, idx, j, it, 0, wlim)) { ok = false; break; }
         SubInfo& ti = sh->ti[st];
         const int p_last = J * rows + lo + cnt;                // one past the last pooled row used here
         const int last_tok = (p_last << l) - 1;                // last token covered
@@ -316,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, CTAS)
         // V of the previous sub-tile
         if (j > 0) {
           const uint32_t pst = (it - 1) % NST;
-          if (!warp_wait(smem_u32(&sh->v_empty[pst]), (((it - 1) / NST) & 1) ^ 1, abort, a.status, 14, idx, j, it, 0)) { ok = false; break; }
+          if (!warp_wait(smem_u32(&sh->v_empty[pst]), (((it - 1) / NST) & 1) ^ 1, abort, a.status, 14, idx, j, it, 0, wlim)) { ok = false; break; }
           if (lane == 0) mbar_arrive_expect_tx(smem_u32(&sh->v_full[pst]), SB);
           __syncwarp();
           if (pv_mine) {
@@ -325,13 +328,14 @@ __global__ void __launch_bounds__(kThreads, CTAS)
               tma_load_3d(smem_u32(sV + pst * SB + kc * 8192 + pv_dst * 128), &maps.m[1 + L + pv_l],
                           smem_u32(&sh->v_full[pst]), kc * 64, pv_prow, hkv);
           }
+          ++viss;
         }
         pv_mine = mine; pv_l = l; pv_dst = dst; pv_prow = prow;
       }
       // V of the item's last sub-tile
       if (ok) {
         const uint32_t pst = (it - 1) % NST;
-        if (!warp_wait(smem_u32(&sh->v_empty[pst]), (((it - 1) / NST) & 1) ^ 1, abort, a.status, 15, idx, 0, it, 0)) { ok = false; break; }
+        if (!warp_wait(smem_u32(&sh->v_empty[pst]), (((it - 1) / NST) & 1) ^ 1, abort, a.status, 15, idx, 0, it, 0, wlim)) { ok = false; break; }
         if (lane == 0) mbar_arrive_expect_tx(smem_u32(&sh->v_full[pst]), SB);
         __syncwarp();
         if (pv_mine) {
@@ -340,16 +344,19 @@ __global__ void __launch_bounds__(kThreads, CTAS)
             tma_load_3d(smem_u32(sV + pst * SB + kc * 8192 + pv_dst * 128), &maps.m[1 + L + pv_l],
                         smem_u32(&sh->v_full[pst]), kc * 64, pv_prow, hkv);
         }
+        ++viss;
       }
     }
-    // drain: every TMA this warp issued must land before the CTA exits
+    // drain: every TMA this warp issued must land before the CTA exits.  The
+    // k-th K (V) load went to stage k % NST, phase k / NST, so the last load
+    // of stage st is number kiss - 1 - ((kiss - 1 - st) % NST) and its phase
+    // parity is ((kiss - 1 - st) / NST) & 1.  K and V are counted apart: after
+    // an abort the V ring trails the K ring by one load.
     if (lane == 0) {
       if (qcnt > 0) drain_wait(smem_u32(&sh->q_full), (qcnt - 1) & 1, a.status);
       for (uint32_t st = 0; st < static_cast<uint32_t>(NST); ++st) {
-        if (it > st) {
-          drain_wait(smem_u32(&sh->k_full[st]), ((it - 1 - st) / NST) & 1, a.status);
-          drain_wait(smem_u32(&sh->v_full[st]), ((it - 1 - st) / NST) & 1, a.status);
-        }
+        if (kiss > st) drain_wait(smem_u32(&sh->k_full[st]), ((kiss - 1 - st) / NST) & 1, a.status);
+        if (viss > st) drain_wait(smem_u32(&sh->v_full[st]), ((viss - 1 - st) / NST) & 1, a.status);
       }
     }
   } else if (warp == 1) {
@@ -368,10 +375,10 @@ __global__ void __launch_bounds__(kThreads, CTAS)
       auto issue_pv = [&](uint32_t jj, bool first_of_item) -> bool {
         const uint32_t g = it + jj, st = g % NST, sb2 = g & 1;
         if (first_of_item && icnt > 0) {
-          if (!bounded_wait(smem_u32(&sh->o_free), (icnt - 1) & 1, abort, a.status, 21, icnt, jj, g, 0)) return false;
+          if (!bounded_wait(smem_u32(&sh->o_free), (icnt - 1) & 1, abort, a.status, 21, icnt, jj, g, 0, wlim)) return false;
         }
-        if (!bounded_wait(smem_u32(&sh->p_full[sb2]), (g >> 1) & 1, abort, a.status, 22, icnt, jj, g, 0)) return false;
-        if (!bounded_wait(smem_u32(&sh->v_full[st]), (g / NST) & 1, abort, a.status, 26, icnt, jj, g, 0)) return false;
+        if (!bounded_wait(smem_u32(&sh->p_full[sb2]), (g >> 1) & 1, abort, a.status, 22, icnt, jj, g, 0, wlim)) return false;
+        if (!bounded_wait(smem_u32(&sh->v_full[st]), (g / NST) & 1, abort, a.status, 26, icnt, jj, g, 0, wlim)) return false;
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < kSub / 16; ++k) {
@@ -387,13 +394,13 @@ __global__ void __launch_bounds__(kThreads, CTAS)
         const int t0 = a.item_tile_off[item], t1 = a.item_tile_off[item + 1];
         if (t1 == t0) continue;
         const uint32_t n = sub_count(a.item_rows[item]);
-        if (!bounded_wait(smem_u32(&sh->q_full), qcnt & 1, abort, a.status, 23, idx, qcnt, it, 0)) { ok = false; break; }
+        if (!bounded_wait(smem_u32(&sh->q_full), qcnt & 1, abort, a.status, 23, idx, qcnt, it, 0, wlim)) { ok = false; break; }
         tc_fence_after();
         ++qcnt;
         for (uint32_t j = 0; j < n && ok; ++j) {
           const uint32_t g = it + j, st = g % NST, sb2 = g & 1;
           // S_j = Q K_j^T into S buffer sb2
-          if (!bounded_wait(smem_u32(&sh->k_full[st]), (g / NST) & 1, abort, a.status, 24, idx, j, g, 0)) { ok = false; break; }
+          if (!bounded_wait(smem_u32(&sh->k_full[st]), (g / NST) & 1, abort, a.status, 24, idx, j, g, 0, wlim)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int kc = 0; kc < KC; ++kc) {
@@ -448,8 +455,8 @@ __global__ void __launch_bounds__(kThreads, CTAS)
       float m = -CUDART_INF_F, lsum = 0.f;
       for (uint32_t j = 0; j < n; ++j, ++it) {
         const uint32_t st = it % NST, sb2 = it & 1;
-        if (!warp_wait(smem_u32(&sh->s_full[sb2]), (it >> 1) & 1, abort, a.status, 31, idx, j, it, 0)) { ok = false; break; }
-        if (!warp_wait(smem_u32(&sh->i_full[st]), (it / NST) & 1, abort, a.status, 32, idx, j, it, 0)) { ok = false; break; }
+        if (!warp_wait(smem_u32(&sh->s_full[sb2]), (it >> 1) & 1, abort, a.status, 31, idx, j, it, 0, wlim)) { ok = false; break; }
+        if (!warp_wait(smem_u32(&sh->i_full[st]), (it / NST) & 1, abort, a.status, 32, idx, j, it, 0, wlim)) { ok = false; break; }
         tc_fence_after();
         const SubInfo& ti = sh->ti[st];
         uint32_t sr[32], sr2[32];
@@ -526,7 +533,7 @@ __global__ void __launch_bounds__(kThreads, CTAS)
           const float f = grow ? fast_exp2(m - mnew) : 1.0f;
           lsum *= f;
           if (grow) m = mnew;
-          if (!warp_wait(smem_u32(&sh->o_ready), (it - 1) & 1, abort, a.status, 33, idx, j, it, 0)) { ok = false; break; }
+          if (!warp_wait(smem_u32(&sh->o_ready), (it - 1) & 1, abort, a.status, 33, idx, j, it, 0, wlim)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
@@ -552,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, CTAS)
       // epilogue: O / l once the item's last PV is done (o_final completes
       // once per item and cannot run ahead: the next item's first PV waits
       // for o_free)
-      if (!warp_wait(smem_u32(&sh->o_final), icnt & 1, abort, a.status, 35, idx, n, it, icnt)) { ok = false; break; }
+      if (!warp_wait(smem_u32(&sh->o_final), icnt & 1, abort, a.status, 35, idx, n, it, icnt, wlim)) { ok = false; break; }
       ++icnt;
       tc_fence_after();
       const float inv = lsum > 0.f ? 1.0f / lsum : 0.f;
@@ -613,13 +620,13 @@ cudaError_t launch_one(const AttnMaps& maps, const AttnArgs& a, int num_sms, cud
                       sizeof(AttnShared<NST>);
   const int grid = a.n_items < CTAS * num_sms ? a.n_items : CTAS * num_sms;
   if (a.block == 64) {
-    cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, F32, NST, CTAS, true>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(attn_kernel<D, F32, NST, CTAS, true>),
+                                   static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     attn_kernel<D, F32, NST, CTAS, true><<<grid, kThreads, smem, s>>>(maps, a);
   } else {
-    cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, F32, NST, CTAS, false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(attn_kernel<D, F32, NST, CTAS, false>),
+                                   static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     attn_kernel<D, F32, NST, CTAS, false><<<grid, kThreads, smem, s>>>(maps, a);
   }

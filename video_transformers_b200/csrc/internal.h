@@ -11,6 +11,12 @@
 
 namespace psa {
 
+// SM count of the current device, looked up once per device.
+int device_sm_count();
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) of kernel `fn` on the
+// current device, done once per (kernel, device) and remembered.
+cudaError_t set_smem_limit(const void* fn, int bytes);
+
 // 2^x for x <= 0 (a difference of log-sum-exps, log2 domain) with relative
 // error about 2.5e-7: x = n + f with n = floor(x) in fp64, 2^f of the
 // fraction rounded to fp32 from the special-function unit, 2^n applied to

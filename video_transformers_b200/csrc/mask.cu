@@ -595,7 +595,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectArgs a)
       double m = 0.0;
       for (int s = 0; s < nvalid; ++s) {
         const float x = bl[s];
-        if (x != -CUDART_INF_F) m += exp2(static_cast<double>(x) - rlse[s]);
+        if (x != -CUDART_INF_F) m += exp2_split(static_cast<double>(x) - rlse[s]);
       }
       const float mass = static_cast<float>(m / nvalid);
       if (a.mass_out) a.mass_out[static_cast<int64_t>(row) * a.nkb + J] = mass;
@@ -801,8 +801,8 @@ cudaError_t launch_score(const CUtensorMap* mapA, const CUtensorMap* mapB, const
     switch (a.cols_per_block) {
 #define PSA_SCORE2_CASE(CPB)                                                                       \
   case CPB: {                                                                                      \
-    cudaError_t e = cudaFuncSetAttribute(score2_kernel<CPB>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                                         static_cast<int>(smem2));                                 \
+    cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(score2_kernel<CPB>),            \
+                                   static_cast<int>(smem2));                                       \
     if (e != cudaSuccess) return e;                                                                \
     score2_kernel<CPB><<<grid2, kThreads, smem2, s>>>(*mapA, *mapB, a);                            \
     return cudaGetLastError();                                                                     \
@@ -819,8 +819,8 @@ cudaError_t launch_score(const CUtensorMap* mapA, const CUtensorMap* mapB, const
   switch (a.cols_per_block) {
 #define PSA_SCORE_CASE(CPB)                                                                       \
   case CPB: {                                                                                     \
-    cudaError_t e = cudaFuncSetAttribute(score_kernel<CPB>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                                         static_cast<int>(smem));                                 \
+    cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(score_kernel<CPB>),             \
+                                   static_cast<int>(smem));                                       \
     if (e != cudaSuccess) return e;                                                               \
     score_kernel<CPB><<<grid, kThreads, smem, s>>>(*mapA, *mapB, a);                              \
     break;                                                                                        \
@@ -839,9 +839,10 @@ cudaError_t launch_score(const CUtensorMap* mapA, const CUtensorMap* mapB, const
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t s) {
   const int rows = a.B * a.Hq * a.nqb;
   const int wgrid = (rows + kSelWarps - 1) / kSelWarps;
-  if (a.rows_per_block > 128) {
-    select_kernel<<<rows, kSelThreads, 0, s>>>(a);
-  } else if (a.nkb <= 32) {
+  // rows_per_block <= 128 always (8 sampled rows, 1 mean row, or block / S
+  // antidiagonal groups), which both kernels' row-LSE arrays rely on
+  if (a.rows_per_block > 128) return cudaErrorInvalidValue;
+  if (a.nkb <= 32) {
     select_warp_kernel<1><<<wgrid, 32 * kSelWarps, 0, s>>>(a);
   } else if (a.nkb <= 64) {
     select_warp_kernel<2><<<wgrid, 32 * kSelWarps, 0, s>>>(a);

@@ -185,9 +185,7 @@ __global__ void cast_kernel(const float4* __restrict__ src, uint2* __restrict__ 
 }
 
 int grid_for(int64_t work, int threads) {
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = device_sm_count();
   const int64_t want = (work + threads - 1) / threads;
   const int64_t cap = static_cast<int64_t>(sms) * 16;
   return static_cast<int>(want < cap ? (want > 0 ? want : 1) : cap);

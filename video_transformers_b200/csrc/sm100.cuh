@@ -73,26 +73,36 @@ __device__ __forceinline__ void record_timeout(int* status, int site, int c0, in
   }
 }
 
-// Wait for phase `parity` of an mbarrier, giving up after kWaitLimitNs (or
-// kWaitLimitIters polls), or as soon as another thread of the CTA has raised
-// *abort.  On its own time-out the thread raises *abort and records the wait
-// site and counters (record_timeout).  Returns false when the caller must
-// abandon its work.
+// Wait for phase `parity` of an mbarrier, giving up after `limit_ns` of
+// %globaltimer (or kWaitLimitIters polls), or as soon as another thread of
+// the CTA has raised *abort.  On its own time-out the thread raises *abort and
+// records the wait site and counters (record_timeout).  Returns false when
+// the caller must abandon its work.
 __device__ __forceinline__ bool bounded_wait(uint32_t bar, uint32_t parity, volatile int* abort, int* status,
-                                             int site = 0, int c0 = 0, int c1 = 0, int c2 = 0, int c3 = 0) {
+                                             int site = 0, int c0 = 0, int c1 = 0, int c2 = 0, int c3 = 0,
+                                             uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 31u) == 0) {
       if (*abort) return false;
-      if (globaltimer() - t0 > kWaitLimitNs || i >= kWaitLimitIters) {
+      if (globaltimer() - t0 > limit_ns || i >= kWaitLimitIters) {
         *abort = 1;
         record_timeout(status, site, c0, c1, c2, c3);
         return false;
       }
     }
   }
+}
+
+// Limit of the protocol waits of a kernel whose workspace header starts at
+// `status`: the 64-bit value at byte 40 of the header when it is non-zero
+// (set by psa_debug_set_wait_limit), else kWaitLimitNs.  Drain waits never
+// use it.
+__device__ __forceinline__ uint64_t protocol_wait_limit(const int* status) {
+  const uint64_t v = *reinterpret_cast<const volatile unsigned long long*>(status + 10);
+  return v ? v : kWaitLimitNs;
 }
 
 // Wait used while a CTA winds down: no abort flag, same two limits.
@@ -109,8 +119,9 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, int* s
 // Warp-uniform form for code that continues into .sync.aligned instructions:
 // every lane waits, and the warp gives up together if any lane gave up.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort, int* status,
-                                          int site = 0, int c0 = 0, int c1 = 0, int c2 = 0, int c3 = 0) {
-  const bool ok = bounded_wait(bar, parity, abort, status, site, c0, c1, c2, c3);
+                                          int site = 0, int c0 = 0, int c1 = 0, int c2 = 0, int c3 = 0,
+                                          uint64_t limit_ns = kWaitLimitNs) {
+  const bool ok = bounded_wait(bar, parity, abort, status, site, c0, c1, c2, c3, limit_ns);
   return __all_sync(0xffffffffu, ok);
 }
 
