@@ -236,17 +236,19 @@ PSA_API psa_status_t psa_attention_plan_stats(const psa_shape_t* shape, const vo
  * the first 36 bytes of every workspace. */
 PSA_API psa_status_t psa_get_device_status(void* workspace, void* stream);
 
-/* Debug and test aid: sets the limit, in nanoseconds, of the protocol waits
- * (the waits between the producer, MMA and softmax roles) of the attention
- * kernel when it runs on `workspace`; 0 restores the built-in limit (2 s).
- * The value sits at bytes 40..47 of the workspace header; it outlives
- * psa_get_device_status, which clears only the first 36 bytes.  A limit
- * shorter than the work makes the kernel give up early: the call's outputs
- * are then incomplete and psa_get_device_status returns PSA_ERR_TIMEOUT
- * with the site of the first wait that gave up.  The waits that drain a
- * CTA's in-flight copies and MMAs before it exits keep the built-in limit.
- * Synchronises on `stream`.  `workspace` must be 8-byte aligned. */
-PSA_API psa_status_t psa_debug_set_wait_limit(void* workspace, uint64_t limit_ns, void* stream);
+/* Debug and test aid for the time-out path of the attention kernel when it
+ * runs on `workspace` (the pages have no counterpart).  With trap != 0,
+ * every CTA waits once, right after its first K load, on a barrier that no
+ * thread arrives at; that wait gives up after limit_ns nanoseconds (0: the
+ * built-in 2 s), long before any other wait of the kernel could, so the
+ * CTA raises its abort flag, every role unwinds, the copies and MMAs in
+ * flight are drained, TMEM is freed, and psa_get_device_status returns
+ * PSA_ERR_TIMEOUT naming wait site 10.  The call's outputs are then
+ * incomplete.  The two values sit at bytes 40..51 of the workspace header
+ * and outlive psa_get_device_status, which clears only the first 36 bytes;
+ * call again with trap = 0 to restore normal operation.  Synchronises on
+ * `stream`.  `workspace` must be 8-byte aligned. */
+PSA_API psa_status_t psa_debug_wait_control(void* workspace, uint64_t limit_ns, int32_t trap, void* stream);
 
 /* Message of the last failed call on this thread ("" if none). */
 PSA_API const char* psa_last_error(void);

@@ -180,7 +180,7 @@ def test_binding_refuses_cpu_tensors():
         P.psa_build_pyramid(s, k, k, None, None)
 
 
-def test_debug_wait_limit_rejects_null_and_misaligned():
-    assert P.lib().psa_debug_set_wait_limit(None, 5, None) == P.PSA_ERR_INVALID_ARG
-    assert P.lib().psa_debug_set_wait_limit(ctypes.c_void_p(0x1003), 5, None) == P.PSA_ERR_INVALID_ARG
+def test_debug_wait_control_rejects_null_and_misaligned():
+    assert P.lib().psa_debug_wait_control(None, 5, 1, None) == P.PSA_ERR_INVALID_ARG
+    assert P.lib().psa_debug_wait_control(ctypes.c_void_p(0x1003), 5, 0, None) == P.PSA_ERR_INVALID_ARG
     assert "workspace" in P.psa_last_error()

@@ -3,11 +3,11 @@
   * More than 1024 KV blocks: the mask generator's CTA-wide select kernel
     (the warp kernel holds at most 1024 keys per row), with both level
     policies and causal masking, and attention on the resulting mask.
-  * A bounded device wait that runs out: with the protocol wait limit of
-    the attention kernel set to 1 ns the kernel gives up, reports
-    PSA_ERR_TIMEOUT with the site of the wait through
-    psa_get_device_status, and a normal call on the same workspace
-    afterwards is correct.
+  * A bounded device wait that runs out: with the debug trap armed, every
+    CTA of the attention kernel waits once on a barrier nothing arrives at
+    (limit 1 ms), gives up, unwinds, and PSA_ERR_TIMEOUT with that wait's
+    site comes back through psa_get_device_status; a normal call on the
+    same workspace afterwards is correct.
 """
 import re
 
@@ -24,8 +24,7 @@ from psa_run import SKIP, attn_errors, levels_of, run_attention, run_mask, run_p
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
-# wait sites of the attention kernel (producer 11-15, MMA issuer 21-26, softmax 31-35)
-ATTN_SITES = {11, 12, 13, 14, 15, 21, 22, 23, 24, 26, 31, 32, 33, 35}
+TRAP_SITE = 10          # the attention kernel's debug trap wait
 
 
 @pytest.mark.parametrize("policy,causal", [("mass", False), ("quantile", True)])
@@ -96,7 +95,7 @@ def test_attention_wait_timeout_is_reported_and_recoverable():
     kp, vp, _ = run_pyramid(shape, k, v)
     ws = P.workspace(P.psa_attention_workspace_bytes(shape), DEV)
     out = torch.empty_like(q)
-    P.psa_debug_set_wait_limit(ws, 1)
+    P.psa_debug_wait_control(ws, 1000000, trap=True)
     P.psa_attention_fwd(shape, q, k, v, kp, vp, mask, shape.d ** -0.5, out, None, ws)
     st = P.psa_get_device_status(ws)
     msg = P.psa_last_error()
@@ -104,12 +103,12 @@ def test_attention_wait_timeout_is_reported_and_recoverable():
     m = re.search(r"site (\d+), block (\d+), thread (\d+)", msg)
     assert m, msg
     site, blk, thr = (int(x) for x in m.groups())
-    assert site in ATTN_SITES, msg
+    assert site == TRAP_SITE, msg
     assert 0 <= blk < 2 * torch.cuda.get_device_properties(0).multi_processor_count
     assert 0 <= thr < 192
-    # the record was read and cleared; the limit stays until reset
+    # the record was read and cleared; the debug words stay until reset
     assert P.psa_get_device_status(ws) == P.PSA_OK
-    P.psa_debug_set_wait_limit(ws, 0)
+    P.psa_debug_wait_control(ws, 0, trap=False)
     out2, lse2, _ = run_attention(shape, q, k, v, kp, vp, mask, shape.d ** -0.5, ws=ws)
     torch.cuda.synchronize()
     ws2 = P.workspace(P.psa_attention_workspace_bytes(shape), DEV)

@@ -29,7 +29,7 @@ EXPORTS = [
     "psa_pyramid_bytes", "psa_pyramid_level_offset", "psa_build_pyramid",
     "psa_mask_workspace_bytes", "psa_make_mask",
     "psa_attention_workspace_bytes", "psa_attention_fwd", "psa_attention_fwd_static", "psa_attention_plan_stats",
-    "psa_get_device_status", "psa_get_static_device_status", "psa_debug_set_wait_limit",
+    "psa_get_device_status", "psa_get_static_device_status", "psa_debug_wait_control",
     "psa_last_error", "psa_version",
 ]
 
@@ -72,7 +72,7 @@ def _load(path: str = LIB_PATH):
         "psa_attention_plan_stats": (I, [S, P, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64), P]),
         "psa_get_device_status": (I, [P, P]),
         "psa_get_static_device_status": (I, [P]),
-        "psa_debug_set_wait_limit": (I, [P, ctypes.c_uint64, P]),
+        "psa_debug_wait_control": (I, [P, ctypes.c_uint64, I, P]),
         "psa_last_error": (ctypes.c_char_p, []),
         "psa_version": (I, []),
     }
@@ -208,8 +208,9 @@ def psa_get_static_device_status(stream=None) -> int:
     return lib().psa_get_static_device_status(_stream(stream))
 
 
-def psa_debug_set_wait_limit(workspace, limit_ns: int, stream=None):
-    _check(lib().psa_debug_set_wait_limit(_ptr(workspace, "workspace"), ctypes.c_uint64(limit_ns), _stream(stream)))
+def psa_debug_wait_control(workspace, limit_ns: int, trap: bool = False, stream=None):
+    _check(lib().psa_debug_wait_control(_ptr(workspace, "workspace"), ctypes.c_uint64(limit_ns), int(bool(trap)),
+                                        _stream(stream)))
 
 
 # ------------------------------------------------------------------------- buffers

@@ -278,12 +278,13 @@ AttnLayout attn_layout(const psa_shape_t* s) {
   return L;
 }
 
-// Byte offset, inside every workspace header, of the 64-bit protocol wait
-// limit read by the attention kernel (0 = the built-in limit).
+// Byte offset, inside every workspace header, of the debug words read by the
+// attention kernel: the 64-bit limit of its debug trap wait (0 = the
+// built-in limit) at 40, the trap flag at 48.
 constexpr size_t kWaitLimitOffset = 40;
 
 // Reads the status word and time-out record at the start of a workspace
-// header, clears them (36 bytes: the wait limit after them is kept), and
+// header, clears them (36 bytes: the debug words after them are kept), and
 // turns them into a status and message.
 psa_status_t read_status(void* hdr, void* stream) {
   int w[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
@@ -530,14 +531,19 @@ psa_status_t psa_get_device_status(void* ws, void* stream) {
   return read_status(ws, stream);
 }
 
-psa_status_t psa_debug_set_wait_limit(void* ws, uint64_t limit_ns, void* stream) {
+psa_status_t psa_debug_wait_control(void* ws, uint64_t limit_ns, int32_t trap, void* stream) {
   g_err[0] = 0;
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 7u)) return fail(PSA_ERR_INVALID_ARG, "workspace is NULL or misaligned");
+  struct {
+    unsigned long long limit;
+    int trap;
+    int pad;
+  } v = {limit_ns, trap ? 1 : 0, 0};
+  static_assert(sizeof(v) == 16, "debug words");
   cudaStream_t str = static_cast<cudaStream_t>(stream);
-  const unsigned long long v = limit_ns;
   PSA_CUDA(cudaMemcpyAsync(static_cast<char*>(ws) + kWaitLimitOffset, &v, sizeof(v), cudaMemcpyHostToDevice, str),
-           "wait limit copy");
-  PSA_CUDA(cudaStreamSynchronize(str), "wait limit sync");
+           "debug word copy");
+  PSA_CUDA(cudaStreamSynchronize(str), "debug word sync");
   return PSA_OK;
 }
 

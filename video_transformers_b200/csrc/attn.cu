@@ -72,6 +72,7 @@ struct AttnShared {
   uint64_t i_full[NST], i_empty[NST];
   uint64_t s_full[2], p_full[2];
   uint64_t o_ready, o_final, o_free, drain;
+  uint64_t never;       // no thread ever arrives here (the debug trap of the time-out path)
   uint32_t tmem_base;
   int abort;
   SubInfo ti[NST];
@@ -174,6 +175,7 @@ __global__ void __launch_bounds__(kThreads, CTAS)
     mbar_init(smem_u32(&sh->o_final), 1);
     mbar_init(smem_u32(&sh->o_free), 128);
     mbar_init(smem_u32(&sh->drain), 1);
+    mbar_init(smem_u32(&sh->never), 1);
     sh->abort = 0;
     fence_mbar_init();
   }
@@ -184,7 +186,6 @@ __global__ void __launch_bounds__(kThreads, CTAS)
   const uint32_t tmem = sh->tmem_base;
   const uint32_t tO = tmem + 128;
   volatile int* abort = &sh->abort;
-  const uint64_t wlim = protocol_wait_limit(a.status);
 
   if (warp == 0) {
     // =============================== producer ===============================
@@ -193,6 +194,7 @@ __global__ void __launch_bounds__(kThreads, CTAS)
     }
     uint32_t it = 0, qcnt = 0;       // it: sub-tiles loaded so far
     uint32_t kiss = 0, viss = 0;     // K and V sub-tile loads issued (the drain waits for exactly these)
+    bool trap = debug_wait_trap(a.status);
     bool ok = true;
     for (int idx = blockIdx.x; idx < a.n_items && ok; idx += gridDim.x) {
       const int item = a.queue[idx];
@@ -203,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, CTAS)
       const int b = bh / a.Hq, h = bh - b * a.Hq;
       const int hkv = b * a.Hkv + h / (a.Hq / a.Hkv);
       const int q0 = tq * 128;
-      if (!warp_wait(smem_u32(&sh->q_empty), (qcnt & 1) ^ 1, abort, a.status, 11, idx, qcnt, it, 0, wlim)) { ok = false; break; }
+      if (!warp_wait(smem_u32(&sh->q_empty), (qcnt & 1) ^ 1, abort, a.status, 11, idx, qcnt, it, 0)) { ok = false; break; }
       if (lane == 0) {
         const uint32_t bar = smem_u32(&sh->q_full);
         mbar_arrive_expect_tx(bar, QB);
@@ -250,7 +252,7 @@ __global__ void __launch_bounds__(kThreads, CTAS)
         const uint32_t ph = (it / NST) & 1;
 
         // K
-        if (!warp_wait(smem_u32(&sh->k_empty[st]), ph ^ 1, abort, a.status, 12, idx, j, it, 0, wlim)) { ok = false; break; }
+        if (!warp_wait(smem_u32(&sh->k_empty[st]), ph ^ 1, abort, a.status, 12, idx, j, it, 0)) { ok = false; break; }
         if (lane == 0) mbar_arrive_expect_tx(smem_u32(&sh->k_full[st]), SB);
         __syncwarp();
         if (mine) {
@@ -260,9 +262,19 @@ __global__ void __launch_bounds__(kThreads, CTAS)
                         kc * 64, prow, hkv);
         }
         ++kiss;
+        if (trap) {
+          // debug trap: with a K load in flight, wait on a barrier no thread
+          // arrives at, so that the wait runs out (after the debug limit,
+          // long before any other wait could) and the CTA unwinds
+          trap = false;
+          if (!warp_wait(smem_u32(&sh->never), 0, abort, a.status, 10, idx, j, it, 0, debug_trap_limit(a.status))) {
+            ok = false;
+            break;
+          }
+        }
 
         // sub-tile record
-        if (!warp_wait(smem_u32(&sh->i_empty[st]), ph ^ 1, abort, a.status, 13, idx, j, it, 0, wlim)) { ok = false; break; }
+        if (!warp_wait(smem_u32(&sh->i_empty[st]), ph ^ 1, abort, a.status, 13, idx, j, it, 0)) { ok = false; break; }
         SubInfo& ti = sh->ti[st];
         const int p_last = J * rows + lo + cnt;                // one past the last pooled row used here
         const int last_tok = (p_last << l) - 1;                // last token covered
@@ -319,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, CTAS)
         // V of the previous sub-tile
         if (j > 0) {
           const uint32_t pst = (it - 1) % NST;
-          if (!warp_wait(smem_u32(&sh->v_empty[pst]), (((it - 1) / NST) & 1) ^ 1, abort, a.status, 14, idx, j, it, 0, wlim)) { ok = false; break; }
+          if (!warp_wait(smem_u32(&sh->v_empty[pst]), (((it - 1) / NST) & 1) ^ 1, abort, a.status, 14, idx, j, it, 0)) { ok = false; break; }
           if (lane == 0) mbar_arrive_expect_tx(smem_u32(&sh->v_full[pst]), SB);
           __syncwarp();
           if (pv_mine) {
@@ -335,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, CTAS)
       // V of the item's last sub-tile
       if (ok) {
         const uint32_t pst = (it - 1) % NST;
-        if (!warp_wait(smem_u32(&sh->v_empty[pst]), (((it - 1) / NST) & 1) ^ 1, abort, a.status, 15, idx, 0, it, 0, wlim)) { ok = false; break; }
+        if (!warp_wait(smem_u32(&sh->v_empty[pst]), (((it - 1) / NST) & 1) ^ 1, abort, a.status, 15, idx, 0, it, 0)) { ok = false; break; }
         if (lane == 0) mbar_arrive_expect_tx(smem_u32(&sh->v_full[pst]), SB);
         __syncwarp();
         if (pv_mine) {
@@ -375,10 +387,10 @@ __global__ void __launch_bounds__(kThreads, CTAS)
       auto issue_pv = [&](uint32_t jj, bool first_of_item) -> bool {
         const uint32_t g = it + jj, st = g % NST, sb2 = g & 1;
         if (first_of_item && icnt > 0) {
-          if (!bounded_wait(smem_u32(&sh->o_free), (icnt - 1) & 1, abort, a.status, 21, icnt, jj, g, 0, wlim)) return false;
+          if (!bounded_wait(smem_u32(&sh->o_free), (icnt - 1) & 1, abort, a.status, 21, icnt, jj, g, 0)) return false;
         }
-        if (!bounded_wait(smem_u32(&sh->p_full[sb2]), (g >> 1) & 1, abort, a.status, 22, icnt, jj, g, 0, wlim)) return false;
-        if (!bounded_wait(smem_u32(&sh->v_full[st]), (g / NST) & 1, abort, a.status, 26, icnt, jj, g, 0, wlim)) return false;
+        if (!bounded_wait(smem_u32(&sh->p_full[sb2]), (g >> 1) & 1, abort, a.status, 22, icnt, jj, g, 0)) return false;
+        if (!bounded_wait(smem_u32(&sh->v_full[st]), (g / NST) & 1, abort, a.status, 26, icnt, jj, g, 0)) return false;
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < kSub / 16; ++k) {
@@ -394,13 +406,13 @@ __global__ void __launch_bounds__(kThreads, CTAS)
         const int t0 = a.item_tile_off[item], t1 = a.item_tile_off[item + 1];
         if (t1 == t0) continue;
         const uint32_t n = sub_count(a.item_rows[item]);
-        if (!bounded_wait(smem_u32(&sh->q_full), qcnt & 1, abort, a.status, 23, idx, qcnt, it, 0, wlim)) { ok = false; break; }
+        if (!bounded_wait(smem_u32(&sh->q_full), qcnt & 1, abort, a.status, 23, idx, qcnt, it, 0)) { ok = false; break; }
         tc_fence_after();
         ++qcnt;
         for (uint32_t j = 0; j < n && ok; ++j) {
           const uint32_t g = it + j, st = g % NST, sb2 = g & 1;
           // S_j = Q K_j^T into S buffer sb2
-          if (!bounded_wait(smem_u32(&sh->k_full[st]), (g / NST) & 1, abort, a.status, 24, idx, j, g, 0, wlim)) { ok = false; break; }
+          if (!bounded_wait(smem_u32(&sh->k_full[st]), (g / NST) & 1, abort, a.status, 24, idx, j, g, 0)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int kc = 0; kc < KC; ++kc) {
@@ -455,8 +467,8 @@ __global__ void __launch_bounds__(kThreads, CTAS)
       float m = -CUDART_INF_F, lsum = 0.f;
       for (uint32_t j = 0; j < n; ++j, ++it) {
         const uint32_t st = it % NST, sb2 = it & 1;
-        if (!warp_wait(smem_u32(&sh->s_full[sb2]), (it >> 1) & 1, abort, a.status, 31, idx, j, it, 0, wlim)) { ok = false; break; }
-        if (!warp_wait(smem_u32(&sh->i_full[st]), (it / NST) & 1, abort, a.status, 32, idx, j, it, 0, wlim)) { ok = false; break; }
+        if (!warp_wait(smem_u32(&sh->s_full[sb2]), (it >> 1) & 1, abort, a.status, 31, idx, j, it, 0)) { ok = false; break; }
+        if (!warp_wait(smem_u32(&sh->i_full[st]), (it / NST) & 1, abort, a.status, 32, idx, j, it, 0)) { ok = false; break; }
         tc_fence_after();
         const SubInfo& ti = sh->ti[st];
         uint32_t sr[32], sr2[32];
@@ -533,7 +545,7 @@ __global__ void __launch_bounds__(kThreads, CTAS)
           const float f = grow ? fast_exp2(m - mnew) : 1.0f;
           lsum *= f;
           if (grow) m = mnew;
-          if (!warp_wait(smem_u32(&sh->o_ready), (it - 1) & 1, abort, a.status, 33, idx, j, it, 0, wlim)) { ok = false; break; }
+          if (!warp_wait(smem_u32(&sh->o_ready), (it - 1) & 1, abort, a.status, 33, idx, j, it, 0)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
@@ -559,7 +571,7 @@ __global__ void __launch_bounds__(kThreads, CTAS)
       // epilogue: O / l once the item's last PV is done (o_final completes
       // once per item and cannot run ahead: the next item's first PV waits
       // for o_free)
-      if (!warp_wait(smem_u32(&sh->o_final), icnt & 1, abort, a.status, 35, idx, n, it, icnt, wlim)) { ok = false; break; }
+      if (!warp_wait(smem_u32(&sh->o_final), icnt & 1, abort, a.status, 35, idx, n, it, icnt)) { ok = false; break; }
       ++icnt;
       tc_fence_after();
       const float inv = lsum > 0.f ? 1.0f / lsum : 0.f;

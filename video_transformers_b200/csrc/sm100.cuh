@@ -96,11 +96,15 @@ __device__ __forceinline__ bool bounded_wait(uint32_t bar, uint32_t parity, vola
   }
 }
 
-// Limit of the protocol waits of a kernel whose workspace header starts at
-// `status`: the 64-bit value at byte 40 of the header when it is non-zero
-// (set by psa_debug_set_wait_limit), else kWaitLimitNs.  Drain waits never
-// use it.
-__device__ __forceinline__ uint64_t protocol_wait_limit(const int* status) {
+// Debug trap of the time-out path, armed through the workspace header by
+// psa_debug_wait_control: the 32-bit word at byte 48 (non-zero: the kernel
+// waits once on a barrier that nothing arrives at) and the 64-bit limit of
+// that one wait at byte 40 (0: kWaitLimitNs).  Every other wait keeps
+// kWaitLimitNs.
+__device__ __forceinline__ bool debug_wait_trap(const int* status) {
+  return *reinterpret_cast<const volatile int*>(status + 12) != 0;
+}
+__device__ __forceinline__ uint64_t debug_trap_limit(const int* status) {
   const uint64_t v = *reinterpret_cast<const volatile unsigned long long*>(status + 10);
   return v ? v : kWaitLimitNs;
 }
