@@ -14,6 +14,8 @@
  *                       its KV blocks, each read at its assigned level with a
  *                       +ln(2^l) logit bias
  *
+ * and the gradients of the last step, psa_attention_bwd.
+ *
  * Conventions shared by every entry point
  * ---------------------------------------
  *  - Tensors are contiguous row-major [B, H, N, d] in device memory, owned by
@@ -189,6 +191,38 @@ PSA_API psa_status_t psa_attention_fwd(const psa_shape_t* shape, const void* q, 
                                const void* k_pyr, const void* v_pyr, const uint8_t* mask,
                                float sm_scale, void* out, float* lse,
                                void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Backward pass of stage 3 (the pages give none; news review, Methodology
+ * 4, says the model trains end to end through the pooled attention, and the
+ * summary article, Results, pairs PSA with distillation).  The derivative
+ * of psa_attention_fwd's definition with the mask held fixed: with
+ * P = exp(z - lse) over the row's key set, dP = dO . V^l[p], D = dO . O and
+ * dZ = P (dP - D),
+ *   dq_i = sm_scale sum_p dZ_ip K^l[p],
+ *   dK^l[p] = sm_scale sum_i dZ_ip q_i,   dV^l[p] = sum_i P_ip dO_i,
+ * and through the pooling (level l token t is the mean of input tokens
+ * t 2^l .. t 2^l + 2^l - 1):  dk[t] = sum_l dK^l[t >> l] / 2^l, same for v.
+ *
+ * Inputs: the forward's q, k, v, pyramid buffers, mask and sm_scale, its
+ * output `out` and its lse (both required), and dout = dL/dout; all
+ * [B, H, N, d] bf16 except lse (fp32 [B, Hq, N]).  Outputs dq [B, Hq, N, d],
+ * dk and dv [B, Hkv, N, d], bf16, fully overwritten (rows with no visible
+ * key get dq = 0; KV tokens no query uses get 0).  Products are bf16 with
+ * fp32 accumulation; P and dZ are rounded to bf16 before their products,
+ * dK^l and dV^l are summed in fp32 before the pooling backward.  bf16
+ * tensors only (fp32 shapes: PSA_ERR_UNSUPPORTED).  The workspace (size
+ * from psa_attention_bwd_workspace_bytes) holds the forward's tile plan,
+ * the transposed plan of the dK / dV kernel and the fp32 level gradients;
+ * like every workspace it is zero-filled once before first use and carries
+ * the status word read by psa_get_device_status.
+ * ------------------------------------------------------------------------ */
+PSA_API size_t psa_attention_bwd_workspace_bytes(const psa_shape_t* shape);
+PSA_API psa_status_t psa_attention_bwd(const psa_shape_t* shape, const void* q, const void* k, const void* v,
+                                       const void* k_pyr, const void* v_pyr, const uint8_t* mask,
+                                       float sm_scale, const void* out, const float* lse, const void* dout,
+                                       void* dq, void* dk, void* dv,
+                                       void* workspace, size_t workspace_bytes, void* stream);
 
 /* psa_attention_fwd without a workspace argument, for callers that cannot
  * allocate device memory themselves: for example a plugin inside a host

@@ -29,6 +29,7 @@ EXPORTS = [
     "psa_pyramid_bytes", "psa_pyramid_level_offset", "psa_build_pyramid",
     "psa_mask_workspace_bytes", "psa_make_mask",
     "psa_attention_workspace_bytes", "psa_attention_fwd", "psa_attention_fwd_static", "psa_attention_plan_stats",
+    "psa_attention_bwd_workspace_bytes", "psa_attention_bwd",
     "psa_get_device_status", "psa_get_static_device_status", "psa_debug_wait_control",
     "psa_last_error", "psa_version",
 ]
@@ -69,6 +70,8 @@ def _load(path: str = LIB_PATH):
         "psa_attention_workspace_bytes": (Z, [S]),
         "psa_attention_fwd": (I, [S, P, P, P, P, P, P, F, P, P, P, Z, P]),
         "psa_attention_fwd_static": (I, [S, P, P, P, P, P, P, F, P, P, P]),
+        "psa_attention_bwd_workspace_bytes": (Z, [S]),
+        "psa_attention_bwd": (I, [S, P, P, P, P, P, P, F, P, P, P, P, P, P, P, Z, P]),
         "psa_attention_plan_stats": (I, [S, P, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64), P]),
         "psa_get_device_status": (I, [P, P]),
         "psa_get_static_device_status": (I, [P]),
@@ -191,6 +194,20 @@ def psa_attention_fwd_static(shape: Shape, q, k, v, k_pyr, v_pyr, mask, sm_scale
                                           _ptr(k_pyr, "k_pyr", L1), _ptr(v_pyr, "v_pyr", L1), _ptr(mask, "mask"),
                                           ctypes.c_float(sm_scale), _ptr(out, "out"), _ptr(lse, "lse", False),
                                           _stream(stream)))
+
+
+def psa_attention_bwd_workspace_bytes(shape: Shape) -> int:
+    return lib().psa_attention_bwd_workspace_bytes(ctypes.byref(shape))
+
+
+def psa_attention_bwd(shape: Shape, q, k, v, k_pyr, v_pyr, mask, sm_scale: float, out, lse, dout, dq, dk, dv,
+                      workspace, stream=None):
+    L1 = shape.levels > 1
+    _check(lib().psa_attention_bwd(ctypes.byref(shape), _ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"),
+                                   _ptr(k_pyr, "k_pyr", L1), _ptr(v_pyr, "v_pyr", L1), _ptr(mask, "mask"),
+                                   ctypes.c_float(sm_scale), _ptr(out, "out"), _ptr(lse, "lse"), _ptr(dout, "dout"),
+                                   _ptr(dq, "dq"), _ptr(dk, "dk"), _ptr(dv, "dv"), _ptr(workspace, "workspace"),
+                                   ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream)))
 
 
 def psa_attention_plan_stats(shape: Shape, workspace, stream=None):

@@ -18,7 +18,8 @@ OBJ = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libpsa.so")
 ROOT = os.path.dirname(HERE)
 
-SOURCES = ["api.cu", "pyramid.cu", "mask.cu", "meankey.cu", "plan.cu", "attn.cu"]
+SOURCES = ["api.cu", "pyramid.cu", "mask.cu", "meankey.cu", "plan.cu", "attn.cu", "attn_dq.cu", "attn_dkv.cu",
+           "attn_bwd.cu"]
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-lineinfo", "-O3", "-std=c++17",
@@ -37,7 +38,7 @@ def nvcc() -> str:
 
 def _deps(src: str):
     deps = [src]
-    for h in ("internal.h", "sm100.cuh", "exp2_poly.h"):
+    for h in ("internal.h", "sm100.cuh", "exp2_poly.h", "attn_common.cuh"):
         deps.append(os.path.join(CSRC, h))
     deps.append(os.path.join(ROOT, "include", "psa.h"))
     return deps

@@ -298,6 +298,45 @@ psa_status_t read_status(void* hdr, void* stream) {
               w[0], w[2], w[3], w[4], w[5], w[6], w[7], w[8]);
 }
 
+// ------------------------------------------------------------------ backward workspace
+struct BwdLayout {
+  AttnLayout fwd;                  // the forward's tile plan, at the start of the workspace
+  size_t lse2p, dp, tcnt, toff, eqt, emask, dkl, dvl, total;
+  int n_titems, level_base[5], level_tiles[4];
+  int64_t max_entries, level_off[4];
+};
+BwdLayout bwd_layout(const psa_shape_t* s) {
+  BwdLayout L{};
+  L.fwd = attn_layout(s);
+  size_t off = L.fwd.total;
+  const size_t BHq = static_cast<size_t>(s->B) * s->Hq;
+  const int64_t BHkv = static_cast<int64_t>(s->B) * s->Hkv;
+  const size_t padded = BHq * static_cast<size_t>(L.fwd.n_qtiles) * 128;
+  L.lse2p = off; off = align_up(off + padded * 4, 256);
+  L.dp = off;    off = align_up(off + padded * 4, 256);
+  int n = 0;
+  int64_t elems = 0;
+  for (int l = 0; l < s->levels; ++l) {
+    L.level_base[l] = n;
+    L.level_tiles[l] = static_cast<int>(ceil_div(s->N >> l, 128));
+    n += static_cast<int>(BHkv * L.level_tiles[l]);
+    L.level_off[l] = elems;
+    elems += BHkv * (s->N >> l) * s->d;
+  }
+  for (int l = s->levels; l < 4; ++l) { L.level_tiles[l] = 0; L.level_off[l] = 0; }
+  L.level_base[s->levels] = n;
+  L.n_titems = n;
+  L.max_entries = static_cast<int64_t>(n) * (s->Hq / s->Hkv) * L.fwd.n_qtiles;
+  L.tcnt = off;  off = align_up(off + static_cast<size_t>(n) * 4, 256);
+  L.toff = off;  off = align_up(off + static_cast<size_t>(n + 1) * 4, 256);
+  L.eqt = off;   off = align_up(off + static_cast<size_t>(L.max_entries) * 4, 256);
+  L.emask = off; off = align_up(off + static_cast<size_t>(L.max_entries) * 4, 256);
+  L.dkl = off;   off = align_up(off + static_cast<size_t>(elems) * 4, 256);
+  L.dvl = off;   off = align_up(off + static_cast<size_t>(elems) * 4, 256);
+  L.total = off;
+  return L;
+}
+
 }  // namespace
 
 extern "C" {
@@ -507,6 +546,132 @@ psa_status_t psa_attention_fwd(const psa_shape_t* s, const void* q, const void* 
   aa.lse = lse;
   aa.status = reinterpret_cast<int*>(w + L.status);
   PSA_CUDA(psa::launch_attention(maps, aa, num_sms(), st), "attention launch");
+  return PSA_OK;
+}
+
+size_t psa_attention_bwd_workspace_bytes(const psa_shape_t* s) {
+  if (check_shape(s) != PSA_OK || s->dtype != PSA_DT_BF16) return 0;
+  return bwd_layout(s).total;
+}
+
+psa_status_t psa_attention_bwd(const psa_shape_t* s, const void* q, const void* k, const void* v, const void* k_pyr,
+                               const void* v_pyr, const uint8_t* mask, float sm_scale, const void* out,
+                               const float* lse, const void* dout, void* dq, void* dk, void* dv, void* ws,
+                               size_t ws_bytes, void* stream) {
+  g_err[0] = 0;
+  PSA_TRY(check_shape(s));
+  if (s->dtype != PSA_DT_BF16) return fail(PSA_ERR_UNSUPPORTED, "the backward pass takes bf16 tensors only");
+  PSA_TRY(check_ptr(q, "q"));
+  PSA_TRY(check_ptr(k, "k"));
+  PSA_TRY(check_ptr(v, "v"));
+  if (s->levels > 1) {
+    PSA_TRY(check_ptr(k_pyr, "k_pyr"));
+    PSA_TRY(check_ptr(v_pyr, "v_pyr"));
+  }
+  if (!mask) return fail(PSA_ERR_INVALID_ARG, "mask is NULL");
+  PSA_TRY(check_ptr(out, "out"));
+  PSA_TRY(check_ptr(lse, "lse"));
+  PSA_TRY(check_ptr(dout, "dout"));
+  PSA_TRY(check_ptr(dq, "dq"));
+  PSA_TRY(check_ptr(dk, "dk"));
+  PSA_TRY(check_ptr(dv, "dv"));
+  if (!(sm_scale > 0.f) || sm_scale != sm_scale) return fail(PSA_ERR_INVALID_ARG, "sm_scale must be > 0");
+  const BwdLayout L = bwd_layout(s);
+  if (L.fwd.max_segs >= (1ll << 31) || L.fwd.max_tiles >= (1ll << 31) || L.max_entries >= (1ll << 31))
+    return fail(PSA_ERR_UNSUPPORTED, "tile plan would exceed 2^31 entries");
+  if (!ws || !aligned16(ws)) return fail(PSA_ERR_WORKSPACE, "workspace is NULL or not 16-byte aligned");
+  if (ws_bytes < L.total) return fail(PSA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, L.total);
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  const int64_t BHq = static_cast<int64_t>(s->B) * s->Hq, BHkv = static_cast<int64_t>(s->B) * s->Hkv;
+  const char* kp = static_cast<const char*>(k_pyr);
+  const char* vp = static_cast<const char*>(v_pyr);
+  // tensor maps: Q and dO in 128-row boxes; K / V levels in the forward's
+  // segment boxes (dQ kernel) and in 128-row boxes (dK / dV kernel)
+  CUtensorMap mq[10], mkv[10];
+  PSA_TRY(map3(&mq[0], q, BHq, s->N, s->d, 128));
+  PSA_TRY(map3(&mq[1], dout, BHq, s->N, s->d, 128));
+  mkv[0] = mq[0];
+  mkv[1] = mq[1];
+  for (int l = 0; l < s->levels; ++l) {
+    const void* kb = l == 0 ? k : static_cast<const void*>(kp + pyr_level_offset(s, l, 2));
+    const void* vb = l == 0 ? v : static_cast<const void*>(vp + pyr_level_offset(s, l, 2));
+    const int box = (s->block >> l) < 64 ? (s->block >> l) : 64;
+    PSA_TRY(map3(&mq[2 + l], kb, BHkv, s->N >> l, s->d, box));
+    PSA_TRY(map3(&mq[2 + s->levels + l], vb, BHkv, s->N >> l, s->d, box));
+    PSA_TRY(map3(&mkv[2 + l], kb, BHkv, s->N >> l, s->d, 128));
+    PSA_TRY(map3(&mkv[2 + s->levels + l], vb, BHkv, s->N >> l, s->d, 128));
+  }
+  const int nkb = static_cast<int>(ceil_div(s->N, s->block));
+  // 1. the forward's tile plan (dQ walks it)
+  psa::PlanArgs pa{};
+  pa.B = s->B; pa.Hq = s->Hq; pa.N = s->N; pa.block = s->block; pa.nqb = nkb; pa.nkb = nkb;
+  pa.levels = s->levels; pa.causal = s->causal != 0; pa.n_items = L.fwd.n_items; pa.mask = mask;
+  pa.item_nseg = reinterpret_cast<int*>(w + L.fwd.nseg);
+  pa.item_ntile = reinterpret_cast<int*>(w + L.fwd.ntile);
+  pa.item_rows = reinterpret_cast<int*>(w + L.fwd.nrows);
+  pa.item_seg_off = reinterpret_cast<int*>(w + L.fwd.seg_off);
+  pa.item_tile_off = reinterpret_cast<int*>(w + L.fwd.tile_off);
+  pa.tile_seg_off = reinterpret_cast<int*>(w + L.fwd.tile_seg_off);
+  pa.segs = reinterpret_cast<int*>(w + L.fwd.segs);
+  pa.queue = reinterpret_cast<int*>(w + L.fwd.queue);
+  pa.hist = reinterpret_cast<int*>(w + L.fwd.hist);
+  pa.n_hist = L.fwd.n_hist;
+  pa.lpt_queue = 0;
+  pa.stats = reinterpret_cast<long long*>(w + L.fwd.stats);
+  PSA_CUDA(psa::launch_plan(pa, st), "plan launch");
+  // 2. D = dO . O and lse in log2 units, padded
+  float* lse2p = reinterpret_cast<float*>(w + L.lse2p);
+  float* dpad = reinterpret_cast<float*>(w + L.dp);
+  PSA_CUDA(psa::launch_bwd_prep(out, dout, lse, lse2p, dpad, BHq, s->N, s->d, L.fwd.n_qtiles, st), "prep launch");
+  // 3. dQ
+  psa::DqArgs qa{};
+  qa.B = s->B; qa.Hq = s->Hq; qa.Hkv = s->Hkv; qa.N = s->N; qa.d = s->d; qa.block = s->block;
+  qa.levels = s->levels; qa.causal = s->causal != 0; qa.n_items = L.fwd.n_items; qa.n_qtiles = L.fwd.n_qtiles;
+  qa.scale_log2 = sm_scale * 1.4426950408889634f;
+  qa.sm_scale = sm_scale;
+  qa.item_tile_off = pa.item_tile_off;
+  qa.item_rows = pa.item_rows;
+  qa.tile_seg_off = pa.tile_seg_off;
+  qa.segs = pa.segs;
+  qa.queue = pa.queue;
+  qa.lse2p = lse2p;
+  qa.dp = dpad;
+  qa.dq = dq;
+  qa.status = reinterpret_cast<int*>(w + L.fwd.status);
+  PSA_CUDA(psa::launch_dq(mq, qa, num_sms(), st), "dq launch");
+  // 4. transposed plan, 5. dK^l / dV^l
+  psa::TPlanArgs ta{};
+  ta.B = s->B; ta.Hq = s->Hq; ta.Hkv = s->Hkv; ta.N = s->N; ta.block = s->block; ta.nqb = nkb; ta.nkb = nkb;
+  ta.levels = s->levels; ta.causal = s->causal != 0; ta.n_qtiles = L.fwd.n_qtiles; ta.n_items = L.n_titems;
+  for (int l = 0; l < 5; ++l) ta.level_base[l] = l <= s->levels ? L.level_base[l] : L.n_titems;
+  for (int l = 0; l < 4; ++l) ta.level_tiles[l] = L.level_tiles[l];
+  ta.mask = mask;
+  ta.item_cnt = reinterpret_cast<int*>(w + L.tcnt);
+  ta.item_off = reinterpret_cast<int*>(w + L.toff);
+  ta.entry_qt = reinterpret_cast<int*>(w + L.eqt);
+  ta.entry_mask = reinterpret_cast<unsigned*>(w + L.emask);
+  PSA_CUDA(psa::launch_tplan(ta, st), "transposed plan launch");
+  psa::DkvArgs ka{};
+  ka.B = s->B; ka.Hq = s->Hq; ka.Hkv = s->Hkv; ka.N = s->N; ka.d = s->d; ka.block = s->block;
+  ka.levels = s->levels; ka.causal = s->causal != 0; ka.n_qtiles = L.fwd.n_qtiles; ka.n_items = L.n_titems;
+  for (int l = 0; l < 5; ++l) ka.level_base[l] = ta.level_base[l];
+  for (int l = 0; l < 4; ++l) { ka.level_tiles[l] = L.level_tiles[l]; ka.level_off[l] = L.level_off[l]; }
+  ka.scale_log2 = sm_scale * 1.4426950408889634f;
+  ka.sm_scale = sm_scale;
+  ka.item_off = ta.item_off;
+  ka.entry_qt = ta.entry_qt;
+  ka.entry_mask = ta.entry_mask;
+  ka.lse2p = lse2p;
+  ka.dp = dpad;
+  ka.dkl = reinterpret_cast<float*>(w + L.dkl);
+  ka.dvl = reinterpret_cast<float*>(w + L.dvl);
+  ka.status = reinterpret_cast<int*>(w + L.fwd.status);
+  PSA_CUDA(psa::launch_dkv(mkv, ka, num_sms(), st), "dkv launch");
+  // 6. through the pooling of every level
+  PSA_CUDA(psa::launch_pool_bwd(ka.dkl, L.level_off, dk, BHkv, s->N, s->d, s->levels, st), "pool backward (K)");
+  PSA_CUDA(psa::launch_pool_bwd(ka.dvl, L.level_off, dv, BHkv, s->N, s->d, s->levels, st), "pool backward (V)");
   return PSA_OK;
 }
 

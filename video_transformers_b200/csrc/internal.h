@@ -127,6 +127,77 @@ struct AttnArgs {
 cudaError_t launch_attention(const CUtensorMap* maps, const AttnArgs& a, int num_sms,
                              cudaStream_t s);
 
+// ---- stage 3, backward ----------------------------------------------------
+// D_i = dO_i . O_i and lse_i * log2(e) per query row, written into arrays
+// padded to whole 128-row query tiles ([B*Hq][n_qtiles*128]); padding rows
+// get lse2 = +inf (so their probabilities are exactly 0) and D = 0.
+cudaError_t launch_bwd_prep(const void* out, const void* dout, const float* lse, float* lse2p, float* dp,
+                            int64_t BHq, int N, int d, int n_qtiles, cudaStream_t s);
+
+struct DqArgs {
+  int B, Hq, Hkv, N, d, block, levels, causal;
+  int n_items, n_qtiles;
+  float scale_log2;       // sm_scale * log2(e)
+  float sm_scale;
+  const int* item_tile_off;
+  const int* item_rows;
+  const int* tile_seg_off;
+  const int* segs;
+  const int* queue;
+  const float* lse2p;     // padded [B*Hq][n_qtiles*128]
+  const float* dp;        // padded D
+  void* dq;               // [B,Hq,N,d] bf16
+  int* status;
+};
+// maps: [0] = Q, [1] = dO (3D [d, N, B*Hq], box 64 x 128), [2 + l] = K level l,
+// [2 + L + l] = V level l (box 64 x min(block/2^l, 64)).
+cudaError_t launch_dq(const CUtensorMap* maps, const DqArgs& a, int num_sms, cudaStream_t s);
+
+// Transposed plan of the dK/dV kernel.  A work item is a 128-row tile of one
+// pyramid level of one KV head: pooled rows [128 t, 128 t + 128) of level l,
+// i.e. 128 / (block >> l) consecutive KV blocks.  Its entries are the query
+// tiles (query head of the KV head's group, 128-row query tile) for which
+// some block of the tile holds level l; each entry carries a bit mask, bit
+// 2 jb + hf = block jb of the tile is at level l for query half hf (for
+// 128-token blocks both half bits are equal).
+struct TPlanArgs {
+  int B, Hq, Hkv, N, block, nqb, nkb, levels, causal, n_qtiles;
+  int n_items;
+  int level_base[5];      // first item of level l; level_base[levels] = n_items
+  int level_tiles[4];     // tiles per KV head at level l
+  const uint8_t* mask;
+  int* item_cnt;          // [n_items]
+  int* item_off;          // [n_items + 1]
+  int* entry_qt;          // [max entries]  h_local * n_qtiles + tq
+  unsigned* entry_mask;   // [max entries]
+};
+cudaError_t launch_tplan(const TPlanArgs& a, cudaStream_t s);
+
+struct DkvArgs {
+  int B, Hq, Hkv, N, d, block, levels, causal, n_qtiles;
+  int n_items;
+  int level_base[5];
+  int level_tiles[4];
+  float scale_log2, sm_scale;
+  const int* item_off;
+  const int* entry_qt;
+  const unsigned* entry_mask;
+  const float* lse2p;
+  const float* dp;
+  float* dkl;             // fp32 level gradients, level l at dkl + level_off[l] (elements)
+  float* dvl;
+  int64_t level_off[4];   // element offset of level l ([B*Hkv][N >> l][d])
+  int* status;
+};
+// maps: [0] = Q, [1] = dO (box 64 x 128), [2 + l] = K level l, [2 + L + l] =
+// V level l (box 64 x 128 rows).
+cudaError_t launch_dkv(const CUtensorMap* maps, const DkvArgs& a, int num_sms, cudaStream_t s);
+
+// dK[t] = dK^0[t] + sum_{l >= 1} dK^l[t >> l] / 2^l (same for V), fp32 level
+// gradients -> bf16 output [B*Hkv][N][d].
+cudaError_t launch_pool_bwd(const float* gl, const int64_t* level_off, void* out, int64_t BHkv, int N, int d,
+                            int levels, cudaStream_t s);
+
 // Segment word of the tile plan: bits [0,2) level, [2,4) half mask (bit 0:
 // query rows 0..63 of the tile use it, bit 1: rows 64..127; 0 marks a
 // padding segment of zeros), [4,32) KV block index.
