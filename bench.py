@@ -411,10 +411,58 @@ def run_psa(args, rank, world, local_rank):
         line["mask_roofline"] = mr
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"], line["parity"] = cpu_baseline(w, q, k, v, path, args)
+    if not args.no_backward:
+        line["backward"] = measure_backward(path, w, stream, flops, pk)
     if rank == 0 and world == 1 and not args.no_configs:
         m["steps"] = args.steps
         line["configs"] = run_configs(args, w, path, m, clocks, pk, dev, stream)
     return line
+
+
+def measure_backward(path, w, stream, flops_fwd, peaks_, reps=3):
+    """psa_attention_bwd at the same workload and mask: the forward's output
+    and lse, a random upstream gradient, then `reps` timed calls.  Its
+    throughput counts 2.5x the forward's executed FLOPs (the five GEMMs of
+    the forward's shape in the gradient: S, dP, dV, dK and dQ), the usual
+    convention; the kernels execute more (S and dP are recomputed by the
+    dQ and the dK/dV kernels, and the dK/dV tiles are level-homogeneous
+    128-row tiles whose rows a query tile may not use)."""
+    P = path.P
+    if w.dtype != "bf16":
+        return None
+    dev = path.q.device
+    lse = torch.empty(path.q.shape[:3], dtype=torch.float32, device=dev)
+    P.psa_attention_fwd(path.shape, path.q, path.k, path.v, path.kp, path.vp, path.mask, w.sm_scale, path.out, lse,
+                        path.aws)
+    g = torch.Generator(device=dev)
+    g.manual_seed(1234)
+    dout = torch.randn(path.q.shape, generator=g, device=dev, dtype=torch.float32).to(path.q.dtype)
+    dq, dk, dv = torch.empty_like(path.q), torch.empty_like(path.k), torch.empty_like(path.v)
+    ws = P.workspace(P.psa_attention_bwd_workspace_bytes(path.shape), dev)
+
+    def call():
+        P.psa_attention_bwd(path.shape, path.q, path.k, path.v, path.kp, path.vp, path.mask, w.sm_scale, path.out,
+                            lse, dout, dq, dk, dv, ws)
+    call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    st = P.psa_get_device_status(ws)
+    if st != P.PSA_OK:
+        raise RuntimeError("device status %d after the backward: %s" % (st, P.psa_last_error()))
+    ms = e0.elapsed_time(e1) / reps
+    bf16_burst, bf16_sus = peaks_[0], peaks_[1]
+    tf = 2.5 * flops_fwd / (ms * 1e-3) / 1e12
+    del dq, dk, dv, ws, dout, lse
+    torch.cuda.empty_cache()
+    return {"entry_point": "psa_attention_bwd", "ms": ms, "reps": reps, "tflops": tf,
+            "flop_convention": "2.5 x the forward's executed FLOPs", "frac_of_sustained": tf / bf16_sus,
+            "frac_of_burst": tf / bf16_burst,
+            "kernels": "plan (3) + prep + dq_kernel + tplan (3) + dkv_kernel + pool_bwd (2) = 11 launches"}
 
 
 def launches_per_step(w):
@@ -636,6 +684,7 @@ def main():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-preset records of the default line")
+    ap.add_argument("--no-backward", action="store_true", help="skip the timing of psa_attention_bwd")
     ap.add_argument("--config-steps", type=int, default=10, help="timed steps per preset in the configs record")
     ap.add_argument("--config-parity-blocks", type=int, default=8,
                     help="query blocks of one head per preset checked against the oracle")

@@ -9,6 +9,7 @@ prints them at the end (tests/conftest.py)."""
 from __future__ import annotations
 
 COUNTS = []          # (test label, flagged pairs, compared pairs)
+NOTES = []           # free-form lines printed at the end of the session (measured error ratios)
 MAX_FRACTION = 1e-3
 
 
@@ -17,3 +18,7 @@ def check_band(label: str, n_flagged: int, n_pairs: int, max_fraction: float = M
     assert n_pairs > 0, label
     assert n_flagged <= max_fraction * n_pairs, \
         "%s: %d of %d pairs in the ambiguity band (> %.2g)" % (label, n_flagged, n_pairs, max_fraction)
+
+
+def note(line: str):
+    NOTES.append(line)

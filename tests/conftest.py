@@ -24,6 +24,10 @@ def pytest_terminal_summary(terminalreporter):
         import amb_report
     except ImportError:
         return
+    if amb_report.NOTES:
+        terminalreporter.write_sep("-", "measured errors")
+        for line in amb_report.NOTES:
+            terminalreporter.write_line(line)
     if not amb_report.COUNTS:
         return
     tot_f = sum(c[1] for c in amb_report.COUNTS)

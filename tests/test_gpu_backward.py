@@ -17,6 +17,7 @@ import torch
 import oracle.psa_oracle as O
 import video_transformers_b200 as P
 import workloads as W
+from amb_report import note
 from psa_run import SKIP, params_for, run_attention, run_mask, run_pyramid, shape_for
 
 pytestmark = pytest.mark.gpu
@@ -48,6 +49,8 @@ def compare(name, got, ref):
     err = np.abs(g - ref)
     mx, mean = err.max(), err.mean()
     scale_mx, scale_mean = np.abs(ref).max(), np.abs(ref).mean()
+    note("backward %s: max-abs %.3g (%.4f of max|ref| %.3g), mean-abs %.3g (%.4f of mean|ref| %.3g)"
+         % (name, mx, mx / scale_mx, scale_mx, mean, mean / scale_mean, scale_mean))
     assert mx <= REL_MAX * scale_mx and mean <= REL_MEAN * scale_mean, \
         (name, mx, mean, scale_mx, scale_mean, mx / scale_mx, mean / scale_mean)
     return mx / scale_mx, mean / scale_mean
