@@ -3,12 +3,13 @@ oracle's attention_backward, which is pinned by torch autograd, finite
 differences and the dense special case (tests/test_oracle_pins.py).
 
 Tolerance, per gradient (dq, dk, dv) against the fp64 oracle on the same
-bf16 inputs: max-abs error <= 2e-2 * max|ref| and mean-abs error <= 1e-2 *
+bf16 inputs: max-abs error <= 2e-2 * max|ref| and mean-abs error <= 6e-3 *
 mean|ref|.  The GPU rounds P and dZ to bf16 (relative 2^-9) before their
 products, reads the bf16 pyramid levels (the oracle pools in fp64) and the
 bf16 forward output in D = dO.O, and rounds the result to bf16 (alone a
-mean error of about 0.15 % of mean|ref| on these inputs); the bounds leave
-a margin of several times those terms.  Rows and tokens that nothing
+mean error of about 0.15 % of mean|ref| on these inputs).  Measured on
+B200 over the cases below: at most 1.07 % of max|ref| and 0.30 % of
+mean|ref|, so the bounds leave a margin of about 2x.  Rows and tokens that nothing
 reaches must come back as exact zeros."""
 import numpy as np
 import pytest
@@ -22,7 +23,7 @@ from psa_run import SKIP, params_for, run_attention, run_mask, run_pyramid, shap
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
-REL_MAX, REL_MEAN = 2e-2, 1e-2
+REL_MAX, REL_MEAN = 2e-2, 6e-3
 
 
 def gen(seed):
