@@ -17,11 +17,13 @@
 //               dV += P^T dO_hf and dK += dS^T Q_hf with A read from TMEM
 //               (M 128, N = d).  Half hf of an entry is accumulated before
 //               the next entry's S^T of the same half is issued.
-//   warps 2..5  one KV row per thread: p = 2^(s * sm_scale * log2 e + l -
-//               lse2[q]) (0 when the row's block is not at level l for this
-//               query half, or the pooled token is after the query under
-//               causal masking), ds = p (dp - D[q]); then the epilogue
-//               writes the item's dK^l (times sm_scale) and dV^l rows in fp32.
+//   warps 2..9  two warps per KV row quarter, each on 32 of a half's 64
+//               query columns: p = 2^(s * sm_scale * log2 e + l - lse2[q])
+//               (0 when the row's block is not at level l for this query
+//               half, or the pooled token is after the query under causal
+//               masking), ds = p (dp - D[q]); then the epilogue writes the
+//               item's dV^l (warps 2..5) and dK^l times sm_scale (warps
+//               6..9) rows in fp32.
 // TMEM (512 columns): S^T halves at [0, 64) and [64, 128), dP^T halves at
 // [128, 256), dV at [256, 256 + d), dK at [256 + d, 256 + 2 d).
 // Every wait is bounded; a time-out sets the workspace status word.
@@ -34,7 +36,9 @@
 namespace psa {
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kSoftWarps = 8;                       // two per TMEM lane quarter
+constexpr int kSoftThreads = 32 * kSoftWarps;
+constexpr int kThreads = 64 + kSoftThreads;
 
 struct DkvMaps {
   CUtensorMap m[10];
@@ -84,10 +88,10 @@ __global__ void __launch_bounds__(kThreads, 1) dkv_kernel(const __grid_constant_
       mbar_init(smem_u32(&sh->q_full[i]), 1);
       mbar_init(smem_u32(&sh->q_empty[i]), 1);
       mbar_init(smem_u32(&sh->s_full[i]), 1);
-      mbar_init(smem_u32(&sh->p_full[i]), 128);
+      mbar_init(smem_u32(&sh->p_full[i]), kSoftThreads);
     }
     mbar_init(smem_u32(&sh->acc_full), 1);
-    mbar_init(smem_u32(&sh->acc_free), 128);
+    mbar_init(smem_u32(&sh->acc_free), kSoftThreads);
     mbar_init(smem_u32(&sh->drain), 1);
     sh->abort = 0;
     fence_mbar_init();
@@ -219,6 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1) dkv_kernel(const __grid_constant_
   } else {
     // =============================== softmax / epilogue ===============================
     const int q = warp & 3;
+    const int cg = (warp - 2) >> 2;                       // 32-column group of each half
     const int r = q * 32 + lane;                          // KV row of the tile
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     uint32_t kcnt = 0, g = 0;
@@ -235,11 +240,12 @@ __global__ void __launch_bounds__(kThreads, 1) dkv_kernel(const __grid_constant_
       const int last_tok = ((p + 1) << l) - 1;            // last token the pooled row averages
       const float bias = static_cast<float>(l);           // ln 2^l in log2 units
       const int64_t orow = a.level_off[l] + (static_cast<int64_t>(b * a.Hkv + hkv) * Nl + p) * D;
+      float* gout = cg == 0 ? a.dvl : a.dkl;
+      const float oscale = cg == 0 ? 1.0f : a.sm_scale;
       if (ne == 0) {
         if (row_in) {
-          float4* dk4 = reinterpret_cast<float4*>(a.dkl + orow);
-          float4* dv4 = reinterpret_cast<float4*>(a.dvl + orow);
-          for (int c = 0; c < D / 4; ++c) { dk4[c] = make_float4(0.f, 0.f, 0.f, 0.f); dv4[c] = make_float4(0.f, 0.f, 0.f, 0.f); }
+          float4* o4 = reinterpret_cast<float4*>(gout + orow);
+          for (int c = 0; c < D / 4; ++c) o4[c] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
         continue;
       }
@@ -251,61 +257,59 @@ __global__ void __launch_bounds__(kThreads, 1) dkv_kernel(const __grid_constant_
         for (int hf = 0; hf < 2; ++hf) {
           if (!warp_wait(smem_u32(&sh->s_full[hf]), g & 1, abort, a.status, 61, idx, e, g, hf)) { ok = false; break; }
           tc_fence_after();
-          uint32_t sr[32], sr2[32], dr[32], dr2[32];
-          tmem_ld32(tS + hf * 64 + lane_off, sr);
-          tmem_ld32(tS + hf * 64 + 32 + lane_off, sr2);
-          tmem_ld32(tP + hf * 64 + lane_off, dr);
-          tmem_ld32(tP + hf * 64 + 32 + lane_off, dr2);
+          uint32_t sr[32], dr[32];
+          tmem_ld32(tS + hf * 64 + cg * 32 + lane_off, sr);
+          tmem_ld32(tP + hf * 64 + cg * 32 + lane_off, dr);
           const bool valid = row_in && ((bits >> (2 * jb + hf)) & 1u);
-          const int q_first = tq * 128 + hf * 64;         // token of column 0 of this half
-          const bool edge = a.causal && last_tok > q_first;
+          const int q_first = tq * 128 + hf * 64 + cg * 32;   // token of this thread's column 0
+          // column c (query token q_first + c) sees the pooled row iff the
+          // row is valid and, under causal masking, last_tok <= q_first + c:
+          // the hidden columns are exactly c < cut
+          const int cut = !valid ? 32 : (a.causal ? max(0, min(32, last_tok - q_first)) : 0);
           const float sc = a.scale_log2;
-          const float* lz = &sh->lse2[st][hf * 64];
-          const float* dz = &sh->dd[st][hf * 64];
-          uint32_t pk[32], gk[32];
+          const float4* lz4 = reinterpret_cast<const float4*>(&sh->lse2[st][hf * 64 + cg * 32]);
+          const float4* dz4 = reinterpret_cast<const float4*>(&sh->dd[st][hf * 64 + cg * 32]);
+          uint32_t pk[16], gk[16];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            float pv[2], gv[2];
+          for (int i4 = 0; i4 < 8; ++i4) {
+            const float4 lv = lz4[i4], dv = dz4[i4];
+            const float lz[4] = {lv.x, lv.y, lv.z, lv.w}, dz[4] = {dv.x, dv.y, dv.z, dv.w};
+            float pv[4], gv[4];
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int c = 2 * i + u;
-              const float s = __uint_as_float(c < 32 ? sr[c] : sr2[c - 32]);
-              const float dpv = __uint_as_float(c < 32 ? dr[c] : dr2[c - 32]);
-              float x = fmaf(s, sc, bias - lz[c]);
-              if (!valid || (edge && last_tok > q_first + c)) x = -CUDART_INF_F;
+            for (int u = 0; u < 4; ++u) {
+              const int c = 4 * i4 + u;
+              const float x = c < cut ? -CUDART_INF_F : fmaf(__uint_as_float(sr[c]), sc, bias - lz[u]);
               pv[u] = fast_exp2(x);
-              gv[u] = pv[u] * (dpv - dz[c]);
+              gv[u] = pv[u] * (__uint_as_float(dr[c]) - dz[u]);
             }
-            pk[i] = pack_bf16(pv[0], pv[1]);
-            gk[i] = pack_bf16(gv[0], gv[1]);
+            pk[2 * i4] = pack_bf16(pv[0], pv[1]);
+            pk[2 * i4 + 1] = pack_bf16(pv[2], pv[3]);
+            gk[2 * i4] = pack_bf16(gv[0], gv[1]);
+            gk[2 * i4 + 1] = pack_bf16(gv[2], gv[3]);
           }
-          tmem_st32(tS + hf * 64 + lane_off, pk);
-          tmem_st32(tP + hf * 64 + lane_off, gk);
+          tmem_st16(tS + hf * 64 + cg * 16 + lane_off, pk);
+          tmem_st16(tP + hf * 64 + cg * 16 + lane_off, gk);
           tmem_st_wait();
           tc_fence_before();
           mbar_arrive(smem_u32(&sh->p_full[hf]));
         }
       }
       if (!ok) break;
-      // epilogue: the item's dK^l, dV^l rows
+      // epilogue: warps of column group 0 write dV^l, group 1 dK^l (times sm_scale)
       if (!warp_wait(smem_u32(&sh->acc_full), kcnt & 1, abort, a.status, 62, idx, kcnt, 0, 0)) { ok = false; break; }
       ++kcnt;
       tc_fence_after();
+      const uint32_t tacc = cg == 0 ? tV : tK;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
-        uint32_t v[32], k[32];
-        tmem_ld32(tV + c * 32 + lane_off, v);
-        tmem_ld32(tK + c * 32 + lane_off, k);
+        uint32_t v[32];
+        tmem_ld32(tacc + c * 32 + lane_off, v);
         if (row_in) {
-          float4* dv4 = reinterpret_cast<float4*>(a.dvl + orow + c * 32);
-          float4* dk4 = reinterpret_cast<float4*>(a.dkl + orow + c * 32);
+          float4* o4 = reinterpret_cast<float4*>(gout + orow + c * 32);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            dv4[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                 __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
-            dk4[i] = make_float4(__uint_as_float(k[4 * i]) * a.sm_scale, __uint_as_float(k[4 * i + 1]) * a.sm_scale,
-                                 __uint_as_float(k[4 * i + 2]) * a.sm_scale, __uint_as_float(k[4 * i + 3]) * a.sm_scale);
-          }
+          for (int i = 0; i < 8; ++i)
+            o4[i] = make_float4(__uint_as_float(v[4 * i]) * oscale, __uint_as_float(v[4 * i + 1]) * oscale,
+                                __uint_as_float(v[4 * i + 2]) * oscale, __uint_as_float(v[4 * i + 3]) * oscale);
         }
       }
       tc_fence_before();

@@ -17,8 +17,9 @@
 //               with dS read from TMEM (A) and K from shared memory (B,
 //               MN-major), so S_{j+1} / dP_{j+1} run while the softmax
 //               warpgroup works on sub-tile j.
-//   warps 2..5  one query row per thread: p and ds, ds as bf16 into the S
-//               buffer; the epilogue writes dQ * sm_scale.
+//   warps 2..9  two warps per query row quarter, each on 32 of a sub-tile's
+//               64 columns: p and ds, ds as bf16 into the S buffer; the
+//               epilogue writes dQ * sm_scale, each warp half of the row.
 // TMEM (512 columns): S at [0, 128), dP at [128, 256), dQ at [256, 256 + d).
 // Every wait is bounded; a time-out sets the workspace status word.
 #include <cuda_bf16.h>
@@ -31,7 +32,9 @@
 namespace psa {
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kSoftWarps = 8;                       // two per TMEM lane quarter
+constexpr int kSoftThreads = 32 * kSoftWarps;
+constexpr int kThreads = 64 + kSoftThreads;
 constexpr int kSub = kSubRows;
 
 struct DqMaps {
@@ -77,14 +80,14 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
       mbar_init(smem_u32(&sh->kv_full[i]), 1);
       mbar_init(smem_u32(&sh->kv_empty[i]), 1);
       mbar_init(smem_u32(&sh->i_full[i]), 32);
-      mbar_init(smem_u32(&sh->i_empty[i]), 128);
+      mbar_init(smem_u32(&sh->i_empty[i]), kSoftThreads);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&sh->s_full[i]), 1);
-      mbar_init(smem_u32(&sh->ds_full[i]), 128);
+      mbar_init(smem_u32(&sh->ds_full[i]), kSoftThreads);
     }
     mbar_init(smem_u32(&sh->o_final), 1);
-    mbar_init(smem_u32(&sh->o_free), 128);
+    mbar_init(smem_u32(&sh->o_free), kSoftThreads);
     mbar_init(smem_u32(&sh->drain), 1);
     sh->abort = 0;
     fence_mbar_init();
@@ -245,9 +248,11 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
   } else {
     // =============================== softmax / epilogue ===============================
     const int q = warp & 3;
+    const int cg = (warp - 2) >> 2;                       // 32-column group of each sub-tile
     const int row = q * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     const int my_half = H2 ? (row >> 6) : 0;
+    constexpr int DH = D / 2;                             // dQ columns this warp writes
     uint32_t it = 0, icnt = 0;
     bool ok = true;
     for (int idx = blockIdx.x; idx < a.n_items && ok; idx += gridDim.x) {
@@ -256,11 +261,11 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
       const int bh = item / a.n_qtiles, tq = item - bh * a.n_qtiles;
       const int tok = tq * 128 + row;
       const int64_t orow = static_cast<int64_t>(bh) * a.N + tok;
-      __nv_bfloat16* dq = static_cast<__nv_bfloat16*>(a.dq);
+      __nv_bfloat16* dq = static_cast<__nv_bfloat16*>(a.dq) + orow * D + cg * DH;
       if (t1 == t0) {
         if (tok < a.N) {
-          uint4* o = reinterpret_cast<uint4*>(dq + orow * D);
-          for (int c = 0; c < D / 8; ++c) o[c] = make_uint4(0u, 0u, 0u, 0u);
+          uint4* o = reinterpret_cast<uint4*>(dq);
+          for (int c = 0; c < DH / 8; ++c) o[c] = make_uint4(0u, 0u, 0u, 0u);
         }
         continue;
       }
@@ -274,53 +279,43 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
         if (!warp_wait(smem_u32(&sh->i_full[st]), (it / NST) & 1, abort, a.status, 92, idx, j, it, 0)) { ok = false; break; }
         tc_fence_after();
         const SubInfo& ti = sh->ti[st];
-        uint32_t sr[32], sr2[32], dr[32], dr2[32];
-        tmem_ld32(tS + sb2 * kSub + lane_off, sr);
-        tmem_ld32(tS + sb2 * kSub + 32 + lane_off, sr2);
-        tmem_ld32(tP + sb2 * kSub + lane_off, dr);
-        tmem_ld32(tP + sb2 * kSub + 32 + lane_off, dr2);
+        uint32_t sr[32], dr[32];
+        tmem_ld32(tS + sb2 * kSub + cg * 32 + lane_off, sr);
+        tmem_ld32(tP + sb2 * kSub + cg * 32 + lane_off, dr);
         // exp2 argument of every column: s * sc + level - lse2 (or -inf)
-        float x[kSub];
+        float x[32];
         const float sc = a.scale_log2;
         if (ti.fast) {
-          const float4 c4 = *reinterpret_cast<const float4*>(ti.cb[my_half]);
-          const float cb[4] = {c4.x - lse2, c4.y - lse2, c4.z - lse2, c4.w - lse2};
+          const float cb0 = ti.cb[my_half][2 * cg] - lse2, cb1 = ti.cb[my_half][2 * cg + 1] - lse2;
 #pragma unroll
-          for (int c = 0; c < kSub; ++c)
-            x[c] = fmaf(__uint_as_float(c < 32 ? sr[c] : sr2[c - 32]), sc, cb[c >> 4]);
+          for (int c = 0; c < 32; ++c) x[c] = fmaf(__uint_as_float(sr[c]), sc, c < 16 ? cb0 : cb1);
         } else {
 #pragma unroll
-          for (int c4 = 0; c4 < kSub / 4; ++c4) {
-            const float4 bv = *reinterpret_cast<const float4*>(&ti.bias[my_half][4 * c4]);
+          for (int c4 = 0; c4 < 8; ++c4) {
+            const float4 bv = *reinterpret_cast<const float4*>(&ti.bias[my_half][32 * cg + 4 * c4]);
             const float bb[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int c = 4 * c4 + u;
-              x[c] = fmaf(__uint_as_float(c < 32 ? sr[c] : sr2[c - 32]), sc, bb[u] - lse2);
-            }
+            for (int u = 0; u < 4; ++u) x[4 * c4 + u] = fmaf(__uint_as_float(sr[4 * c4 + u]), sc, bb[u] - lse2);
           }
           if (ti.causal_check) {
 #pragma unroll
-            for (int c4 = 0; c4 < kSub / 4; ++c4) {
-              const int4 iv = *reinterpret_cast<const int4*>(&ti.info[4 * c4]);
+            for (int c4 = 0; c4 < 8; ++c4) {
+              const int4 iv = *reinterpret_cast<const int4*>(&ti.info[32 * cg + 4 * c4]);
               const int ii[4] = {iv.x, iv.y, iv.z, iv.w};
 #pragma unroll
-              for (int u = 0; u < 4; ++u)
-                if (ii[u] > tok) x[4 * c4 + u] = -CUDART_INF_F;
+              for (int u = 0; u < 4; ++u) x[4 * c4 + u] = ii[u] > tok ? -CUDART_INF_F : x[4 * c4 + u];
             }
           }
         }
         mbar_arrive(smem_u32(&sh->i_empty[st]));
-        uint32_t pk[32];
+        uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
+        for (int i = 0; i < 16; ++i) {
           const int c = 2 * i;
           const float p0 = fast_exp2(x[c]), p1 = fast_exp2(x[c + 1]);
-          const float d0 = __uint_as_float(c < 32 ? dr[c] : dr2[c - 32]);
-          const float d1 = __uint_as_float(c + 1 < 32 ? dr[c + 1] : dr2[c + 1 - 32]);
-          pk[i] = pack_bf16(p0 * (d0 - Dv), p1 * (d1 - Dv));
+          pk[i] = pack_bf16(p0 * (__uint_as_float(dr[c]) - Dv), p1 * (__uint_as_float(dr[c + 1]) - Dv));
         }
-        tmem_st32(tS + sb2 * kSub + lane_off, pk);
+        tmem_st16(tS + sb2 * kSub + cg * 16 + lane_off, pk);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(smem_u32(&sh->ds_full[sb2]));
@@ -330,11 +325,11 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
       ++icnt;
       tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < DH / 32; ++c) {
         uint32_t o[32];
-        tmem_ld32(tQ + c * 32 + lane_off, o);
+        tmem_ld32(tQ + cg * DH + c * 32 + lane_off, o);
         if (tok < a.N) {
-          uint4* dst = reinterpret_cast<uint4*>(dq + orow * D + c * 32);
+          uint4* dst = reinterpret_cast<uint4*>(dq + c * 32);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             uint4 v;
