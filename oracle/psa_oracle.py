@@ -61,6 +61,16 @@ reason in the design notes):
   R12 backward pass: the mask (the levels) is a fixed selection and is not
       differentiated; gradients flow through the pooling of each level as a
       mean (1/2^l to each averaged token).
+  R13 FP8 path ([news] Practical Implications mentions mixed FP16/FP8
+      precision and nothing more): the query and key operands of the score
+      product are rounded to e4m3 (3 mantissa bits, largest value 448,
+      nearest value with ties to even, saturating).  Each query row is
+      scaled by 448 / max|q_row|; every key of a KV head, at every pyramid
+      level, by 448 / max|K| over that head's level 0 (a mean is no larger
+      than the largest of its terms, so no level saturates).  Scales and
+      the scaled values are computed in fp32; the score is the product of
+      the e4m3 values times both scales.  Values and probabilities stay as
+      in R1-R4.
 
 Pins: every function here is checked by ``tests/test_oracle_pins.py``
 against closed forms, invariants, brute force or an independent library
@@ -421,6 +431,81 @@ def ambiguous_pairs_quantile(mass: np.ndarray, thresholds, levels: int, causal: 
             if len(lev) > 1:
                 amb[b, h, I, J] = True
     return amb
+
+
+# ======================================================================================
+# FP8 (e4m3) query / key operands, reading R13
+# ======================================================================================
+
+E4M3_MAX = 448.0
+
+
+def e4m3_codes(x32) -> np.ndarray:
+    """The e4m3 byte of each fp32 value: nearest e4m3 value, ties to even,
+    saturating at +-448 (the clip; the cast of an in-range value is the
+    library's round-to-nearest-even conversion)."""
+    import torch
+    t = torch.as_tensor(np.clip(np.asarray(x32, dtype=np.float32), -E4M3_MAX, E4M3_MAX))
+    return t.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def e4m3_values(codes) -> np.ndarray:
+    """float64 value of each e4m3 byte."""
+    import torch
+    return torch.as_tensor(np.asarray(codes, dtype=np.uint8)).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def _fp32(x) -> np.ndarray:
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            return x.detach().to("cpu", torch.float32).numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.asarray(x, dtype=np.float32)
+
+
+def _scale_and_inverse(am: np.ndarray):
+    """fp32 dequantization scale max/448 and quantization multiplier 448/max
+    (0 and 0 for an all-zero row or head)."""
+    am = am.astype(np.float32)
+    nz = am > 0
+    inv = np.where(nz, np.float32(E4M3_MAX) / np.where(nz, am, np.float32(1)), np.float32(0)).astype(np.float32)
+    scale = (am / np.float32(E4M3_MAX)).astype(np.float32)
+    return scale, inv
+
+
+def quantize_rows_e4m3(x):
+    """Reading R13 for the query side: x [B, H, N, d] -> (codes uint8
+    [B, H, N, d], scale fp32 [B, H, N]); row value = e4m3 value * scale."""
+    xf = _fp32(x)
+    am = np.abs(xf).max(axis=-1)
+    scale, inv = _scale_and_inverse(am)
+    codes = e4m3_codes((xf * inv[..., None]).astype(np.float32))
+    return codes, scale
+
+
+def quantize_heads_e4m3(levels):
+    """Reading R13 for the key side: levels = [K (level 0), K^1, ...], each
+    [B, H, n_l, d] -> (codes per level, scale fp32 [B, H]) with one scale
+    per head from level 0's largest magnitude."""
+    l0 = _fp32(levels[0])
+    am = np.abs(l0).reshape(l0.shape[0], l0.shape[1], -1).max(axis=-1)
+    scale, inv = _scale_and_inverse(am)
+    codes = [e4m3_codes((_fp32(x) * inv[:, :, None, None]).astype(np.float32)) for x in levels]
+    return codes, scale
+
+
+def attention_fp8(q, kp, vp, mask, block: int, sm_scale: float, causal: bool, rows=None):
+    """Adaptive pyramid attention (as :func:`attention`) with the query rows
+    and the key levels replaced by their e4m3 values times their scales
+    (reading R13); values, bias and softmax unchanged.  kp / vp: the levels
+    as the attention receives them (level 0 first)."""
+    qc, qs = quantize_rows_e4m3(q)
+    kc, ks = quantize_heads_e4m3(kp)
+    qd = e4m3_values(qc) * qs.astype(np.float64)[..., None]
+    kd = [e4m3_values(c) * ks.astype(np.float64)[:, :, None, None] for c in kc]
+    return attention(qd, kd, [_f64(x) for x in vp], mask, block, sm_scale, causal, rows=rows)
 
 
 # ======================================================================================

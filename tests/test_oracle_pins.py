@@ -33,6 +33,10 @@ something other than itself.
                         equivalence; identical-group invariance; NaN in a
                         skipped block changes nothing; pure-Python brute force
                         over an exhaustive {0,1,2,3,SKIP} mask; empty rows
+  e4m3_codes /         hand-derived e4m3 bytes (ties to even, subnormals,
+  e4m3_values /        saturation); decode of every byte by the format formula;
+  quantize_*_e4m3 /    row and head maxima map to 448, shared level-0 key scale,
+  attention_fp8         half-ulp error bound; e4m3-exact inputs give attention
   attention_backward /  torch autograd through torch avg_pool1d and softmax
   pool_backward         (independent routines), with and without causal
                         masking and GQA; central finite differences; all level
@@ -991,3 +995,107 @@ def test_mutation_antidiag_group_width(monkeypatch):
     assert np.abs(m.sum(axis=-1) - 1).max() < 1e-12          # the invariant alone cannot see it
     with pytest.raises(AssertionError):
         test_antidiag_mass_bruteforce_strided(4, True)
+
+
+# --------------------------------------------------------------------------------------
+# FP8 (e4m3) operands, reading R13
+# --------------------------------------------------------------------------------------
+
+def pin_e4m3_golden(golden_dir, mod=O):
+    g = json.load(open(os.path.join(golden_dir, "e4m3_hand.json")))
+    got = mod.e4m3_codes(np.array([c["x"] for c in g["cases"]], dtype=np.float32))
+    return int((got.astype(np.int64) != np.array([c["code"] for c in g["cases"]])).sum())
+
+
+def test_e4m3_golden(golden_dir):
+    assert pin_e4m3_golden(golden_dir) == 0
+
+
+def test_e4m3_values_decode_by_formula():
+    """Every byte but the two NaN codes decodes to the value the format
+    definition gives (pure-Python decode)."""
+    codes = np.array([c for c in range(256) if c & 0x7F != 0x7F], dtype=np.uint8)
+    got = O.e4m3_values(codes)
+    for c, v in zip(codes.tolist(), got.tolist()):
+        s, e, m = c >> 7, (c >> 3) & 15, c & 7
+        want = (2.0 ** -6) * m / 8 if e == 0 else 2.0 ** (e - 7) * (1 + m / 8)
+        assert v == (-want if s else want), (c, v, want)
+
+
+def test_quantize_rows_e4m3_properties():
+    x = rand(2, 3, 40, 16).astype(np.float32)
+    x[0, 0, 5] = 0.0                                   # an all-zero row
+    codes, scale = O.quantize_rows_e4m3(x)
+    vals = O.e4m3_values(codes)
+    assert np.all(codes[0, 0, 5] == 0) and scale[0, 0, 5] == 0
+    am = np.abs(x).max(axis=-1)
+    nz = am > 0
+    # each row's largest magnitude maps to +-448 exactly
+    assert np.all(np.abs(vals).max(axis=-1)[nz] == 448.0)
+    np.testing.assert_array_equal(scale, (am / np.float32(448)).astype(np.float32))
+    # relative error of every normal-range element: at most half an e4m3 ulp (2^-4)
+    y = x * (np.float32(448) / np.where(nz, am, 1))[..., None]
+    normal = np.abs(y) >= 2.0 ** -6
+    assert np.all(np.abs(vals - y)[normal] <= 2.0 ** -4 * np.abs(y)[normal] + 1e-6)
+
+
+def test_quantize_heads_e4m3_shares_level0_scale():
+    k = rand(1, 2, 64, 8).astype(np.float32)
+    kl, _ = O.build_pyramid(k, k, 4)
+    codes, scale = O.quantize_heads_e4m3(kl)
+    am = np.abs(k).reshape(1, 2, -1).max(axis=-1)
+    np.testing.assert_array_equal(scale, (am / np.float32(448)).astype(np.float32))
+    for lv in range(4):
+        vals = O.e4m3_values(codes[lv])
+        assert np.abs(vals).max() <= 448.0
+    assert np.abs(O.e4m3_values(codes[0])).reshape(1, 2, -1).max(axis=-1).tolist() == [[448.0, 448.0]]
+
+
+def test_attention_fp8_exact_inputs_equal_attention():
+    """Inputs whose scaled values are already e4m3 numbers (every row and
+    head has an element of magnitude 448, all values on the e4m3 grid, so
+    the scale is 1) give exactly the plain attention."""
+    rng = np.random.default_rng(3)
+    grid = O.e4m3_values(np.array([c for c in range(256) if c & 0x7F != 0x7F], dtype=np.uint8))
+    grid = grid[np.abs(grid) <= 64]
+    N, d, blk = 64, 8, 16
+    q = rng.choice(grid, size=(1, 1, N, d))
+    k = rng.choice(grid, size=(1, 1, N, d))
+    q[..., 0] = 448.0
+    k[0, 0, 0, 0] = 448.0
+    v = rng.standard_normal((1, 1, N, d))
+    mask = np.zeros((1, 1, N // blk, N // blk), dtype=np.uint8)
+    scale = 1.0 / 448.0 / 8.0
+    o8, l8 = O.attention_fp8(q, [k], [v], mask, blk, scale, False)
+    o, l = O.attention(q, [k], [v], mask, blk, scale, False)
+    np.testing.assert_array_equal(o8, o)
+    np.testing.assert_array_equal(l8, l)
+
+
+def test_mutation_e4m3_ties_away(monkeypatch, golden_dir):
+    """Rounding ties away from zero instead of to even fails the golden."""
+    def bad(x32):
+        x = np.clip(np.asarray(x32, dtype=np.float64), -448, 448)
+        grid = O.e4m3_values(np.arange(256, dtype=np.uint8))
+        out = []
+        for v in x.ravel():
+            dist = np.abs(grid - v)
+            dist[np.isnan(dist)] = np.inf
+            best = np.flatnonzero(dist == dist.min())
+            out.append(max(best, key=lambda c: abs(grid[c])))
+        return np.array(out, dtype=np.uint8).reshape(x.shape)
+    monkeypatch.setattr(O, "e4m3_codes", bad)
+    assert pin_e4m3_golden(golden_dir, O) > 0
+
+
+def test_mutation_head_scale_per_level(monkeypatch):
+    """A key scale taken per level instead of from level 0 breaks the
+    shared-scale property."""
+    orig = O.quantize_heads_e4m3
+
+    def bad(levels):
+        out = [orig([x]) for x in levels]
+        return [c[0][0] for c in out], out[-1][1]
+    monkeypatch.setattr(O, "quantize_heads_e4m3", bad)
+    with pytest.raises(AssertionError):
+        test_quantize_heads_e4m3_shares_level0_scale()
