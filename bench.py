@@ -411,6 +411,8 @@ def run_psa(args, rank, world, local_rank):
         line["mask_roofline"] = mr
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"], line["parity"] = cpu_baseline(w, q, k, v, path, args)
+    if not args.no_fp8:
+        line["fp8"] = measure_fp8(path, w, stream, flops, pk)
     if not args.no_backward:
         line["backward"] = measure_backward(path, w, stream, flops, pk)
     if rank == 0 and world == 1 and not args.no_configs:
@@ -463,6 +465,43 @@ def measure_backward(path, w, stream, flops_fwd, peaks_, reps=3):
             "flop_convention": "2.5 x the forward's executed FLOPs", "frac_of_sustained": tf / bf16_sus,
             "frac_of_burst": tf / bf16_burst,
             "kernels": "plan (3) + prep + dq_kernel + tplan (3) + dkv_kernel + pool_bwd (2) = 11 launches"}
+
+
+def measure_fp8(path, w, stream, flops_fwd, peaks_, reps=5):
+    """psa_attention_fwd_fp8 (e4m3 Q and K, reading R13) at the same
+    workload and mask, quantization included, and how far its output moves
+    from the bf16 path's."""
+    P = path.P
+    if w.dtype != "bf16" or w.d != 128:
+        return None
+    ws = P.workspace(P.psa_attention_fp8_workspace_bytes(path.shape), path.q.device)
+    out8 = torch.empty_like(path.out)
+
+    def call():
+        P.psa_attention_fwd_fp8(path.shape, path.q, path.k, path.v, path.kp, path.vp, path.mask, w.sm_scale, out8,
+                                None, ws)
+    call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    st = P.psa_get_device_status(ws)
+    if st != P.PSA_OK:
+        raise RuntimeError("device status %d after the FP8 path: %s" % (st, P.psa_last_error()))
+    ms = e0.elapsed_time(e1) / reps
+    path.attention()
+    torch.cuda.synchronize()
+    diff = (out8.float() - path.out.float()).abs()
+    tf = flops_fwd / (ms * 1e-3) / 1e12
+    r = {"entry_point": "psa_attention_fwd_fp8", "ms": ms, "reps": reps, "tflops": tf,
+         "frac_of_burst_bf16": tf / peaks_[0], "includes": "e4m3 quantization of Q and every K level, plan, attention",
+         "vs_bf16_path": {"max_abs": diff.max().item(), "mean_abs": diff.mean().item()}}
+    del ws, out8
+    torch.cuda.empty_cache()
+    return r
 
 
 def launches_per_step(w):
@@ -685,6 +724,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-preset records of the default line")
     ap.add_argument("--no-backward", action="store_true", help="skip the timing of psa_attention_bwd")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the timing of psa_attention_fwd_fp8")
     ap.add_argument("--config-steps", type=int, default=10, help="timed steps per preset in the configs record")
     ap.add_argument("--config-parity-blocks", type=int, default=8,
                     help="query blocks of one head per preset checked against the oracle")

@@ -193,6 +193,37 @@ PSA_API psa_status_t psa_attention_fwd(const psa_shape_t* shape, const void* q, 
                                void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * FP8 path of stage 3 (news review, Practical Implications, mentions mixed
+ * FP16 / FP8 precision and nothing more; the scheme is this library's
+ * reading).  The score product runs on e4m3 operands: each query row is
+ * scaled by 448 / max|q_row| and every key of a KV head, at every pyramid
+ * level, by 448 / max|K| over that head's level 0; scales and scaled
+ * values are fp32, each rounded to the nearest e4m3 value (ties to even,
+ * saturating at +-448).  The score of query i and pooled key p is then
+ * sm_scale * q_scale[i] * k_scale[head] * (q8_i . k8_p) + l ln 2; V, the
+ * probabilities (bf16) and the output (bf16) are as in psa_attention_fwd.
+ * bf16 tensors with d = 128 only (else PSA_ERR_UNSUPPORTED).  The
+ * rounding of Q and K costs accuracy: on the presets' inputs the output
+ * moves by up to about 0.1 (mean about 0.01) from the bf16 path's.
+ *
+ * psa_quantize_qk_fp8: q -> q8 codes [B, Hq, N, d] (one byte each) and
+ * q_scale fp32 [B, Hq, N]; k (level 0) and the levels of k_pyr -> k8
+ * [B, Hkv, N, d] and k8_pyr (levels 1..L-1 back to back, one byte per
+ * element, level l at the element offset psa_pyramid_level_offset gives
+ * divided by 2), and k_scale fp32 [B, Hkv].  psa_attention_fwd_fp8 does
+ * the same into its workspace (psa_attention_fp8_workspace_bytes), then
+ * the attention.
+ * ------------------------------------------------------------------------ */
+PSA_API psa_status_t psa_quantize_qk_fp8(const psa_shape_t* shape, const void* q, const void* k, const void* k_pyr,
+                                         uint8_t* q8, float* q_scale, uint8_t* k8, uint8_t* k8_pyr,
+                                         float* k_scale, void* stream);
+PSA_API size_t psa_attention_fp8_workspace_bytes(const psa_shape_t* shape);
+PSA_API psa_status_t psa_attention_fwd_fp8(const psa_shape_t* shape, const void* q, const void* k, const void* v,
+                                           const void* k_pyr, const void* v_pyr, const uint8_t* mask,
+                                           float sm_scale, void* out, float* lse,
+                                           void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * Backward pass of stage 3 (the pages give none; news review, Methodology
  * 4, says the model trains end to end through the pooled attention, and the
  * summary article, Results, pairs PSA with distillation).  The derivative

@@ -7,6 +7,7 @@ import re
 import subprocess
 
 import pytest
+import torch
 
 import video_transformers_b200 as P
 
@@ -184,3 +185,15 @@ def test_debug_wait_control_rejects_null_and_misaligned():
     assert P.lib().psa_debug_wait_control(None, 5, 1, None) == P.PSA_ERR_INVALID_ARG
     assert P.lib().psa_debug_wait_control(ctypes.c_void_p(0x1003), 5, 0, None) == P.PSA_ERR_INVALID_ARG
     assert "workspace" in P.psa_last_error()
+
+
+def test_fp8_path_rejects_unsupported_shapes():
+    s64 = P.make_shape(1, 2, 2, 256, 64, 64, 4)
+    assert P.psa_attention_fp8_workspace_bytes(s64) == 0
+    x = torch.empty(16, dtype=torch.uint8)
+    st = P.lib().psa_attention_fwd_fp8(ctypes.byref(s64), *([ctypes.c_void_p(16)] * 6), ctypes.c_float(0.1),
+                                       ctypes.c_void_p(16), None, ctypes.c_void_p(16), 1 << 30, None)
+    assert st == P.PSA_ERR_UNSUPPORTED and "128" in P.psa_last_error()
+    sf = P.make_shape(1, 2, 2, 256, 128, 64, 4, dtype=P.PSA_DT_FP32)
+    assert P.psa_attention_fp8_workspace_bytes(sf) == 0
+    assert P.psa_attention_fp8_workspace_bytes(P.make_shape(1, 2, 2, 256, 128, 64, 4)) > 0

@@ -1,0 +1,125 @@
+"""The FP8 path (reading R13) through the C ABI against the oracle.
+
+* psa_quantize_qk_fp8: the e4m3 codes of Q and of every K level, and the
+  fp32 scales, bit for bit equal to the oracle's (an encoding: exact).
+* psa_attention_fwd_fp8: against the oracle's attention on the same e4m3
+  operands (attention_fp8, fed the GPU's pyramid), with the bf16 path's
+  tolerances (max-abs 2e-2, mean-abs 2e-3): the FP8 kernel's own arithmetic
+  is the bf16 kernel's.  The accuracy cost of the rounding itself (against
+  the plain oracle attention) is reported, not bounded."""
+import numpy as np
+import pytest
+import torch
+
+import oracle.psa_oracle as O
+import video_transformers_b200 as P
+import workloads as W
+from amb_report import note
+from psa_run import SKIP, attn_errors, levels_of, params_for, run_mask, run_pyramid, shape_for
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+MAX_ABS, MEAN_ABS = 2e-2, 2e-3
+
+
+def gen(seed):
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    return g
+
+
+def run_fp8(shape, q, k, v, kp, vp, mask, sm_scale):
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    ws = P.workspace(P.psa_attention_fp8_workspace_bytes(shape), q.device)
+    L1 = shape.levels > 1
+    P.psa_attention_fwd_fp8(shape, q, k, v, kp if L1 else None, vp if L1 else None, mask.contiguous(), sm_scale, out,
+                            lse, ws)
+    st = P.psa_get_device_status(ws)
+    assert st == P.PSA_OK, P.psa_last_error()
+    torch.cuda.synchronize()
+    return out, lse
+
+
+@pytest.mark.parametrize("d,L,N", [(128, 4, 1000), (64, 3, 520), (128, 1, 300)])
+def test_quantize_codes_bit_exact(d, L, N):
+    g = gen(5)
+    B, Hq, Hkv = 2, 4, 2
+    q = (torch.randn(B, Hq, N, d, generator=g) * 3).bfloat16().to(DEV)
+    k = torch.randn(B, Hkv, N, d, generator=g).bfloat16().to(DEV)
+    q[0, 1, 7] = 0                                       # an all-zero query row: codes 0, scale 0
+    shape = P.make_shape(B, Hq, Hkv, N, d, 64, L)
+    kp, _, _ = run_pyramid(shape, k, k)
+    q8 = torch.empty(q.shape, dtype=torch.uint8, device=DEV)
+    qs = torch.empty(q.shape[:3], dtype=torch.float32, device=DEV)
+    k8 = torch.empty(k.shape, dtype=torch.uint8, device=DEV)
+    kp8 = torch.empty(max(1, P.psa_pyramid_bytes(shape) // 2), dtype=torch.uint8, device=DEV)
+    ks = torch.empty(B, Hkv, dtype=torch.float32, device=DEV)
+    P.psa_quantize_qk_fp8(shape, q, k, kp if L > 1 else None, q8, qs, k8, kp8 if L > 1 else None, ks)
+    torch.cuda.synchronize()
+    oc, osc = O.quantize_rows_e4m3(q)
+    np.testing.assert_array_equal(q8.cpu().numpy(), oc)
+    np.testing.assert_array_equal(qs.cpu().numpy(), osc)
+    levels = levels_of(shape, kp, k) if L > 1 else [k.double().cpu().numpy()]
+    kc, ksc = O.quantize_heads_e4m3([x.astype(np.float32) for x in levels])
+    np.testing.assert_array_equal(k8.cpu().numpy(), kc[0])
+    np.testing.assert_array_equal(ks.cpu().numpy(), ksc)
+    for l in range(1, L):
+        off = P.psa_pyramid_level_offset(shape, l) // 2
+        n = B * Hkv * (N >> l) * d
+        np.testing.assert_array_equal(kp8[off:off + n].view(B, Hkv, N >> l, d).cpu().numpy(), kc[l])
+
+
+@pytest.mark.parametrize("block,causal,L,N,heads", [
+    (128, False, 4, 1000, (2, 1)),
+    (128, True, 4, 520, (4, 2)),
+    (64, True, 4, 456, (2, 2)),
+    (64, False, 3, 300, (3, 1)),
+    (128, False, 1, 256, (1, 1)),
+])
+def test_fp8_attention_random_masks(block, causal, L, N, heads):
+    g = gen(21)
+    Hq, Hkv = heads
+    d, B = 128, 2
+    q = torch.randn(B, Hq, N, d, generator=g).bfloat16().to(DEV)
+    k = torch.randn(B, Hkv, N, d, generator=g).bfloat16().to(DEV)
+    v = torch.randn(B, Hkv, N, d, generator=g).bfloat16().to(DEV)
+    nb = -(-N // block)
+    m = torch.randint(0, L + 1, (B, Hq, nb, nb), generator=g)
+    mask = torch.where(m == L, torch.full_like(m, SKIP), m).to(torch.uint8)
+    mask[0, 0, 0] = SKIP
+    shape = P.make_shape(B, Hq, Hkv, N, d, block, L, causal)
+    kp, vp, _ = run_pyramid(shape, k, v)
+    out, lse = run_fp8(shape, q, k, v, kp, vp, mask.to(DEV), d ** -0.5)
+    kl = levels_of(shape, kp, k) if L > 1 else [k.double().cpu().numpy()]
+    vl = levels_of(shape, vp, v) if L > 1 else [v.double().cpu().numpy()]
+    o8, l8 = O.attention_fp8(q, [x.astype(np.float32) for x in kl], vl, mask, block, d ** -0.5, causal)
+    mx, mean, _ = attn_errors(out, o8)
+    assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean)
+    lg = lse.cpu().numpy().astype(np.float64)
+    fin = np.isfinite(l8)
+    assert np.all(np.isneginf(lg[~fin])) and np.abs(lg[fin] - l8[fin]).max() <= 2e-2
+    o, _ = O.attention(q, kl, vl, mask, block, d ** -0.5, causal)
+    cmx, cmean, _ = attn_errors(out, o)
+    note("fp8 block %d causal %s: vs the e4m3 oracle max %.2e mean %.2e; cost vs plain attention max %.3f mean %.4f"
+         % (block, causal, mx, mean, cmx, cmean))
+    assert torch.all(out[0, 0, :min(block, N)] == 0)
+
+
+@pytest.mark.parametrize("name,grid,heads", [("wan14b", (4, 12, 16), (2, 2)), ("qwen2.5vl", (6, 8, 16), (7, 1))])
+def test_fp8_attention_generated_masks(name, grid, heads):
+    w = W.reduced(name, grid=grid, heads=heads)
+    q, k, v, _ = W.make_qkv(w, device="cpu")
+    q, k, v = q.to(DEV), k.to(DEV), v.to(DEV)
+    shape = shape_for(w)
+    kp, vp, bc = run_pyramid(shape, k, v, with_cos=w.cos_min > -2)
+    mask, _ = run_mask(shape, params_for(w), q, k, bc)
+    out, lse = run_fp8(shape, q, k, v, kp, vp, mask, w.sm_scale)
+    kl, vl = levels_of(shape, kp, k), levels_of(shape, vp, v)
+    o8, _ = O.attention_fp8(q, [x.astype(np.float32) for x in kl], vl, mask.cpu(), w.block, w.sm_scale, w.causal)
+    mx, mean, _ = attn_errors(out, o8)
+    assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean)
+    o, _ = O.attention(q, kl, vl, mask.cpu(), w.block, w.sm_scale, w.causal)
+    cmx, cmean, _ = attn_errors(out, o)
+    note("fp8 %s: vs the e4m3 oracle max %.2e mean %.2e; cost vs plain attention max %.3f mean %.4f"
+         % (name, mx, mean, cmx, cmean))

@@ -19,7 +19,7 @@ LIB = os.path.join(HERE, "libpsa.so")
 ROOT = os.path.dirname(HERE)
 
 SOURCES = ["api.cu", "pyramid.cu", "mask.cu", "meankey.cu", "plan.cu", "attn.cu", "attn_dq.cu", "attn_dkv.cu",
-           "attn_bwd.cu"]
+           "attn_bwd.cu", "fp8.cu"]
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-lineinfo", "-O3", "-std=c++17",

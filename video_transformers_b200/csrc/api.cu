@@ -83,21 +83,25 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 tensor map over `rank` dims (dims[0] innermost, contiguous), 128-byte
+// Tensor map over `rank` dims (dims[0] innermost, contiguous), 128-byte
 // swizzle, zero fill outside the tensor.
-psa_status_t encode_bf16(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
-                         const uint64_t* strides_bytes, const uint32_t* box) {
+psa_status_t encode_map(CUtensorMap* m, CUtensorMapDataType type, const void* base, int rank, const uint64_t* dims,
+                        const uint64_t* strides_bytes, const uint32_t* box) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(PSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   cuuint64_t gd[5], gs[4];
   cuuint32_t bx[5], es[5];
   for (int i = 0; i < rank; ++i) { gd[i] = dims[i]; bx[i] = box[i]; es[i] = 1; }
   for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), gd, gs, bx, es,
+  CUresult r = fn(m, type, rank, const_cast<void*>(base), gd, gs, bx, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(PSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
   return PSA_OK;
+}
+psa_status_t encode_bf16(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+                         const uint64_t* strides_bytes, const uint32_t* box) {
+  return encode_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, rank, dims, strides_bytes, box);
 }
 
 // [BH, rows, d] bf16 viewed as 3D {d, rows, BH}, box {64, box_rows, 1}
@@ -106,6 +110,15 @@ psa_status_t map3(CUtensorMap* m, const void* base, int64_t BH, int64_t rows, in
   const uint64_t str[2] = {static_cast<uint64_t>(d) * 2, static_cast<uint64_t>(rows) * d * 2};
   const uint32_t box[3] = {64, static_cast<uint32_t>(box_rows), 1};
   return encode_bf16(m, base, 3, dims, str, box);
+}
+
+// [BH, rows, d] e4m3 codes (one byte each) viewed as 3D {d, rows, BH}, box
+// {d, box_rows, 1}; d = 128, so a box row is one 128-byte swizzle atom
+psa_status_t map3_u8(CUtensorMap* m, const void* base, int64_t BH, int64_t rows, int d, int box_rows) {
+  const uint64_t dims[3] = {static_cast<uint64_t>(d), static_cast<uint64_t>(rows), static_cast<uint64_t>(BH)};
+  const uint64_t str[2] = {static_cast<uint64_t>(d), static_cast<uint64_t>(rows) * d};
+  const uint32_t box[3] = {static_cast<uint32_t>(d), static_cast<uint32_t>(box_rows), 1};
+  return encode_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, 3, dims, str, box);
 }
 
 // [BH, N, d] bf16 viewed as 4D {d, step, N/step, BH}, box {64, 1, 128, 1}:
@@ -335,6 +348,32 @@ BwdLayout bwd_layout(const psa_shape_t* s) {
   L.dvl = off;   off = align_up(off + static_cast<size_t>(elems) * 4, 256);
   L.total = off;
   return L;
+}
+
+// ------------------------------------------------------------------ FP8 workspace
+struct Fp8Layout {
+  AttnLayout fwd;                  // the tile plan, at the start of the workspace
+  size_t q8, qs, k8, kp8, ks, total;
+};
+Fp8Layout fp8_layout(const psa_shape_t* s) {
+  Fp8Layout L{};
+  L.fwd = attn_layout(s);
+  size_t off = L.fwd.total;
+  const size_t BHq = static_cast<size_t>(s->B) * s->Hq, BHkv = static_cast<size_t>(s->B) * s->Hkv;
+  L.q8 = off;  off = align_up(off + BHq * s->N * s->d, 256);
+  L.qs = off;  off = align_up(off + BHq * s->N * 4, 256);
+  L.k8 = off;  off = align_up(off + BHkv * s->N * s->d, 256);
+  L.kp8 = off; off = align_up(off + pyr_bytes(s, 1), 256);
+  L.ks = off;  off = align_up(off + BHkv * 4, 256);
+  L.total = off;
+  return L;
+}
+
+psa_status_t check_fp8_shape(const psa_shape_t* s) {
+  PSA_TRY(check_shape(s));
+  if (s->dtype != PSA_DT_BF16) return fail(PSA_ERR_UNSUPPORTED, "the FP8 path takes bf16 tensors");
+  if (s->d != 128) return fail(PSA_ERR_UNSUPPORTED, "the FP8 path is built for head dim 128");
+  return PSA_OK;
 }
 
 }  // namespace
@@ -672,6 +711,114 @@ psa_status_t psa_attention_bwd(const psa_shape_t* s, const void* q, const void* 
   // 6. through the pooling of every level
   PSA_CUDA(psa::launch_pool_bwd(ka.dkl, L.level_off, dk, BHkv, s->N, s->d, s->levels, st), "pool backward (K)");
   PSA_CUDA(psa::launch_pool_bwd(ka.dvl, L.level_off, dv, BHkv, s->N, s->d, s->levels, st), "pool backward (V)");
+  return PSA_OK;
+}
+
+psa_status_t psa_quantize_qk_fp8(const psa_shape_t* s, const void* q, const void* k, const void* k_pyr, uint8_t* q8,
+                                 float* q_scale, uint8_t* k8, uint8_t* k8_pyr, float* k_scale, void* stream) {
+  g_err[0] = 0;
+  PSA_TRY(check_shape(s));
+  if (s->dtype != PSA_DT_BF16) return fail(PSA_ERR_UNSUPPORTED, "the FP8 path takes bf16 tensors");
+  PSA_TRY(check_ptr(q, "q"));
+  PSA_TRY(check_ptr(k, "k"));
+  PSA_TRY(check_ptr(q8, "q8"));
+  PSA_TRY(check_ptr(q_scale, "q_scale"));
+  PSA_TRY(check_ptr(k8, "k8"));
+  PSA_TRY(check_ptr(k_scale, "k_scale"));
+  if (s->levels > 1) {
+    PSA_TRY(check_ptr(k_pyr, "k_pyr"));
+    PSA_TRY(check_ptr(k8_pyr, "k8_pyr"));
+  }
+  size_t off[PSA_MAX_LEVELS] = {0, 0, 0, 0};
+  for (int l = 1; l < s->levels; ++l) off[l] = pyr_level_offset(s, l, 1);
+  const int64_t BHq = static_cast<int64_t>(s->B) * s->Hq, BHkv = static_cast<int64_t>(s->B) * s->Hkv;
+  PSA_CUDA(psa::launch_quantize_qk_fp8(q, k, k_pyr, off, BHq, BHkv, s->N, s->d, s->levels, q8, q_scale, k8, k8_pyr,
+                                       k_scale, static_cast<cudaStream_t>(stream)),
+           "fp8 quantize launch");
+  return PSA_OK;
+}
+
+size_t psa_attention_fp8_workspace_bytes(const psa_shape_t* s) {
+  if (check_shape(s) != PSA_OK || s->dtype != PSA_DT_BF16 || s->d != 128) return 0;
+  return fp8_layout(s).total;
+}
+
+psa_status_t psa_attention_fwd_fp8(const psa_shape_t* s, const void* q, const void* k, const void* v,
+                                   const void* k_pyr, const void* v_pyr, const uint8_t* mask, float sm_scale,
+                                   void* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  g_err[0] = 0;
+  PSA_TRY(check_fp8_shape(s));
+  PSA_TRY(check_ptr(q, "q"));
+  PSA_TRY(check_ptr(k, "k"));
+  PSA_TRY(check_ptr(v, "v"));
+  PSA_TRY(check_ptr(out, "out"));
+  if (s->levels > 1) {
+    PSA_TRY(check_ptr(k_pyr, "k_pyr"));
+    PSA_TRY(check_ptr(v_pyr, "v_pyr"));
+  }
+  if (!mask) return fail(PSA_ERR_INVALID_ARG, "mask is NULL");
+  PSA_TRY(check_ptr(lse, "lse", false));
+  if (!(sm_scale > 0.f) || sm_scale != sm_scale) return fail(PSA_ERR_INVALID_ARG, "sm_scale must be > 0");
+  const Fp8Layout L = fp8_layout(s);
+  if (L.fwd.max_segs >= (1ll << 31) || L.fwd.max_tiles >= (1ll << 31))
+    return fail(PSA_ERR_UNSUPPORTED, "tile plan would exceed 2^31 entries");
+  if (!ws || !aligned16(ws)) return fail(PSA_ERR_WORKSPACE, "workspace is NULL or not 16-byte aligned");
+  if (ws_bytes < L.total) return fail(PSA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, L.total);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  const int64_t BHq = static_cast<int64_t>(s->B) * s->Hq, BHkv = static_cast<int64_t>(s->B) * s->Hkv;
+  uint8_t* q8 = reinterpret_cast<uint8_t*>(w + L.q8);
+  uint8_t* k8 = reinterpret_cast<uint8_t*>(w + L.k8);
+  uint8_t* kp8 = reinterpret_cast<uint8_t*>(w + L.kp8);
+  float* qs = reinterpret_cast<float*>(w + L.qs);
+  float* ks = reinterpret_cast<float*>(w + L.ks);
+  size_t off[PSA_MAX_LEVELS] = {0, 0, 0, 0};
+  for (int l = 1; l < s->levels; ++l) off[l] = pyr_level_offset(s, l, 1);
+  PSA_CUDA(psa::launch_quantize_qk_fp8(q, k, k_pyr, off, BHq, BHkv, s->N, s->d, s->levels, q8, qs, k8, kp8, ks, st),
+           "fp8 quantize launch");
+  CUtensorMap maps[9];
+  PSA_TRY(map3_u8(&maps[0], q8, BHq, s->N, s->d, 128));
+  const char* vp = static_cast<const char*>(v_pyr);
+  for (int l = 0; l < s->levels; ++l) {
+    const void* kb = l == 0 ? static_cast<const void*>(k8) : static_cast<const void*>(kp8 + off[l]);
+    const void* vb = l == 0 ? v : static_cast<const void*>(vp + pyr_level_offset(s, l, 2));
+    const int box = (s->block >> l) < 64 ? (s->block >> l) : 64;
+    PSA_TRY(map3_u8(&maps[1 + l], kb, BHkv, s->N >> l, s->d, box));
+    PSA_TRY(map3(&maps[1 + s->levels + l], vb, BHkv, s->N >> l, s->d, box));
+  }
+  const int nkb = static_cast<int>(ceil_div(s->N, s->block));
+  psa::PlanArgs pa{};
+  pa.B = s->B; pa.Hq = s->Hq; pa.N = s->N; pa.block = s->block; pa.nqb = nkb; pa.nkb = nkb;
+  pa.levels = s->levels; pa.causal = s->causal != 0; pa.n_items = L.fwd.n_items; pa.mask = mask;
+  pa.item_nseg = reinterpret_cast<int*>(w + L.fwd.nseg);
+  pa.item_ntile = reinterpret_cast<int*>(w + L.fwd.ntile);
+  pa.item_rows = reinterpret_cast<int*>(w + L.fwd.nrows);
+  pa.item_seg_off = reinterpret_cast<int*>(w + L.fwd.seg_off);
+  pa.item_tile_off = reinterpret_cast<int*>(w + L.fwd.tile_off);
+  pa.tile_seg_off = reinterpret_cast<int*>(w + L.fwd.tile_seg_off);
+  pa.segs = reinterpret_cast<int*>(w + L.fwd.segs);
+  pa.queue = reinterpret_cast<int*>(w + L.fwd.queue);
+  pa.hist = reinterpret_cast<int*>(w + L.fwd.hist);
+  pa.n_hist = L.fwd.n_hist;
+  pa.lpt_queue = 0;
+  pa.stats = reinterpret_cast<long long*>(w + L.fwd.stats);
+  PSA_CUDA(psa::launch_plan(pa, st), "plan launch");
+  psa::AttnArgs aa{};
+  aa.B = s->B; aa.Hq = s->Hq; aa.Hkv = s->Hkv; aa.N = s->N; aa.d = s->d; aa.block = s->block;
+  aa.levels = s->levels; aa.causal = s->causal != 0; aa.n_items = L.fwd.n_items; aa.n_qtiles = L.fwd.n_qtiles;
+  aa.scale_log2 = sm_scale * 1.4426950408889634f;
+  aa.item_tile_off = pa.item_tile_off;
+  aa.item_rows = pa.item_rows;
+  aa.tile_seg_off = pa.tile_seg_off;
+  aa.segs = pa.segs;
+  aa.queue = pa.queue;
+  aa.out = out;
+  aa.out_fp32 = 0;
+  aa.lse = lse;
+  aa.status = reinterpret_cast<int*>(w + L.fwd.status);
+  aa.qscale = qs;
+  aa.kscale = ks;
+  PSA_CUDA(psa::launch_attention_fp8(maps, aa, num_sms(), st), "fp8 attention launch");
   return PSA_OK;
 }
 

@@ -125,12 +125,18 @@ __device__ __forceinline__ uint32_t sub_count(int rows) { return static_cast<uin
 // H2: the query tile holds two 64-token query blocks whose segment lists
 // differ, so records are kept per query half (block 64); with 128-token
 // blocks both halves always agree and the per-half work is compiled out.
-template <int D, bool OUT_F32, int NST, int CTAS, bool H2>
+// QK8: the FP8 path.  Q and K arrive as e4m3 codes (128-byte rows at d = 128,
+// one 128-byte-swizzled chunk), S = Q K^T runs as kind::f8f6f4 MMAs (K = 32
+// per instruction), and the softmax scale of a row carries the row's query
+// scale times its KV head's key scale; V, P and O are as in the bf16 path.
+template <int D, bool OUT_F32, int NST, int CTAS, bool H2, bool QK8 = false>
 __global__ void __launch_bounds__(kThreads, CTAS)
     attn_kernel(const __grid_constant__ AttnMaps maps, const AttnArgs a) {
-  constexpr int QB = D * 256;          // bytes of the 128-row Q tile
-  constexpr int SB = D * 128;          // bytes of a 64-row K or V stage
-  constexpr int KC = D / 64;           // 64-channel chunks
+  static_assert(!QK8 || D == 128, "the FP8 path is built for d = 128");
+  constexpr int QB = QK8 ? D * 128 : D * 256;    // bytes of the 128-row Q tile
+  constexpr int SBK = QK8 ? D * 64 : D * 128;    // bytes of a 64-row K stage
+  constexpr int SB = D * 128;                    // bytes of a 64-row V stage
+  constexpr int KC = D / 64;                     // 64-channel bf16 chunks
   constexpr uint32_t kTmemCols = 256;
   using Shared = AttnShared<NST>;
 
@@ -138,7 +144,7 @@ __global__ void __launch_bounds__(kThreads, CTAS)
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = base;
   uint8_t* sK = sQ + QB;               // NST stages
-  uint8_t* sV = sK + NST * SB;         // NST stages
+  uint8_t* sV = sK + NST * SBK;        // NST stages
   Shared* sh = reinterpret_cast<Shared*>(sV + NST * SB);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -197,8 +203,12 @@ __global__ void __launch_bounds__(kThreads, CTAS)
       if (lane == 0) {
         const uint32_t bar = smem_u32(&sh->q_full);
         mbar_arrive_expect_tx(bar, QB);
+        if (QK8) {
+          tma_load_3d(smem_u32(sQ), &maps.m[0], bar, 0, q0, bh);
+        } else {
 #pragma unroll
-        for (int kc = 0; kc < KC; ++kc) tma_load_3d(smem_u32(sQ + kc * 16384), &maps.m[0], bar, kc * 64, q0, bh);
+          for (int kc = 0; kc < KC; ++kc) tma_load_3d(smem_u32(sQ + kc * 16384), &maps.m[0], bar, kc * 64, q0, bh);
+        }
       }
       ++qcnt;
       // V loads run one sub-tile behind the K loads: V_j is needed only after
@@ -241,13 +251,17 @@ __global__ void __launch_bounds__(kThreads, CTAS)
 
         // K
         if (!warp_wait(smem_u32(&sh->k_empty[st]), ph ^ 1, abort, a.status, 12, idx, j, it, 0)) { ok = false; break; }
-        if (lane == 0) mbar_arrive_expect_tx(smem_u32(&sh->k_full[st]), SB);
+        if (lane == 0) mbar_arrive_expect_tx(smem_u32(&sh->k_full[st]), SBK);
         __syncwarp();
         if (mine) {
+          if (QK8) {
+            tma_load_3d(smem_u32(sK + st * SBK + dst * 128), &maps.m[1 + l], smem_u32(&sh->k_full[st]), 0, prow, hkv);
+          } else {
 #pragma unroll
-          for (int kc = 0; kc < KC; ++kc)
-            tma_load_3d(smem_u32(sK + st * SB + kc * 8192 + dst * 128), &maps.m[1 + l], smem_u32(&sh->k_full[st]),
-                        kc * 64, prow, hkv);
+            for (int kc = 0; kc < KC; ++kc)
+              tma_load_3d(smem_u32(sK + st * SBK + kc * 8192 + dst * 128), &maps.m[1 + l], smem_u32(&sh->k_full[st]),
+                          kc * 64, prow, hkv);
+          }
         }
         ++kiss;
         if (trap) {
@@ -314,6 +328,7 @@ __global__ void __launch_bounds__(kThreads, CTAS)
     // =============================== MMA issuer ===============================
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, kSub, false);
+      constexpr uint32_t idS8 = idesc_e4m3_f32(128, kSub);
       constexpr uint32_t idO = idesc_bf16_f32(128, D, true);
       uint32_t it = 0, qcnt = 0, icnt = 0;
       bool ok = true;
@@ -353,12 +368,18 @@ __global__ void __launch_bounds__(kThreads, CTAS)
           // S_j = Q K_j^T into S buffer sb2
           if (!bounded_wait(smem_u32(&sh->k_full[st]), (g / NST) & 1, abort, a.status, 24, idx, j, g, 0)) { ok = false; break; }
           tc_fence_after();
+          if (QK8) {
 #pragma unroll
-          for (int kc = 0; kc < KC; ++kc) {
+            for (int k = 0; k < D / 32; ++k)
+              umma_ss_f8(tmem + sb2 * kSub, dQ + ((32 * k) >> 4), dK + ((st * SBK + 32 * k) >> 4), idS8, k != 0);
+          } else {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              umma_ss(tmem + sb2 * kSub, dQ + ((kc * 16384 + 32 * k) >> 4),
-                      dK + ((st * SB + kc * 8192 + 32 * k) >> 4), idS, (kc | k) != 0);
+            for (int kc = 0; kc < KC; ++kc) {
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                umma_ss(tmem + sb2 * kSub, dQ + ((kc * 16384 + 32 * k) >> 4),
+                        dK + ((st * SBK + kc * 8192 + 32 * k) >> 4), idS, (kc | k) != 0);
+              }
             }
           }
           umma_commit(smem_u32(&sh->s_full[sb2]));
@@ -404,6 +425,14 @@ __global__ void __launch_bounds__(kThreads, CTAS)
       }
       const uint32_t n = sub_count(a.item_rows[item]);
       float m = -CUDART_INF_F, lsum = 0.f;
+      // softmax scale of this row (log2 units); the FP8 path folds in the
+      // row's query scale and its KV head's key scale
+      float row_sc = a.scale_log2;
+      if (QK8) {
+        const int b = bh / a.Hq, h = bh - b * a.Hq;
+        const int hkv = b * a.Hkv + h / (a.Hq / a.Hkv);
+        row_sc *= (tok < a.N ? a.qscale[orow] : 0.f) * a.kscale[hkv];
+      }
       for (uint32_t j = 0; j < n; ++j, ++it) {
         const uint32_t st = it % NST, sb2 = it & 1;
         if (!warp_wait(smem_u32(&sh->s_full[sb2]), (it >> 1) & 1, abort, a.status, 31, idx, j, it, 0)) { ok = false; break; }
@@ -417,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, CTAS)
 #pragma unroll
         for (int i = 0; i < 32; ++i) { s[i] = __uint_as_float(sr[i]); s[32 + i] = __uint_as_float(sr2[i]); }
         // exp2 argument of column c in chunk k: s[c] * sc + cb[k] - m
-        float sc = a.scale_log2;
+        float sc = row_sc;
         float cb[4];
         float mt;
         const bool fast_tile = ti.fast != 0;
@@ -563,23 +592,24 @@ __global__ void __launch_bounds__(kThreads, CTAS)
 #define PSA_ATTN_CTAS 2
 #endif
 
-template <int D, bool F32>
+template <int D, bool F32, bool QK8 = false>
 cudaError_t launch_one(const AttnMaps& maps, const AttnArgs& a, int num_sms, cudaStream_t s) {
   constexpr int CTAS = PSA_ATTN_CTAS;
   constexpr int NST = CTAS == 1 ? (D == 128 ? 5 : 8) : 2;
-  const size_t smem = 1024 + static_cast<size_t>(D) * 256 + 2 * NST * static_cast<size_t>(D) * 128 +
-                      sizeof(AttnShared<NST>);
+  constexpr size_t QB = QK8 ? static_cast<size_t>(D) * 128 : static_cast<size_t>(D) * 256;
+  constexpr size_t SBK = QK8 ? static_cast<size_t>(D) * 64 : static_cast<size_t>(D) * 128;
+  const size_t smem = 1024 + QB + NST * (SBK + static_cast<size_t>(D) * 128) + sizeof(AttnShared<NST>);
   const int grid = a.n_items < CTAS * num_sms ? a.n_items : CTAS * num_sms;
   if (a.block == 64) {
-    cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(attn_kernel<D, F32, NST, CTAS, true>),
+    cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(attn_kernel<D, F32, NST, CTAS, true, QK8>),
                                    static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    attn_kernel<D, F32, NST, CTAS, true><<<grid, kThreads, smem, s>>>(maps, a);
+    attn_kernel<D, F32, NST, CTAS, true, QK8><<<grid, kThreads, smem, s>>>(maps, a);
   } else {
-    cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(attn_kernel<D, F32, NST, CTAS, false>),
+    cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(attn_kernel<D, F32, NST, CTAS, false, QK8>),
                                    static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    attn_kernel<D, F32, NST, CTAS, false><<<grid, kThreads, smem, s>>>(maps, a);
+    attn_kernel<D, F32, NST, CTAS, false, QK8><<<grid, kThreads, smem, s>>>(maps, a);
   }
   return cudaGetLastError();
 }
@@ -592,6 +622,14 @@ cudaError_t launch_attention(const CUtensorMap* maps, const AttnArgs& a, int num
   for (int i = 1 + 2 * a.levels; i < 9; ++i) m.m[i] = maps[0];
   if (a.d == 128) return a.out_fp32 ? launch_one<128, true>(m, a, num_sms, s) : launch_one<128, false>(m, a, num_sms, s);
   return a.out_fp32 ? launch_one<64, true>(m, a, num_sms, s) : launch_one<64, false>(m, a, num_sms, s);
+}
+
+cudaError_t launch_attention_fp8(const CUtensorMap* maps, const AttnArgs& a, int num_sms, cudaStream_t s) {
+  if (a.d != 128 || a.out_fp32) return cudaErrorInvalidValue;
+  AttnMaps m;
+  for (int i = 0; i < 1 + 2 * a.levels; ++i) m.m[i] = maps[i];
+  for (int i = 1 + 2 * a.levels; i < 9; ++i) m.m[i] = maps[0];
+  return launch_one<128, false, true>(m, a, num_sms, s);
 }
 
 }  // namespace psa
