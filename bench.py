@@ -18,7 +18,9 @@ mask fetches for I); skipped blocks and tile padding are not work.
 this path) on the machine's host cores, on a bounded sample of the same
 workload, in the same unit.  With torchrun (N > 1) every rank runs its own
 full workload instance (weak scaling, no data-path collective); only the
-timing is reduced (max over ranks).
+timing is reduced (max over ranks).  --split heads instead splits one
+problem's heads over the ranks (strong scaling), with the all-gather of the
+output timed apart.
 """
 from __future__ import annotations
 
@@ -166,6 +168,29 @@ def max_over_ranks(ms: float, world: int, device) -> float:
     t = torch.tensor([ms], device=device, dtype=torch.float64)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def head_partition(Hq: int, Hkv: int, rank: int, world: int):
+    """The KV heads [hkv0, hkv1) and query heads [hq0, hq1) of one rank when
+    the heads of one problem are split over `world` GPUs: KV heads in equal
+    contiguous runs, each with the query heads that read it (GQA groups are
+    never split).  Needs Hkv % world == 0."""
+    if Hkv % world:
+        raise ValueError("Hkv = %d is not a multiple of %d GPUs" % (Hkv, world))
+    per = Hkv // world
+    grp = Hq // Hkv
+    hkv0, hkv1 = rank * per, (rank + 1) * per
+    return hkv0 * grp, hkv1 * grp, hkv0, hkv1
+
+
+def gather_heads(x: torch.Tensor, world: int) -> torch.Tensor:
+    """All-gather of a [B, H_local, ...] tensor along the head axis: the full
+    output on every rank (NCCL over NVLink on GPUs; any backend works)."""
+    if world <= 1:
+        return x
+    parts = [torch.empty_like(x) for _ in range(world)]
+    torch.distributed.all_gather(parts, x.contiguous())
+    return torch.cat(parts, dim=1)
 
 
 def aggregate_tflops(flops_per_rank: float, world: int, ms_per_step: float) -> float:
@@ -340,7 +365,15 @@ def run_psa(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     w = workload(args)
     log(args, "generating %s inputs" % w.name)
-    q, k, v, gen = W.make_qkv(w, device=dev, seed=w.seed + rank)
+    split = args.split == "heads" and world > 1
+    q, k, v, gen = W.make_qkv(w, device=dev, seed=w.seed if split else w.seed + rank)
+    if split:
+        # one problem, its heads split over the ranks (every rank draws the
+        # same inputs and keeps its own heads)
+        hq0, hq1, hkv0, hkv1 = head_partition(w.Hq, w.Hkv, rank, world)
+        q, k, v = q[:, hq0:hq1].contiguous(), k[:, hkv0:hkv1].contiguous(), v[:, hkv0:hkv1].contiguous()
+        w = w.replace(name="%s[heads %d-%d of %d]" % (w.name, hq0, hq1 - 1, W.PRESETS[w.name].Hq if w.name in W.PRESETS else w.Hq),
+                      Hq=hq1 - hq0, Hkv=hkv1 - hkv0)
     torch.cuda.synchronize()
     log(args, "inputs ready")
     path = Path(w, q, k, v)
@@ -367,7 +400,24 @@ def run_psa(args, rank, world, local_rank):
     n_tiles, n_rows = m["n_tiles"], m["n_rows"]
     pyr_ms, mask_ms, attn_ms, dense_ms = m["pyr_ms"], m["mask_ms"], m["attn_ms"], m["dense_ms"]
     ms_per_step = m["total_ms"] / args.steps
-    value = aggregate_tflops(flops, world, ms_per_step)
+    if split:
+        # strong scaling: the ranks share one problem; sum their work
+        tot = torch.tensor([flops], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(tot)
+        value = float(tot.item()) / (ms_per_step * 1e-3) / 1e12
+    else:
+        value = aggregate_tflops(flops, world, ms_per_step)
+    gather_ms = None
+    if split and not args.no_gather:
+        # the full output on every rank, timed apart from the step
+        torch.distributed.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        full = gather_heads(path.out, world)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        gather_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        del full
 
     # end to end through the public API with host buffers
     e2e = run_e2e(path, w, flops, args, stream) if not args.no_e2e else None
@@ -380,14 +430,17 @@ def run_psa(args, rank, world, local_rank):
     hist = torch.bincount(path.mask.flatten().long(), minlength=256).cpu()
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "strong" if split else "weak",
         "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "fp32 in, bf16 MMA",
         "data": "synthetic (smooth Gaussian field + noise, seeded)" if w.recipe == "field" else "synthetic iid N(0,1)",
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "block": w.block,
                    "levels": w.levels, "causal": w.causal, "mask": w.mask_mode, "policy": w.policy, "thresholds": list(w.thresholds),
                    "l2": "inputs (%.2f GB) larger than L2; no flush" % ((q.numel() + 2 * k.numel()) * q.element_size() / 1e9),
                    "step": "psa_build_pyramid + psa_make_mask + psa_attention_fwd",
-                   "parallelism": "replicas, one workload instance per GPU" if world > 1 else "single GPU"},
+                   "parallelism": ("heads split over %d GPUs (KV heads in equal runs, no data-path collective; "
+                                   "all-gather of O timed apart)" % world) if split else
+                                  ("replicas, one workload instance per GPU" if world > 1 else "single GPU")},
         "stages_ms": {"pyramid": pyr_ms, "mask": mask_ms, "attention": attn_ms},
         "attn_fwd_ms": attn_ms, "attn_fwd_tflops": attn_tflops,
         "executed_tflop_per_step": flops / 1e12, "dense_tflop": dense / 1e12,
@@ -403,6 +456,7 @@ def run_psa(args, rank, world, local_rank):
         "pyramid_roofline": {"bound": "hbm", "achieved": pyr_bytes / (pyr_ms * 1e-3) / 1e9, "peak": hbm,
                              "unit": "GB/s", "frac": pyr_bytes / (pyr_ms * 1e-3) / 1e9 / hbm},
         "e2e": e2e,
+        "gather_out_ms": gather_ms,
         "gpu_launches": launches_per_step(w) * args.steps,
         "clocks": clocks,
     }
@@ -725,6 +779,9 @@ def main():
     ap.add_argument("--no-configs", action="store_true", help="skip the per-preset records of the default line")
     ap.add_argument("--no-backward", action="store_true", help="skip the timing of psa_attention_bwd")
     ap.add_argument("--no-fp8", action="store_true", help="skip the timing of psa_attention_fwd_fp8")
+    ap.add_argument("--split", default="replicas", choices=["replicas", "heads"],
+                    help="N > 1: one workload instance per GPU (weak scaling) or one problem's heads split (strong)")
+    ap.add_argument("--no-gather", action="store_true", help="with --split heads: skip the all-gather of O")
     ap.add_argument("--config-steps", type=int, default=10, help="timed steps per preset in the configs record")
     ap.add_argument("--config-parity-blocks", type=int, default=8,
                     help="query blocks of one head per preset checked against the oracle")
