@@ -170,3 +170,27 @@ def test_backward_many_items_per_cta(d, block):
     rq, rk, rv = O.attention_backward(sel(q), sel(k), sel(v), sel(mask).cpu(), block, sm_scale, False, 4, sel(dout))
     for n, a, b in (("dq", sel(dq), rq), ("dk", sel(dk), rk), ("dv", sel(dv), rv)):
         compare(n, a, b)
+
+
+@pytest.mark.parametrize("d,block", [(128, 128), (64, 64)])
+def test_backward_is_deterministic(d, block):
+    """Three calls on the same inputs give bit-identical gradients (the
+    kernels have no atomics and a fixed order of work inside every tile;
+    a race between the warps that share a TMEM buffer would show here)."""
+    g = gen(81)
+    H, N = 40, 1024
+    q = torch.randn(1, H, N, d, generator=g).bfloat16().to(DEV)
+    k = torch.randn(1, H, N, d, generator=g).bfloat16().to(DEV)
+    v = torch.randn(1, H, N, d, generator=g).bfloat16().to(DEV)
+    nb = N // block
+    m = torch.randint(0, 5, (1, H, nb, nb), generator=g)
+    mask = torch.where(m == 4, torch.full_like(m, SKIP), m).to(torch.uint8).to(DEV)
+    shape = P.make_shape(1, H, H, N, d, block, 4)
+    kp, vp, _ = run_pyramid(shape, k, v)
+    out, lse, _ = run_attention(shape, q, k, v, kp, vp, mask, d ** -0.5)
+    dout = torch.randn(q.shape, generator=g).bfloat16().to(DEV)
+    first = run_backward(shape, q, k, v, kp, vp, mask, d ** -0.5, out, lse, dout)
+    for _ in range(2):
+        again = run_backward(shape, q, k, v, kp, vp, mask, d ** -0.5, out, lse, dout)
+        for a, b in zip(first, again):
+            assert torch.equal(a, b)

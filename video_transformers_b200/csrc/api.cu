@@ -626,13 +626,14 @@ psa_status_t psa_attention_bwd(const psa_shape_t* s, const void* q, const void* 
   const int64_t BHq = static_cast<int64_t>(s->B) * s->Hq, BHkv = static_cast<int64_t>(s->B) * s->Hkv;
   const char* kp = static_cast<const char*>(k_pyr);
   const char* vp = static_cast<const char*>(v_pyr);
-  // tensor maps: Q and dO in 128-row boxes; K / V levels in the forward's
-  // segment boxes (dQ kernel) and in 128-row boxes (dK / dV kernel)
+  // tensor maps: for the dQ kernel Q and dO in 128-row boxes and the K / V
+  // levels in the forward's segment boxes; for the dK / dV kernel Q and dO
+  // in 64-row boxes and the K / V levels in 128-row boxes
   CUtensorMap mq[10], mkv[10];
   PSA_TRY(map3(&mq[0], q, BHq, s->N, s->d, 128));
   PSA_TRY(map3(&mq[1], dout, BHq, s->N, s->d, 128));
-  mkv[0] = mq[0];
-  mkv[1] = mq[1];
+  PSA_TRY(map3(&mkv[0], q, BHq, s->N, s->d, 64));       // the dK / dV kernel streams 64-row query halves
+  PSA_TRY(map3(&mkv[1], dout, BHq, s->N, s->d, 64));
   for (int l = 0; l < s->levels; ++l) {
     const void* kb = l == 0 ? k : static_cast<const void*>(kp + pyr_level_offset(s, l, 2));
     const void* vb = l == 0 ? v : static_cast<const void*>(vp + pyr_level_offset(s, l, 2));

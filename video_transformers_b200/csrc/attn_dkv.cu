@@ -8,8 +8,10 @@
 // Its entries (from the transposed plan) are the query tiles that use some
 // block of the tile at level l.  One persistent CTA per SM, 6 warps:
 //   warp 0      TMA producer: the K^l / V^l tile once per item; per entry
-//               the 128-row Q and dO tiles and the padded lse2 / D rows into
-//               a two-stage ring.
+//               and 64-row query half, the Q and dO rows and the padded
+//               lse2 / D values into a four-slot ring of half-tiles (a slot
+//               is freed as soon as its half is accumulated, so the next
+//               loads start a half-step earlier than with whole tiles).
 //   warp 1      tcgen05 issuer (one thread), per 64-column query half hf:
 //               S^T = K Q_hf^T and dP^T = V dO_hf^T (M 128 KV rows, N 64,
 //               both operands from shared memory) into TMEM, then, once the
@@ -25,7 +27,10 @@
 //               item's dV^l (warps 2..5) and dK^l times sm_scale (warps
 //               6..9) rows in fp32.
 // TMEM (512 columns): S^T halves at [0, 64) and [64, 128), dP^T halves at
-// [128, 256), dV at [256, 256 + d), dK at [256 + d, 256 + 2 d).
+// [128, 256), dV at [256, 256 + d), dK at [256 + d, 256 + 2 d).  P^T and
+// dS^T overwrite S^T and dP^T in place: the packed bf16 pairs of query
+// columns 32 c .. 32 c + 31 go to buffer columns 32 c .. 32 c + 15, written by
+// the warp that read those columns.
 // Every wait is bounded; a time-out sets the workspace status word.
 #include <cuda_bf16.h>
 #include <math_constants.h>
@@ -44,15 +49,17 @@ struct DkvMaps {
   CUtensorMap m[10];
 };
 
+constexpr int kSlots = 4;     // query half-tiles in flight
+
 struct DkvShared {
   uint64_t kv_full, kv_empty;
-  uint64_t q_full[2], q_empty[2];
+  uint64_t q_full[kSlots], q_empty[kSlots];
   uint64_t s_full[2], p_full[2];
   uint64_t acc_full, acc_free, drain;
   uint32_t tmem_base;
   int abort;
-  alignas(16) float lse2[2][128];
-  alignas(16) float dd[2][128];
+  alignas(16) float lse2[kSlots][64];
+  alignas(16) float dd[kSlots][64];
 };
 
 __device__ __forceinline__ void item_of(const DkvArgs& a, int item, int& l, int& b, int& hkv, int& t) {
@@ -67,16 +74,17 @@ __device__ __forceinline__ void item_of(const DkvArgs& a, int item, int& l, int&
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) dkv_kernel(const __grid_constant__ DkvMaps maps, const DkvArgs a) {
-  constexpr int TB = D * 256;          // bytes of a 128-row tile (K, V, Q or dO)
-  constexpr int KC = D / 64;           // 64-channel chunks, 16 KB each
+  constexpr int TB = D * 256;          // bytes of a 128-row tile (K or V)
+  constexpr int HB = D * 128;          // bytes of a 64-row half-tile (Q or dO)
+  constexpr int KC = D / 64;           // 64-channel chunks
   constexpr uint32_t kTmemCols = 512;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = base;
   uint8_t* sV = sK + TB;
-  uint8_t* sQ = sV + TB;               // 2 stages
-  uint8_t* sG = sQ + 2 * TB;           // dO, 2 stages
-  DkvShared* sh = reinterpret_cast<DkvShared*>(sG + 2 * TB);
+  uint8_t* sQ = sV + TB;               // kSlots half-tiles
+  uint8_t* sG = sQ + kSlots * HB;      // dO, kSlots half-tiles
+  DkvShared* sh = reinterpret_cast<DkvShared*>(sG + kSlots * HB);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int L = a.levels;
@@ -84,9 +92,11 @@ __global__ void __launch_bounds__(kThreads, 1) dkv_kernel(const __grid_constant_
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&sh->kv_full), 1);
     mbar_init(smem_u32(&sh->kv_empty), 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kSlots; ++i) {
       mbar_init(smem_u32(&sh->q_full[i]), 1);
       mbar_init(smem_u32(&sh->q_empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&sh->s_full[i]), 1);
       mbar_init(smem_u32(&sh->p_full[i]), kSoftThreads);
     }
@@ -126,28 +136,31 @@ __global__ void __launch_bounds__(kThreads, 1) dkv_kernel(const __grid_constant_
           tma_load_3d(smem_u32(sV + kc * 16384), &maps.m[2 + L + l], kvb, kc * 64, t * 128, bhkv);
         }
         ++kcnt;
-        for (int e = 0; e < ne; ++e, ++qiss) {
-          const uint32_t st = qiss & 1, ph = (qiss >> 1) & 1;
-          if (!bounded_wait(smem_u32(&sh->q_empty[st]), ph ^ 1, abort, a.status, 42, idx, e, qiss, 0)) { ok = false; break; }
+        for (int e = 0; e < ne && ok; ++e) {
           const int qt = a.entry_qt[e0 + e];
           const int hl = qt / a.n_qtiles, tq = qt - hl * a.n_qtiles;
           const int bhq = b * a.Hq + hkv * grp + hl;
-          const uint32_t qb = smem_u32(&sh->q_full[st]);
-          mbar_arrive_expect_tx(qb, 2 * TB + 2 * 512);
+          for (int hf = 0; hf < 2; ++hf, ++qiss) {
+            const uint32_t sl = qiss % kSlots, ph = (qiss / kSlots) & 1;
+            if (!bounded_wait(smem_u32(&sh->q_empty[sl]), ph ^ 1, abort, a.status, 42, idx, e, qiss, hf)) { ok = false; break; }
+            const uint32_t qb = smem_u32(&sh->q_full[sl]);
+            mbar_arrive_expect_tx(qb, 2 * HB + 2 * 256);
 #pragma unroll
-          for (int kc = 0; kc < KC; ++kc) {
-            tma_load_3d(smem_u32(sQ + st * TB + kc * 16384), &maps.m[0], qb, kc * 64, tq * 128, bhq);
-            tma_load_3d(smem_u32(sG + st * TB + kc * 16384), &maps.m[1], qb, kc * 64, tq * 128, bhq);
+            for (int kc = 0; kc < KC; ++kc) {
+              tma_load_3d(smem_u32(sQ + sl * HB + kc * 8192), &maps.m[0], qb, kc * 64, tq * 128 + hf * 64, bhq);
+              tma_load_3d(smem_u32(sG + sl * HB + kc * 8192), &maps.m[1], qb, kc * 64, tq * 128 + hf * 64, bhq);
+            }
+            const int64_t prow = (static_cast<int64_t>(bhq) * a.n_qtiles + tq) * 128 + hf * 64;
+            bulk_load(smem_u32(&sh->lse2[sl][0]), a.lse2p + prow, 256, qb);
+            bulk_load(smem_u32(&sh->dd[sl][0]), a.dp + prow, 256, qb);
           }
-          const int64_t prow = (static_cast<int64_t>(bhq) * a.n_qtiles + tq) * 128;
-          bulk_load(smem_u32(&sh->lse2[st][0]), a.lse2p + prow, 512, qb);
-          bulk_load(smem_u32(&sh->dd[st][0]), a.dp + prow, 512, qb);
         }
       }
-      // drain: every copy issued must land before the CTA exits
+      // drain: every copy issued must land before the CTA exits (the last
+      // half loaded into slot sl is number qiss - 1 - ((qiss - 1 - sl) % kSlots))
       if (kcnt > 0) drain_wait(smem_u32(&sh->kv_full), (kcnt - 1) & 1, a.status);
-      for (uint32_t st = 0; st < 2; ++st)
-        if (qiss > st) drain_wait(smem_u32(&sh->q_full[st]), ((qiss - 1 - st) / 2) & 1, a.status);
+      for (uint32_t sl = 0; sl < static_cast<uint32_t>(kSlots); ++sl)
+        if (qiss > sl) drain_wait(smem_u32(&sh->q_full[sl]), ((qiss - 1 - sl) / kSlots) & 1, a.status);
     }
   } else if (warp == 1) {
     // =============================== MMA issuer ===============================
@@ -156,24 +169,30 @@ __global__ void __launch_bounds__(kThreads, 1) dkv_kernel(const __grid_constant_
       constexpr uint32_t idA = idesc_bf16_f32(128, D, true);
       const uint64_t dK = sdesc_sw128(smem_u32(sK), 16, 1024);
       const uint64_t dV = sdesc_sw128(smem_u32(sV), 16, 1024);
-      const uint64_t dQk = sdesc_sw128(smem_u32(sQ), 16, 1024);       // Q as the K-major B of S^T
-      const uint64_t dGk = sdesc_sw128(smem_u32(sG), 16, 1024);       // dO as the K-major B of dP^T
-      const uint64_t dQm = sdesc_sw128(smem_u32(sQ), 16384, 1024);    // Q as the MN-major B of dK
-      const uint64_t dGm = sdesc_sw128(smem_u32(sG), 16384, 1024);    // dO as the MN-major B of dV
-      uint32_t kcnt = 0, g = 0;
+      const uint64_t dQk = sdesc_sw128(smem_u32(sQ), 16, 1024);       // Q half as the K-major B of S^T
+      const uint64_t dGk = sdesc_sw128(smem_u32(sG), 16, 1024);       // dO half as the K-major B of dP^T
+      const uint64_t dQm = sdesc_sw128(smem_u32(sQ), 8192, 1024);     // Q half as the MN-major B of dK
+      const uint64_t dGm = sdesc_sw128(smem_u32(sG), 8192, 1024);     // dO half as the MN-major B of dV
+      uint32_t kcnt = 0, u = 0;        // u: query halves consumed (slot u % kSlots)
       bool ok = true;
-      // dV += P^T dO_hf, dK += dS^T Q_hf for entry number ge (stage ge & 1)
-      auto accumulate = [&](uint32_t ge, int hf, bool first) -> bool {
-        if (!bounded_wait(smem_u32(&sh->p_full[hf]), ge & 1, abort, a.status, 52, ge, hf, 0, 0)) return false;
+      // dV += P^T dO_h, dK += dS^T Q_h for half number uh (TMEM buffers hf = uh & 1),
+      // then its slot is released
+      auto accumulate = [&](uint32_t uh, bool first) -> bool {
+        const int hf = uh & 1;
+        if (!bounded_wait(smem_u32(&sh->p_full[hf]), (uh >> 1) & 1, abort, a.status, 52, uh, hf, 0, 0)) return false;
         tc_fence_after();
-        const uint32_t st = ge & 1;
+        const uint32_t sl = uh % kSlots;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const uint32_t off = (st * TB + hf * 8192 + k * 2048) >> 4;
+          const uint32_t off = (sl * HB + k * 2048) >> 4;
           const uint32_t acc = (first && k == 0) ? 0u : 1u;
-          umma_ts(tV, tS + hf * 64 + k * 8, dGm + off, idA, acc);
-          umma_ts(tK, tP + hf * 64 + k * 8, dQm + off, idA, acc);
+          // the packed P^T / dS^T of query columns 32 cg .. 32 cg + 31 sit at
+          // TMEM columns 32 cg .. 32 cg + 15 of the buffer (see the softmax)
+          const uint32_t ac = hf * 64 + k * 8 + (k >> 1) * 16;
+          umma_ts(tV, tS + ac, dGm + off, idA, acc);
+          umma_ts(tK, tP + ac, dQm + off, idA, acc);
         }
+        umma_commit(smem_u32(&sh->q_empty[sl]));
         return true;
       };
       for (int idx = blockIdx.x; idx < a.n_items && ok; idx += gridDim.x) {
@@ -186,33 +205,34 @@ __global__ void __launch_bounds__(kThreads, 1) dkv_kernel(const __grid_constant_
           break;
         }
         tc_fence_after();
-        const uint32_t g0 = g;
-        for (int e = 0; e < ne && ok; ++e, ++g) {
-          const uint32_t st = g & 1;
-          if (!bounded_wait(smem_u32(&sh->q_full[st]), (g >> 1) & 1, abort, a.status, 54, idx, e, g, 0)) { ok = false; break; }
-          tc_fence_after();
-          for (int hf = 0; hf < 2; ++hf) {
-            if (e > 0 && !accumulate(g - 1, hf, g - 1 == g0 && hf == 0)) { ok = false; break; }
+        const uint32_t u0 = u;
+        for (int e = 0; e < ne && ok; ++e) {
+          for (int hf = 0; hf < 2; ++hf, ++u) {
+            // the previous entry's half hf frees TMEM buffer hf before S^T of this one
+            if (e > 0 && !accumulate(u - 2, u - 2 == u0)) { ok = false; break; }
+            const uint32_t sl = u % kSlots;
+            if (!bounded_wait(smem_u32(&sh->q_full[sl]), (u / kSlots) & 1, abort, a.status, 54, idx, e, u, 0)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
 #pragma unroll
             for (int kc = 0; kc < KC; ++kc) {
 #pragma unroll
               for (int k = 0; k < 4; ++k) {
                 const uint32_t ao = (kc * 16384 + 32 * k) >> 4;
-                const uint32_t bo = (st * TB + kc * 16384 + hf * 8192 + 32 * k) >> 4;
+                const uint32_t bo = (sl * HB + kc * 8192 + 32 * k) >> 4;
                 umma_ss(tS + hf * 64, dK + ao, dQk + bo, idS, (kc | k) != 0);
                 umma_ss(tP + hf * 64, dV + ao, dGk + bo, idS, (kc | k) != 0);
               }
             }
             umma_commit(smem_u32(&sh->s_full[hf]));
           }
-          if (!ok) break;
-          if (e > 0) umma_commit(smem_u32(&sh->q_empty[(g - 1) & 1]));
         }
         if (!ok) break;
         for (int hf = 0; hf < 2; ++hf)
-          if (!accumulate(g - 1, hf, g - 1 == g0 && hf == 0)) { ok = false; break; }
+          if (!accumulate(u - 2 + hf, u - 2 + hf == u0)) { ok = false; break; }
         if (!ok) break;
-        umma_commit(smem_u32(&sh->q_empty[(g - 1) & 1]));
         umma_commit(smem_u32(&sh->acc_full));
         umma_commit(smem_u32(&sh->kv_empty));
         ++kcnt;
@@ -226,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1) dkv_kernel(const __grid_constant_
     const int cg = (warp - 2) >> 2;                       // 32-column group of each half
     const int r = q * 32 + lane;                          // KV row of the tile
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-    uint32_t kcnt = 0, g = 0;
+    uint32_t kcnt = 0, g = 0;        // g: entries processed (query halves 2 g, 2 g + 1)
     bool ok = true;
     for (int idx = blockIdx.x; idx < a.n_items && ok; idx += gridDim.x) {
       const int item = a.n_items - 1 - idx;
@@ -250,7 +270,6 @@ __global__ void __launch_bounds__(kThreads, 1) dkv_kernel(const __grid_constant_
         continue;
       }
       for (int e = 0; e < ne && ok; ++e, ++g) {
-        const uint32_t st = g & 1;
         const unsigned bits = a.entry_mask[e0 + e];
         const int qt = a.entry_qt[e0 + e];
         const int tq = qt - (qt / a.n_qtiles) * a.n_qtiles;
@@ -267,8 +286,9 @@ __global__ void __launch_bounds__(kThreads, 1) dkv_kernel(const __grid_constant_
           // the hidden columns are exactly c < cut
           const int cut = !valid ? 32 : (a.causal ? max(0, min(32, last_tok - q_first)) : 0);
           const float sc = a.scale_log2;
-          const float4* lz4 = reinterpret_cast<const float4*>(&sh->lse2[st][hf * 64 + cg * 32]);
-          const float4* dz4 = reinterpret_cast<const float4*>(&sh->dd[st][hf * 64 + cg * 32]);
+          const uint32_t sl = (2 * g + hf) % kSlots;
+          const float4* lz4 = reinterpret_cast<const float4*>(&sh->lse2[sl][cg * 32]);
+          const float4* dz4 = reinterpret_cast<const float4*>(&sh->dd[sl][cg * 32]);
           uint32_t pk[16], gk[16];
 #pragma unroll
           for (int i4 = 0; i4 < 8; ++i4) {
@@ -287,8 +307,10 @@ __global__ void __launch_bounds__(kThreads, 1) dkv_kernel(const __grid_constant_
             gk[2 * i4] = pack_bf16(gv[0], gv[1]);
             gk[2 * i4 + 1] = pack_bf16(gv[2], gv[3]);
           }
-          tmem_st16(tS + hf * 64 + cg * 16 + lane_off, pk);
-          tmem_st16(tP + hf * 64 + cg * 16 + lane_off, gk);
+          // each warp writes its packed half only over columns it has read
+          // itself (its partner may not have loaded its own columns yet)
+          tmem_st16(tS + hf * 64 + cg * 32 + lane_off, pk);
+          tmem_st16(tP + hf * 64 + cg * 32 + lane_off, gk);
           tmem_st_wait();
           tc_fence_before();
           mbar_arrive(smem_u32(&sh->p_full[hf]));
@@ -328,7 +350,8 @@ __global__ void __launch_bounds__(kThreads, 1) dkv_kernel(const __grid_constant_
 
 template <int D>
 cudaError_t launch_d(const DkvMaps& maps, const DkvArgs& a, int num_sms, cudaStream_t s) {
-  const size_t smem = 1024 + 6 * static_cast<size_t>(D) * 256 + sizeof(DkvShared);
+  const size_t smem = 1024 + 2 * static_cast<size_t>(D) * 256 + 2 * kSlots * static_cast<size_t>(D) * 128 +
+                      sizeof(DkvShared);
   const int grid = a.n_items < num_sms ? a.n_items : num_sms;
   if (grid <= 0) return cudaSuccess;
   cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(dkv_kernel<D>), static_cast<int>(smem));

@@ -21,6 +21,9 @@
 //               64 columns: p and ds, ds as bf16 into the S buffer; the
 //               epilogue writes dQ * sm_scale, each warp half of the row.
 // TMEM (512 columns): S at [0, 128), dP at [128, 256), dQ at [256, 256 + d).
+// dS overwrites S in place: the packed bf16 pairs of columns 32 c .. 32 c + 31
+// of a sub-tile go to columns 32 c .. 32 c + 15, written by the warp that
+// read them.
 // Every wait is bounded; a time-out sets the workspace status word.
 #include <cuda_bf16.h>
 #include <math_constants.h>
@@ -206,7 +209,9 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < kSub / 16; ++k)
-          umma_ts(tQ, tS + sb2 * kSub + k * 8, dKm + ((st * SB + k * 2048) >> 4), idO, (jj == 0 && k == 0) ? 0u : 1u);
+          // packed dS of columns 32 c .. 32 c + 31 sits at columns 32 c .. 32 c + 15
+          umma_ts(tQ, tS + sb2 * kSub + k * 8 + (k >> 1) * 16, dKm + ((st * SB + k * 2048) >> 4), idO,
+                  (jj == 0 && k == 0) ? 0u : 1u);
         umma_commit(smem_u32(&sh->kv_empty[st]));
         return true;
       };
@@ -315,7 +320,9 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
           const float p0 = fast_exp2(x[c]), p1 = fast_exp2(x[c + 1]);
           pk[i] = pack_bf16(p0 * (__uint_as_float(dr[c]) - Dv), p1 * (__uint_as_float(dr[c + 1]) - Dv));
         }
-        tmem_st16(tS + sb2 * kSub + cg * 16 + lane_off, pk);
+        // written over columns this warp read itself: its partner may not
+        // have loaded its own columns yet
+        tmem_st16(tS + sb2 * kSub + cg * 32 + lane_off, pk);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(smem_u32(&sh->ds_full[sb2]));

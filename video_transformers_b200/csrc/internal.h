@@ -194,7 +194,7 @@ struct DkvArgs {
   int64_t level_off[4];   // element offset of level l ([B*Hkv][N >> l][d])
   int* status;
 };
-// maps: [0] = Q, [1] = dO (box 64 x 128), [2 + l] = K level l, [2 + L + l] =
+// maps: [0] = Q, [1] = dO (box 64 x 64 rows), [2 + l] = K level l, [2 + L + l] =
 // V level l (box 64 x 128 rows).
 cudaError_t launch_dkv(const CUtensorMap* maps, const DkvArgs& a, int num_sms, cudaStream_t s);
 
