@@ -47,8 +47,8 @@ METRIC = "PSA attn fwd ms/call & achieved TFLOP/s (executed FLOPs) vs B200 BF16 
 # ncu capture of the same workload at 4 heads scaled to the full head count (traffic grows with
 # the heads: the head-major queue keeps one head's KV in L2 at a time); valid only for the
 # attention source it was measured on, identified by its SHA-256.
-ATTN_TRAFFIC = {"wan14b": {"bytes_per_launch": 10 * (743.809280e6 + 71.797504e6),
-                           "attn_cu_sha256": "b99157c006021851afeb671c24c57be7ee988983e6b850d20d79d5b3f8cc9f72"}}
+ATTN_TRAFFIC = {"wan14b": {"bytes_per_launch": 10 * (796.720384e6 + 72.149760e6),
+                           "attn_cu_sha256": "5b61d94266c01037c51aa8d054f153df9ab701c044f29eb211e1a91be54f8c3b"}}
 UNIT = "TFLOP/s"
 KERNELS_PER_STEP = {"pyramid": 1, "blockcos": 0, "score": 1, "select": 1, "plan": 3, "attention": 1}
 # kernels of psa_make_mask per scorer: score + select, or block means (Q, K),
