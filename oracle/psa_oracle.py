@@ -585,7 +585,8 @@ def attention(q, kp, vp, mask, block: int, sm_scale: float, causal: bool,
     return o, lse
 
 
-def attention_backward(q, k, v, mask, block: int, sm_scale: float, causal: bool, levels: int, dout):
+def attention_backward(q, k, v, mask, block: int, sm_scale: float, causal: bool, levels: int, dout,
+                       rows: Optional[Iterable[Tuple[int, int, int]]] = None):
     """Gradients of adaptive pyramid attention with respect to Q, K and V
     (not on the pages' hot path: the news review claims end-to-end
     training, the summary article pairs PSA with distillation).  The mask
@@ -600,7 +601,10 @@ def attention_backward(q, k, v, mask, block: int, sm_scale: float, causal: bool,
     then through the pooling of level l (a mean of 2^l consecutive tokens):
     dK[t] += dK^l[t >> l] / 2^l, and the same for V.  Rows with no visible
     key contribute nothing.  q: [B, Hq, N, d]; k, v: [B, Hkv, N, d];
-    dout: [B, Hq, N, d].  Returns (dq, dk, dv) in float64."""
+    dout: [B, Hq, N, d].  Returns (dq, dk, dv) in float64.  When ``rows``
+    lists (b, h, I) triples only those query blocks are visited: their dq
+    rows are complete (a row's dq depends only on its own key set), dk and
+    dv then hold only those blocks' contributions."""
     q = _f64(q)
     k = _f64(k)
     v = _f64(v)
@@ -614,10 +618,13 @@ def attention_backward(q, k, v, mask, block: int, sm_scale: float, causal: bool,
     dq = np.zeros_like(q)
     dkp = [np.zeros_like(x) for x in kp]
     dvp = [np.zeros_like(x) for x in vp]
+    want = None if rows is None else set(rows)
     for b in range(B):
         for h in range(Hq):
             hk = h // grp
             for I in range(nb):
+                if want is not None and (b, h, I) not in want:
+                    continue
                 i0, i1 = I * block, min((I + 1) * block, N)
                 # the key set of I, remembering where each key came from
                 src = []

@@ -171,3 +171,64 @@ def test_fullsize_mask_variants_sampled(mode, policy):
         assert mx <= 2e-2 and mean <= 2e-3, (mode, policy, h, I, mx, mean)
     assert P.psa_get_device_status(ws) == P.PSA_OK
     check_band("wan14b full size, %s/%s" % (mode, policy), n_amb, n_pairs)
+
+
+def test_fullsize_fp8_wan14b_sampled():
+    """The FP8 path at the Wan2.1-14B shape on the generated mask, checked
+    on sampled query-block rows against the oracle's attention on the same
+    e4m3 operands (the GPU's quantizer codes are pinned bit for bit in
+    test_gpu_fp8.py; here the oracle quantizes the head itself)."""
+    w = W.PRESETS["wan14b"]
+    q, k, v, _ = W.make_qkv(w, device=DEV)
+    shape = shape_for(w)
+    kp, vp, _ = run_pyramid(shape, k, v)
+    mask, _ = run_mask(shape, params_for(w), q, k)
+    out = torch.empty_like(q)
+    ws = P.workspace(P.psa_attention_fp8_workspace_bytes(shape), DEV)
+    P.psa_attention_fwd_fp8(shape, q, k, v, kp, vp, mask, w.sm_scale, out, None, ws)
+    torch.cuda.synchronize()
+    assert P.psa_get_device_status(ws) == P.PSA_OK
+    rows = sample_rows(w, 10, seed=5)
+    for (b, h), Is in by_head(rows).items():
+        hrows = [(0, 0, I) for I in Is]
+        kl = head_levels(shape, k, kp, b, h, w.levels)
+        vl = head_levels(shape, v, vp, b, h, w.levels)
+        o, _ = O.attention_fp8(q[b:b + 1, h:h + 1].cpu(), [x.astype(np.float32) for x in kl], vl,
+                               mask[b:b + 1, h:h + 1].cpu(), w.block, w.sm_scale, False, rows=hrows)
+        mx, mean, _ = attn_errors(out[b:b + 1, h:h + 1], o)
+        assert mx <= 2e-2 and mean <= 2e-3, (h, Is, mx, mean)
+
+
+def test_fullsize_backward_dq_wan14b_sampled():
+    """The backward at the Wan2.1-14B shape at full grid: dq of sampled
+    query blocks against the oracle's backward restricted to those blocks
+    (a row's dq depends only on its own key set), same tolerance as the
+    backward tests (max-abs 2e-2 of max|ref|, mean-abs 6e-3 of mean|ref|)."""
+    w = W.PRESETS["wan14b"]
+    q, k, v, _ = W.make_qkv(w, device=DEV)
+    shape = shape_for(w)
+    kp, vp, _ = run_pyramid(shape, k, v)
+    mask, _ = run_mask(shape, params_for(w), q, k)
+    out, lse, _ = run_attention(shape, q, k, v, kp, vp, mask, w.sm_scale)
+    g = torch.Generator(device=DEV)
+    g.manual_seed(11)
+    dout = torch.randn(q.shape, generator=g, device=DEV).bfloat16()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = P.workspace(P.psa_attention_bwd_workspace_bytes(shape), DEV)
+    P.psa_attention_bwd(shape, q, k, v, kp, vp, mask, w.sm_scale, out, lse, dout, dq, dk, dv, ws)
+    torch.cuda.synchronize()
+    assert P.psa_get_device_status(ws) == P.PSA_OK
+    assert torch.isfinite(dk.float()).all() and torch.isfinite(dv.float()).all()
+    rows = sample_rows(w, 6, seed=17)
+    for (b, h), Is in by_head(rows).items():
+        hrows = [(0, 0, I) for I in Is]
+        rq, _, _ = O.attention_backward(q[b:b + 1, h:h + 1].cpu(), k[b:b + 1, h:h + 1].cpu(),
+                                        v[b:b + 1, h:h + 1].cpu(), mask[b:b + 1, h:h + 1].cpu(), w.block,
+                                        w.sm_scale, False, w.levels, dout[b:b + 1, h:h + 1].cpu(), rows=hrows)
+        for I in Is:
+            sl = slice(I * w.block, min((I + 1) * w.block, w.N))
+            ref = rq[0, 0, sl]
+            got = dq[b, h, sl].double().cpu().numpy()
+            err = np.abs(got - ref)
+            assert err.max() <= 2e-2 * np.abs(ref).max() and err.mean() <= 6e-3 * np.abs(ref).mean(), \
+                (h, I, err.max(), np.abs(ref).max(), err.mean(), np.abs(ref).mean())

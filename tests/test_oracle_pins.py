@@ -1099,3 +1099,16 @@ def test_mutation_head_scale_per_level(monkeypatch):
     monkeypatch.setattr(O, "quantize_heads_e4m3", bad)
     with pytest.raises(AssertionError):
         test_quantize_heads_e4m3_shares_level0_scale()
+
+
+def test_backward_rows_filter_matches_full():
+    """Visiting only some query blocks leaves their dq rows exactly as the
+    full computation gives them (a row's gradient depends on its own key
+    set only)."""
+    q, k, v, mask, blk, scale, causal, L, dout = _bwd_case(True)
+    full = O.attention_backward(q, k, v, mask, blk, scale, causal, L, dout)
+    rows = [(0, 1, 0), (0, 2, 2), (0, 0, 3)]
+    part = O.attention_backward(q, k, v, mask, blk, scale, causal, L, dout, rows=rows)
+    for b, h, I in rows:
+        np.testing.assert_array_equal(part[0][b, h, I * blk:(I + 1) * blk], full[0][b, h, I * blk:(I + 1) * blk])
+    assert np.all(part[0][0, 1, blk:2 * blk] == 0)
