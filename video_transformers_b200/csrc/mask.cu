@@ -15,14 +15,20 @@
 // score2_kernel  the sampling score at d = 128: two row tiles share every K
 //                tile, epilogue warpgroup x owns row tile x, and a work item
 //                covers half of the column tiles (row-LSE partial = half).
-// select_warp_kernel  one warp per (b, h, query block), up to 1024 key
-//                blocks: the same levels as select_kernel, keys in registers.
-// select_kernel  one CTA per (b, h, query block): block masses from the
-//                LSEs, a bitonic sort (mass descending, index ascending), an
-//                fp64 exclusive scan, levels by that prefix (or by rank for
-//                the quantile policy), forced rules.
+// select_bucket_kernel  one warp per (b, h, query block), up to 1024 key
+//                blocks: the same levels as select_kernel without a sort --
+//                a histogram of the masses in 256 buckets and its scan give
+//                every block's level, except in the few buckets a threshold
+//                falls into, whose blocks count their exact prefix (or rank).
+// select_kernel  (more than 1024 key blocks) one CTA per (b, h, query
+//                block): block masses from the LSEs, a bitonic sort (mass
+//                descending, index ascending), an fp64 exclusive scan, levels
+//                by that prefix (or by rank for the quantile policy), forced
+//                rules.
 #include <cuda_bf16.h>
 #include <math_constants.h>
+
+#include <type_traits>
 
 #include "exp2_poly.h"
 #include "internal.h"
@@ -667,24 +673,62 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectArgs a)
 }
 
 // ----------------------------------------------------------------------------
-// select, one warp per (b, h, I), for up to 1024 key blocks: lane l holds the
-// elements l + 32k (k < KPL) in registers; the bitonic network's exchanges
-// across lanes go through shuffles and those across k are register swaps.
-// Same results as select_kernel: keys (descending float mass, ascending J),
-// fp64 exclusive prefix of the float masses in rank order.
+// select by buckets, one warp per (b, h, query block), up to 1024 key blocks.
+// A block's level depends only on which thresholds its exclusive prefix C_J
+// (or its rank) passes, so no full sort is needed:
+// - the masses go into 256 buckets by their fraction of the row's largest
+//   mass (larger mass, lower bucket, so the buckets keep the rank order);
+//   exact zeros go into a bucket of their own after all others;
+// - a histogram of counts and of 64-bit fixed-point mass sums, and its
+//   exclusive scan, give every bucket's first prefix and first rank;
+// - a bucket with no threshold inside the range of prefixes (or ranks) its
+//   blocks can take gives them all one level;
+// - the blocks of the few buckets a threshold falls into are listed,
+//   grouped by bucket, and each counts the members of its own group that
+//   rank before it to get its exact prefix and rank.
+// Fixed-point sums are exact for masses above 2^-39 and do not depend on
+// the order of the additions.
 // ----------------------------------------------------------------------------
-constexpr int kSelWarps = 4;
+constexpr int kBuckets = 256;                   // plus bucket 256 for exact zeros
+constexpr int kBucketSlots = kBuckets + 2;      // slot 257 receives the totals
+constexpr double kFix = 4611686018427387904.0;  // 2^62: fixed-point scale of a mass in [0, 1]
+
+// key of a block: bits [32, 64) the mass's bits inverted (descending mass =
+// ascending key), [11, 20) its bucket, [0, 11) its index.  Equal masses
+// fall in one bucket, so the bucket bits never change the order.
+__device__ __forceinline__ float key_mass(unsigned long long key) {
+  return __uint_as_float(0xFFFFFFFFu - static_cast<unsigned>(key >> 32));
+}
+__device__ __forceinline__ int key_bucket(unsigned long long key) { return static_cast<int>((key >> 11) & 0x1FFu); }
+__device__ __forceinline__ unsigned long long mass_fix(float m) {
+  return static_cast<unsigned long long>(static_cast<double>(m) * kFix);
+}
 
 template <int KPL>
-__global__ void __launch_bounds__(32 * kSelWarps, 4) select_warp_kernel(const SelectArgs a) {
-  __shared__ double rlse_s[kSelWarps][128];
+struct BucketRow {
+  unsigned long long list[32 * KPL];   // keys of the blocks of mixed buckets, grouped by bucket
+  unsigned long long hs[kBucketSlots]; // fixed-point mass sums, then their exclusive prefix
+  unsigned long long tfx[8];           // thresholds in fixed point
+  double rlse[128];
+  int hc[kBucketSlots];                // counts, then the exclusive rank
+  int lend[kBucketSlots];              // start of the bucket's list group, then its end
+  uint8_t ex[32 * KPL];                // exact levels of the listed blocks, by J
+  uint8_t mixed[kBucketSlots];         // a threshold falls inside the bucket
+  uint8_t lv[kBucketSlots];            // the level of every block of an unmixed bucket
+};
+constexpr int bucket_warps(int kpl) { return kpl >= 16 ? 2 : 4; }
+
+template <int KPL>
+__global__ void __launch_bounds__(32 * bucket_warps(KPL)) select_bucket_kernel(const SelectArgs a) {
+  constexpr int NW = bucket_warps(KPL);
+  __shared__ BucketRow<KPL> rows_s[NW];
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const int row = blockIdx.x * kSelWarps + wid;                 // (b*Hq + h)*nqb + I
+  BucketRow<KPL>& sm = rows_s[wid];
+  const int row = blockIdx.x * NW + wid;                        // (b*Hq + h)*nqb + I
   if (row >= a.B * a.Hq * a.nqb) return;
   const int bh = row / a.nqb, I = row - bh * a.nqb;
   const int b = bh / a.Hq, h = bh - b * a.Hq;
   const int hkv = b * a.Hkv + h / (a.Hq / a.Hkv);
-  constexpr int P2 = 32 * KPL;
 
   const int rbeg = I * a.rows_per_block;
   int nvalid;
@@ -694,97 +738,204 @@ __global__ void __launch_bounds__(32 * kSelWarps, 4) select_warp_kernel(const Se
   } else {
     nvalid = min(a.rows_per_block, a.rows - rbeg);
   }
-  double* rlse = rlse_s[wid];
   for (int s = lane; s < nvalid; s += 32) {
     const double x = a.rowlse[static_cast<int64_t>(bh) * a.rows + rbeg + s];
     const double y = a.rowlse[(static_cast<int64_t>(a.B) * a.Hq + bh) * a.rows + rbeg + s];
     const double mx = fmax(x, y);
-    rlse[s] = mx == -CUDART_INF ? mx : mx + log2(exp2(x - mx) + exp2(y - mx));
+    sm.rlse[s] = mx == -CUDART_INF ? mx : mx + log2(exp2(x - mx) + exp2(y - mx));
+  }
+  for (int i = lane; i < kBucketSlots; i += 32) {
+    sm.hs[i] = 0ull;
+    sm.hc[i] = 0;
+  }
+  if (lane < 8) {
+    const float t = a.thresholds[lane];
+    sm.tfx[lane] = t >= 2.0f ? ~0ull : (t <= 0.0f ? 0ull : mass_fix(t));
   }
   __syncwarp();
 
+  // block masses (the same arithmetic as the sorting kernels) and keys
   unsigned long long key[KPL];
+  float mmax = 0.f;
 #pragma unroll
   for (int k = 0; k < KPL; ++k) {
     const int J = lane + 32 * k;
+    key[k] = ~0ull;
     if (J < a.nkb) {
       const float* bl = a.blocklse + (static_cast<int64_t>(bh) * a.nkb + J) * a.rows + rbeg;
       double m = 0.0;
       for (int s = 0; s < nvalid; ++s) {
         const float x = bl[s];
-        if (x != -CUDART_INF_F) m += exp2_split(static_cast<double>(x) - rlse[s]);
+        if (x != -CUDART_INF_F) m += exp2_split(static_cast<double>(x) - sm.rlse[s]);
       }
       const float mass = static_cast<float>(m / nvalid);
       if (a.mass_out) a.mass_out[static_cast<int64_t>(row) * a.nkb + J] = mass;
       key[k] = (static_cast<unsigned long long>(0xFFFFFFFFu - __float_as_uint(mass)) << 32) | static_cast<unsigned>(J);
-    } else {
-      key[k] = ~0ull;
+      mmax = fmaxf(mmax, mass);
     }
   }
-  // bitonic sort, ascending, element e = lane + 32k
 #pragma unroll
-  for (int size = 2; size <= P2; size <<= 1) {
-#pragma unroll
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      if (stride >= 32) {
-        const int ks = stride >> 5;
-#pragma unroll
-        for (int k = 0; k < KPL; ++k) {
-          if ((k & ks) == 0) {
-            const int e = lane + 32 * k;
-            const bool up = (e & size) == 0;
-            const unsigned long long x = key[k], y = key[k | ks];
-            if ((x > y) == up) { key[k] = y; key[k | ks] = x; }
-          }
-        }
-      } else {
-#pragma unroll
-        for (int k = 0; k < KPL; ++k) {
-          const int e = lane + 32 * k;
-          const unsigned long long y = __shfl_xor_sync(0xffffffffu, key[k], stride);
-          const bool up = (e & size) == 0;
-          const bool lower = (lane & stride) == 0;
-          // the lower element of an ascending pair keeps the minimum
-          const bool keep_min = up == lower;
-          key[k] = keep_min ? (key[k] < y ? key[k] : y) : (key[k] < y ? y : key[k]);
-        }
-      }
-    }
-  }
-  // exclusive prefix in rank order (rank r = lane + 32k), then levels
-  const int n_vis = a.causal ? min(I + 1, a.nkb) : a.nkb;
-  double carry = 0.0;
+  for (int o = 16; o > 0; o >>= 1) mmax = fmaxf(mmax, __shfl_xor_sync(0xffffffffu, mmax, o));
+
+  // buckets (monotone in the mass: the fp32 quotient and product round
+  // monotonically) and the histogram.  Exact zeros (every block past the
+  // diagonal of a causal row) add nothing to the sums and are counted by one
+  // ballot, not by atomics that would all hit one address.
 #pragma unroll
   for (int k = 0; k < KPL; ++k) {
-    const int r = lane + 32 * k;
-    const bool real = r < a.nkb;
-    const double v = real ? static_cast<double>(__uint_as_float(0xFFFFFFFFu - static_cast<unsigned>(key[k] >> 32))) : 0.0;
-    double incl = v;
+    const bool valid = key[k] != ~0ull;
+    const float m = valid ? key_mass(key[k]) : 1.f;
+    const unsigned zeros = __ballot_sync(0xffffffffu, m == 0.f);
+    if (lane == 0 && zeros) atomicAdd(&sm.hc[kBuckets], __popc(zeros));
+    if (!valid) continue;
+    int bb = kBuckets;
+    if (m != 0.f) {
+      bb = max(0, min(kBuckets - 1, static_cast<int>(floorf(static_cast<float>(kBuckets) * (1.0f - m / mmax)))));
+      atomicAdd(&sm.hc[bb], 1);
+      atomicAdd(&sm.hs[bb], mass_fix(m));
+    }
+    key[k] |= static_cast<unsigned long long>(bb) << 11;
+  }
+  __syncwarp();
+
+  // exclusive scan over buckets 0..kBuckets; lane l owns buckets 9l .. 9l+8
+  constexpr int PER = 9;                          // 32 * 9 = 288 >= kBuckets + 1
+  {
+    unsigned long long ls = 0ull;
+    int lc = 0;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int bb = lane * PER + i;
+      if (bb <= kBuckets) { ls += sm.hs[bb]; lc += sm.hc[bb]; }
+    }
+    unsigned long long is = ls;
+    int ic = lc;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const double y = __shfl_up_sync(0xffffffffu, incl, o);
+      const unsigned long long ys = __shfl_up_sync(0xffffffffu, is, o);
+      const int yc = __shfl_up_sync(0xffffffffu, ic, o);
+      if (lane >= o) { is += ys; ic += yc; }
+    }
+    unsigned long long cs = is - ls;
+    int cc = ic - lc;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int bb = lane * PER + i;
+      if (bb <= kBuckets) {
+        const unsigned long long vs = sm.hs[bb];
+        const int vc = sm.hc[bb];
+        sm.hs[bb] = cs;
+        sm.hc[bb] = cc;
+        cs += vs;
+        cc += vc;
+      }
+    }
+    if (lane == 31) { sm.hs[kBuckets + 1] = is; sm.hc[kBuckets + 1] = ic; }
+  }
+  __syncwarp();
+
+  const int n_vis = a.causal ? min(I + 1, a.nkb) : a.nkb;
+  auto lev_rank = [&](int r) {
+    int lev = 0;
+    for (int l = 0; l < a.levels; ++l)
+      lev += (static_cast<double>(a.thresholds[l]) <= static_cast<double>(r) / static_cast<double>(n_vis));
+    return lev;
+  };
+  auto lev_fix = [&](unsigned long long C) {
+    int lev = 0;
+    for (int l = 0; l < a.levels; ++l) lev += sm.tfx[l] <= C;
+    return lev;
+  };
+
+  // per bucket: mixed or not, the level of an unmixed one, and the start of
+  // its list group (an exclusive scan of the mixed buckets' counts)
+  int nmix;
+  {
+    int lsum = 0;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int bb = lane * PER + i;
+      if (bb <= kBuckets) {
+        const int c = sm.hc[bb + 1] - sm.hc[bb];
+        bool mx = false;
+        if (c > 0) {
+          if (a.policy == 1) {
+            mx = lev_rank(sm.hc[bb]) != lev_rank(sm.hc[bb + 1] - 1);
+          } else if (bb < kBuckets) {             // exact zeros leave the prefix unchanged
+            for (int l = 0; l < a.levels; ++l) mx |= (sm.hs[bb] < sm.tfx[l] && sm.tfx[l] <= sm.hs[bb + 1]);
+          }
+        }
+        sm.mixed[bb] = mx;
+        sm.lv[bb] = static_cast<uint8_t>(a.policy == 1 ? lev_rank(sm.hc[bb]) : lev_fix(sm.hs[bb]));
+        lsum += mx ? c : 0;
+      }
+    }
+    int incl = lsum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += y;
     }
-    const double C = carry + incl - v;
-    carry += __shfl_sync(0xffffffffu, incl, 31);
-    if (real) {
-      const int J = static_cast<int>(key[k] & 0xFFFFFFFFu);
-      const double x = a.policy == 1 ? static_cast<double>(r) / static_cast<double>(n_vis) : C;
-      int lev = 0;
-      for (int l = 0; l < a.levels; ++l) lev += (static_cast<double>(a.thresholds[l]) <= x);
-      int out = lev >= a.levels ? PSA_SKIP : lev;
-      if (a.n_dense_prefix > 0 &&
-          (static_cast<int64_t>(I) * a.block < a.n_dense_prefix || static_cast<int64_t>(J) * a.block < a.n_dense_prefix))
-        out = 0;
-      if (a.blockcos && a.cos_min > -2.f && out != PSA_SKIP && out >= 1 &&
-          a.blockcos[static_cast<int64_t>(hkv) * a.nkb + J] < a.cos_min)
-        out = 0;
-      if (a.causal) {
-        if (J > I) out = PSA_SKIP;
-        else if (J == I) out = 0;
+    nmix = __shfl_sync(0xffffffffu, incl, 31);
+    int off = incl - lsum;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int bb = lane * PER + i;
+      if (bb <= kBuckets) {
+        sm.lend[bb] = off;
+        off += sm.mixed[bb] ? sm.hc[bb + 1] - sm.hc[bb] : 0;
       }
-      a.mask[static_cast<int64_t>(row) * a.nkb + J] = static_cast<uint8_t>(out);
     }
+  }
+  __syncwarp();
+
+  // list the blocks of mixed buckets (within a group in any order)
+#pragma unroll
+  for (int k = 0; k < KPL; ++k) {
+    if (key[k] == ~0ull) continue;
+    const int bb = key_bucket(key[k]);
+    if (sm.mixed[bb]) sm.list[atomicAdd(&sm.lend[bb], 1)] = key[k];
+  }
+  __syncwarp();
+  // exact prefix / rank of every listed block from the members of its group
+  // with a smaller key
+  for (int i = lane; i < nmix; i += 32) {
+    const unsigned long long kj = sm.list[i];
+    const int bj = key_bucket(kj);
+    const int end = sm.lend[bj], beg = end - (sm.hc[bj + 1] - sm.hc[bj]);
+    unsigned long long psum = 0ull;
+    int pcnt = 0;
+    for (int j = beg; j < end; ++j) {
+      const unsigned long long kk = sm.list[j];
+      if (kk < kj) {
+        psum += mass_fix(key_mass(kk));
+        ++pcnt;
+      }
+    }
+    sm.ex[static_cast<int>(kj & 0x7FFu)] =
+        static_cast<uint8_t>(a.policy == 1 ? lev_rank(sm.hc[bj] + pcnt) : lev_fix(sm.hs[bj] + psum));
+  }
+  __syncwarp();
+
+  // levels, forced rules, the mask
+#pragma unroll
+  for (int k = 0; k < KPL; ++k) {
+    const int J = lane + 32 * k;
+    if (J >= a.nkb) continue;
+    const int bb = key_bucket(key[k]);
+    const int lev = sm.mixed[bb] ? sm.ex[J] : sm.lv[bb];
+    int out = lev >= a.levels ? PSA_SKIP : lev;
+    if (a.n_dense_prefix > 0 &&
+        (static_cast<int64_t>(I) * a.block < a.n_dense_prefix || static_cast<int64_t>(J) * a.block < a.n_dense_prefix))
+      out = 0;
+    if (a.blockcos && a.cos_min > -2.f && out != PSA_SKIP && out >= 1 &&
+        a.blockcos[static_cast<int64_t>(hkv) * a.nkb + J] < a.cos_min)
+      out = 0;
+    if (a.causal) {
+      if (J > I) out = PSA_SKIP;
+      else if (J == I) out = 0;
+    }
+    a.mask[static_cast<int64_t>(row) * a.nkb + J] = static_cast<uint8_t>(out);
   }
 }
 
@@ -838,22 +989,26 @@ cudaError_t launch_score(const CUtensorMap* mapA, const CUtensorMap* mapB, const
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t s) {
   const int rows = a.B * a.Hq * a.nqb;
-  const int wgrid = (rows + kSelWarps - 1) / kSelWarps;
   // rows_per_block <= 128 always (8 sampled rows, 1 mean row, or block / S
   // antidiagonal groups), which both kernels' row-LSE arrays rely on
   if (a.rows_per_block > 128) return cudaErrorInvalidValue;
+  auto bucket = [&](auto kpl) {
+    constexpr int KPL = decltype(kpl)::value;
+    constexpr int NW = bucket_warps(KPL);
+    select_bucket_kernel<KPL><<<(rows + NW - 1) / NW, 32 * NW, 0, s>>>(a);
+  };
   if (a.nkb <= 32) {
-    select_warp_kernel<1><<<wgrid, 32 * kSelWarps, 0, s>>>(a);
+    bucket(std::integral_constant<int, 1>());
   } else if (a.nkb <= 64) {
-    select_warp_kernel<2><<<wgrid, 32 * kSelWarps, 0, s>>>(a);
+    bucket(std::integral_constant<int, 2>());
   } else if (a.nkb <= 128) {
-    select_warp_kernel<4><<<wgrid, 32 * kSelWarps, 0, s>>>(a);
+    bucket(std::integral_constant<int, 4>());
   } else if (a.nkb <= 256) {
-    select_warp_kernel<8><<<wgrid, 32 * kSelWarps, 0, s>>>(a);
+    bucket(std::integral_constant<int, 8>());
   } else if (a.nkb <= 512) {
-    select_warp_kernel<16><<<wgrid, 32 * kSelWarps, 0, s>>>(a);
+    bucket(std::integral_constant<int, 16>());
   } else if (a.nkb <= 1024) {
-    select_warp_kernel<32><<<wgrid, 32 * kSelWarps, 0, s>>>(a);
+    bucket(std::integral_constant<int, 32>());
   } else {
     select_kernel<<<rows, kSelThreads, 0, s>>>(a);
   }
