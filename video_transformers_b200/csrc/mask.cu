@@ -28,8 +28,6 @@
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
-#include <type_traits>
-
 #include "exp2_poly.h"
 #include "internal.h"
 #include "sm100.cuh"
@@ -687,49 +685,76 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectArgs a)
 //   grouped by bucket, and each counts the members of its own group that
 //   rank before it to get its exact prefix and rank.
 // Fixed-point sums are exact for masses above 2^-39 and do not depend on
-// the order of the additions.
+// the order of the additions.  Everything per block lives in shared memory
+// (no per-block registers), so every phase is a plain loop over the blocks.
 // ----------------------------------------------------------------------------
 constexpr int kBuckets = 256;                   // plus bucket 256 for exact zeros
 constexpr int kBucketSlots = kBuckets + 2;      // slot 257 receives the totals
+constexpr int kBucketWarps = 4;                 // rows (warps) per CTA
 constexpr double kFix = 4611686018427387904.0;  // 2^62: fixed-point scale of a mass in [0, 1]
 
-// key of a block: bits [32, 64) the mass's bits inverted (descending mass =
-// ascending key), [11, 20) its bucket, [0, 11) its index.  Equal masses
-// fall in one bucket, so the bucket bits never change the order.
-__device__ __forceinline__ float key_mass(unsigned long long key) {
-  return __uint_as_float(0xFFFFFFFFu - static_cast<unsigned>(key >> 32));
-}
-__device__ __forceinline__ int key_bucket(unsigned long long key) { return static_cast<int>((key >> 11) & 0x1FFu); }
 __device__ __forceinline__ unsigned long long mass_fix(float m) {
   return static_cast<unsigned long long>(static_cast<double>(m) * kFix);
 }
+// rank order: descending mass, then ascending index (masses are >= 0, so
+// their bits order like the values)
+__device__ __forceinline__ unsigned long long rank_key(float m, int J) {
+  return (static_cast<unsigned long long>(0xFFFFFFFFu - __float_as_uint(m)) << 32) | static_cast<unsigned>(J);
+}
 
-template <int KPL>
-struct BucketRow {
-  unsigned long long list[32 * KPL];   // keys of the blocks of mixed buckets, grouped by bucket
-  unsigned long long hs[kBucketSlots]; // fixed-point mass sums, then their exclusive prefix
-  unsigned long long tfx[8];           // thresholds in fixed point
-  double rlse[128];
-  int hc[kBucketSlots];                // counts, then the exclusive rank
-  int lend[kBucketSlots];              // start of the bucket's list group, then its end
-  uint8_t ex[32 * KPL];                // exact levels of the listed blocks, by J
-  uint8_t mixed[kBucketSlots];         // a threshold falls inside the bucket
-  uint8_t lv[kBucketSlots];            // the level of every block of an unmixed bucket
+// 2^x as exp2_split, with 2^n written into the exponent field directly
+__device__ __forceinline__ double exp2_split_exp(double x) {
+  if (x < -1000.0) return 0.0;
+  const double n = floor(x);
+  float p;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(p) : "f"(static_cast<float>(x - n)));
+  return static_cast<double>(p) * __longlong_as_double(static_cast<long long>(static_cast<int>(n) + 1023) << 52);
+}
+
+// per-warp shared memory of select_bucket_kernel for P = nkb rounded up to 32
+struct BucketLayout {
+  int hs, tfx, rlse, mass, hc, lend, bk, list, ex, mixed, lv, bytes;
 };
-constexpr int bucket_warps(int kpl) { return kpl >= 16 ? 2 : 4; }
+__host__ __device__ inline BucketLayout bucket_layout(int P) {
+  BucketLayout L{};
+  int o = 0;
+  L.hs = o;    o += 8 * kBucketSlots;   // u64 fixed-point sums, then their exclusive prefix
+  L.tfx = o;   o += 8 * 8;              // u64 thresholds in fixed point
+  L.rlse = o;  o += 8 * 128;            // f64 row LSEs of the row block's score rows
+  L.mass = o;  o += 4 * P;              // f32 block masses
+  L.hc = o;    o += 4 * kBucketSlots;   // counts, then the exclusive rank
+  L.lend = o;  o += 4 * kBucketSlots;   // start of a bucket's list group, then its end
+  L.bk = o;    o += 2 * P;              // u16 bucket of every block
+  L.list = o;  o += 2 * P;              // u16 blocks of mixed buckets, grouped by bucket
+  L.ex = o;    o += P;                  // exact level of every listed block
+  L.mixed = o; o += kBucketSlots;       // a threshold falls inside the bucket
+  L.lv = o;    o += kBucketSlots;       // the level of every block of an unmixed bucket
+  L.bytes = (o + 15) & ~15;
+  return L;
+}
 
-template <int KPL>
-__global__ void __launch_bounds__(32 * bucket_warps(KPL)) select_bucket_kernel(const SelectArgs a) {
-  constexpr int NW = bucket_warps(KPL);
-  __shared__ BucketRow<KPL> rows_s[NW];
+__global__ void __launch_bounds__(32 * kBucketWarps) select_bucket_kernel(const SelectArgs a) {
+  extern __shared__ __align__(16) uint8_t sel_smem[];
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  BucketRow<KPL>& sm = rows_s[wid];
-  const int row = blockIdx.x * NW + wid;                        // (b*Hq + h)*nqb + I
+  const int row = blockIdx.x * kBucketWarps + wid;              // (b*Hq + h)*nqb + I
   if (row >= a.B * a.Hq * a.nqb) return;
+  const BucketLayout L = bucket_layout((a.nkb + 31) & ~31);
+  uint8_t* base = sel_smem + wid * L.bytes;
+  unsigned long long* hs = reinterpret_cast<unsigned long long*>(base + L.hs);
+  unsigned long long* tfx = reinterpret_cast<unsigned long long*>(base + L.tfx);
+  double* rlse = reinterpret_cast<double*>(base + L.rlse);
+  float* mass = reinterpret_cast<float*>(base + L.mass);
+  int* hc = reinterpret_cast<int*>(base + L.hc);
+  int* lend = reinterpret_cast<int*>(base + L.lend);
+  uint16_t* bk = reinterpret_cast<uint16_t*>(base + L.bk);
+  uint16_t* list = reinterpret_cast<uint16_t*>(base + L.list);
+  uint8_t* ex = base + L.ex;
+  uint8_t* mixed = base + L.mixed;
+  uint8_t* lv = base + L.lv;
+
   const int bh = row / a.nqb, I = row - bh * a.nqb;
   const int b = bh / a.Hq, h = bh - b * a.Hq;
   const int hkv = b * a.Hkv + h / (a.Hq / a.Hkv);
-
   const int rbeg = I * a.rows_per_block;
   int nvalid;
   if (a.mode == 0) {
@@ -742,59 +767,88 @@ __global__ void __launch_bounds__(32 * bucket_warps(KPL)) select_bucket_kernel(c
     const double x = a.rowlse[static_cast<int64_t>(bh) * a.rows + rbeg + s];
     const double y = a.rowlse[(static_cast<int64_t>(a.B) * a.Hq + bh) * a.rows + rbeg + s];
     const double mx = fmax(x, y);
-    sm.rlse[s] = mx == -CUDART_INF ? mx : mx + log2(exp2(x - mx) + exp2(y - mx));
+    rlse[s] = mx == -CUDART_INF ? mx : mx + log2(exp2(x - mx) + exp2(y - mx));
   }
   for (int i = lane; i < kBucketSlots; i += 32) {
-    sm.hs[i] = 0ull;
-    sm.hc[i] = 0;
+    hs[i] = 0ull;
+    hc[i] = 0;
   }
   if (lane < 8) {
     const float t = a.thresholds[lane];
-    sm.tfx[lane] = t >= 2.0f ? ~0ull : (t <= 0.0f ? 0ull : mass_fix(t));
+    tfx[lane] = t >= 2.0f ? ~0ull : (t <= 0.0f ? 0ull : mass_fix(t));
   }
   __syncwarp();
 
-  // block masses (the same arithmetic as the sorting kernels) and keys
-  unsigned long long key[KPL];
+  // block masses (the same arithmetic as select_kernel); with eight score
+  // rows the next block's rows are loaded while this one is summed
   float mmax = 0.f;
+  {
+    const float* rowbase = a.blocklse + static_cast<int64_t>(bh) * a.nkb * a.rows + rbeg;
+    const bool eight = nvalid == 8;
+    float nx[8];
+    if (eight && lane < a.nkb) {
 #pragma unroll
-  for (int k = 0; k < KPL; ++k) {
-    const int J = lane + 32 * k;
-    key[k] = ~0ull;
-    if (J < a.nkb) {
-      const float* bl = a.blocklse + (static_cast<int64_t>(bh) * a.nkb + J) * a.rows + rbeg;
+      for (int u = 0; u < 8; ++u) nx[u] = __ldg(rowbase + static_cast<int64_t>(lane) * a.rows + u);
+    }
+    for (int J = lane; J < a.nkb; J += 32) {
+      const float* bl = rowbase + static_cast<int64_t>(J) * a.rows;
       double m = 0.0;
-      for (int s = 0; s < nvalid; ++s) {
-        const float x = bl[s];
-        if (x != -CUDART_INF_F) m += exp2_split(static_cast<double>(x) - sm.rlse[s]);
+      if (eight) {
+        float cur[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) cur[u] = nx[u];
+        if (J + 32 < a.nkb) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u) nx[u] = __ldg(bl + static_cast<int64_t>(32) * a.rows + u);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (cur[u] != -CUDART_INF_F) m += exp2_split_exp(static_cast<double>(cur[u]) - rlse[u]);
+      } else {
+        // other row counts: groups of eight loads issued together, in row order
+        int s = 0;
+        for (; s + 8 <= nvalid; s += 8) {
+          float x[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) x[u] = __ldg(bl + s + u);
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            if (x[u] != -CUDART_INF_F) m += exp2_split_exp(static_cast<double>(x[u]) - rlse[s + u]);
+        }
+        for (; s < nvalid; ++s) {
+          const float x = __ldg(bl + s);
+          if (x != -CUDART_INF_F) m += exp2_split_exp(static_cast<double>(x) - rlse[s]);
+        }
       }
-      const float mass = static_cast<float>(m / nvalid);
-      if (a.mass_out) a.mass_out[static_cast<int64_t>(row) * a.nkb + J] = mass;
-      key[k] = (static_cast<unsigned long long>(0xFFFFFFFFu - __float_as_uint(mass)) << 32) | static_cast<unsigned>(J);
-      mmax = fmaxf(mmax, mass);
+      const float ms = static_cast<float>(m / nvalid);
+      if (a.mass_out) a.mass_out[static_cast<int64_t>(row) * a.nkb + J] = ms;
+      mass[J] = ms;
+      mmax = fmaxf(mmax, ms);
     }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mmax = fmaxf(mmax, __shfl_xor_sync(0xffffffffu, mmax, o));
+  __syncwarp();
 
   // buckets (monotone in the mass: the fp32 quotient and product round
   // monotonically) and the histogram.  Exact zeros (every block past the
-  // diagonal of a causal row) add nothing to the sums and are counted by one
+  // diagonal of a causal row) add nothing to the sums and are counted by a
   // ballot, not by atomics that would all hit one address.
-#pragma unroll
-  for (int k = 0; k < KPL; ++k) {
-    const bool valid = key[k] != ~0ull;
-    const float m = valid ? key_mass(key[k]) : 1.f;
+  for (int j0 = 0; j0 < a.nkb; j0 += 32) {
+    const int J = j0 + lane;
+    const bool valid = J < a.nkb;
+    const float m = valid ? mass[J] : 1.f;
     const unsigned zeros = __ballot_sync(0xffffffffu, m == 0.f);
-    if (lane == 0 && zeros) atomicAdd(&sm.hc[kBuckets], __popc(zeros));
-    if (!valid) continue;
-    int bb = kBuckets;
-    if (m != 0.f) {
-      bb = max(0, min(kBuckets - 1, static_cast<int>(floorf(static_cast<float>(kBuckets) * (1.0f - m / mmax)))));
-      atomicAdd(&sm.hc[bb], 1);
-      atomicAdd(&sm.hs[bb], mass_fix(m));
+    if (lane == 0 && zeros) atomicAdd(&hc[kBuckets], __popc(zeros));
+    if (valid) {
+      int bb = kBuckets;
+      if (m != 0.f) {
+        bb = max(0, min(kBuckets - 1, static_cast<int>(floorf(static_cast<float>(kBuckets) * (1.0f - m / mmax)))));
+        atomicAdd(&hc[bb], 1);
+        atomicAdd(&hs[bb], mass_fix(m));
+      }
+      bk[J] = static_cast<uint16_t>(bb);
     }
-    key[k] |= static_cast<unsigned long long>(bb) << 11;
   }
   __syncwarp();
 
@@ -806,7 +860,7 @@ __global__ void __launch_bounds__(32 * bucket_warps(KPL)) select_bucket_kernel(c
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
       const int bb = lane * PER + i;
-      if (bb <= kBuckets) { ls += sm.hs[bb]; lc += sm.hc[bb]; }
+      if (bb <= kBuckets) { ls += hs[bb]; lc += hc[bb]; }
     }
     unsigned long long is = ls;
     int ic = lc;
@@ -822,15 +876,15 @@ __global__ void __launch_bounds__(32 * bucket_warps(KPL)) select_bucket_kernel(c
     for (int i = 0; i < PER; ++i) {
       const int bb = lane * PER + i;
       if (bb <= kBuckets) {
-        const unsigned long long vs = sm.hs[bb];
-        const int vc = sm.hc[bb];
-        sm.hs[bb] = cs;
-        sm.hc[bb] = cc;
+        const unsigned long long vs = hs[bb];
+        const int vc = hc[bb];
+        hs[bb] = cs;
+        hc[bb] = cc;
         cs += vs;
         cc += vc;
       }
     }
-    if (lane == 31) { sm.hs[kBuckets + 1] = is; sm.hc[kBuckets + 1] = ic; }
+    if (lane == 31) { hs[kBuckets + 1] = is; hc[kBuckets + 1] = ic; }
   }
   __syncwarp();
 
@@ -843,7 +897,7 @@ __global__ void __launch_bounds__(32 * bucket_warps(KPL)) select_bucket_kernel(c
   };
   auto lev_fix = [&](unsigned long long C) {
     int lev = 0;
-    for (int l = 0; l < a.levels; ++l) lev += sm.tfx[l] <= C;
+    for (int l = 0; l < a.levels; ++l) lev += tfx[l] <= C;
     return lev;
   };
 
@@ -856,17 +910,17 @@ __global__ void __launch_bounds__(32 * bucket_warps(KPL)) select_bucket_kernel(c
     for (int i = 0; i < PER; ++i) {
       const int bb = lane * PER + i;
       if (bb <= kBuckets) {
-        const int c = sm.hc[bb + 1] - sm.hc[bb];
+        const int c = hc[bb + 1] - hc[bb];
         bool mx = false;
         if (c > 0) {
           if (a.policy == 1) {
-            mx = lev_rank(sm.hc[bb]) != lev_rank(sm.hc[bb + 1] - 1);
+            mx = lev_rank(hc[bb]) != lev_rank(hc[bb + 1] - 1);
           } else if (bb < kBuckets) {             // exact zeros leave the prefix unchanged
-            for (int l = 0; l < a.levels; ++l) mx |= (sm.hs[bb] < sm.tfx[l] && sm.tfx[l] <= sm.hs[bb + 1]);
+            for (int l = 0; l < a.levels; ++l) mx |= (hs[bb] < tfx[l] && tfx[l] <= hs[bb + 1]);
           }
         }
-        sm.mixed[bb] = mx;
-        sm.lv[bb] = static_cast<uint8_t>(a.policy == 1 ? lev_rank(sm.hc[bb]) : lev_fix(sm.hs[bb]));
+        mixed[bb] = mx;
+        lv[bb] = static_cast<uint8_t>(a.policy == 1 ? lev_rank(hc[bb]) : lev_fix(hs[bb]));
         lsum += mx ? c : 0;
       }
     }
@@ -882,48 +936,46 @@ __global__ void __launch_bounds__(32 * bucket_warps(KPL)) select_bucket_kernel(c
     for (int i = 0; i < PER; ++i) {
       const int bb = lane * PER + i;
       if (bb <= kBuckets) {
-        sm.lend[bb] = off;
-        off += sm.mixed[bb] ? sm.hc[bb + 1] - sm.hc[bb] : 0;
+        lend[bb] = off;
+        off += mixed[bb] ? hc[bb + 1] - hc[bb] : 0;
       }
     }
   }
   __syncwarp();
 
   // list the blocks of mixed buckets (within a group in any order)
-#pragma unroll
-  for (int k = 0; k < KPL; ++k) {
-    if (key[k] == ~0ull) continue;
-    const int bb = key_bucket(key[k]);
-    if (sm.mixed[bb]) sm.list[atomicAdd(&sm.lend[bb], 1)] = key[k];
-  }
-  __syncwarp();
-  // exact prefix / rank of every listed block from the members of its group
-  // with a smaller key
-  for (int i = lane; i < nmix; i += 32) {
-    const unsigned long long kj = sm.list[i];
-    const int bj = key_bucket(kj);
-    const int end = sm.lend[bj], beg = end - (sm.hc[bj + 1] - sm.hc[bj]);
-    unsigned long long psum = 0ull;
-    int pcnt = 0;
-    for (int j = beg; j < end; ++j) {
-      const unsigned long long kk = sm.list[j];
-      if (kk < kj) {
-        psum += mass_fix(key_mass(kk));
-        ++pcnt;
-      }
+  if (nmix > 0) {
+    for (int J = lane; J < a.nkb; J += 32) {
+      const int bb = bk[J];
+      if (mixed[bb]) list[atomicAdd(&lend[bb], 1)] = static_cast<uint16_t>(J);
     }
-    sm.ex[static_cast<int>(kj & 0x7FFu)] =
-        static_cast<uint8_t>(a.policy == 1 ? lev_rank(sm.hc[bj] + pcnt) : lev_fix(sm.hs[bj] + psum));
+    __syncwarp();
+    // exact prefix / rank of every listed block from the members of its
+    // group with a smaller rank key
+    for (int i = lane; i < nmix; i += 32) {
+      const int Jj = list[i];
+      const unsigned long long kj = rank_key(mass[Jj], Jj);
+      const int bj = bk[Jj];
+      const int end = lend[bj], beg = end - (hc[bj + 1] - hc[bj]);
+      unsigned long long psum = 0ull;
+      int pcnt = 0;
+      for (int j = beg; j < end; ++j) {
+        const int Jk = list[j];
+        const float mk = mass[Jk];
+        if (rank_key(mk, Jk) < kj) {
+          psum += mass_fix(mk);
+          ++pcnt;
+        }
+      }
+      ex[Jj] = static_cast<uint8_t>(a.policy == 1 ? lev_rank(hc[bj] + pcnt) : lev_fix(hs[bj] + psum));
+    }
+    __syncwarp();
   }
-  __syncwarp();
 
   // levels, forced rules, the mask
-#pragma unroll
-  for (int k = 0; k < KPL; ++k) {
-    const int J = lane + 32 * k;
-    if (J >= a.nkb) continue;
-    const int bb = key_bucket(key[k]);
-    const int lev = sm.mixed[bb] ? sm.ex[J] : sm.lv[bb];
+  for (int J = lane; J < a.nkb; J += 32) {
+    const int bb = bk[J];
+    const int lev = mixed[bb] ? ex[J] : lv[bb];
     int out = lev >= a.levels ? PSA_SKIP : lev;
     if (a.n_dense_prefix > 0 &&
         (static_cast<int64_t>(I) * a.block < a.n_dense_prefix || static_cast<int64_t>(J) * a.block < a.n_dense_prefix))
@@ -992,23 +1044,11 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t s) {
   // rows_per_block <= 128 always (8 sampled rows, 1 mean row, or block / S
   // antidiagonal groups), which both kernels' row-LSE arrays rely on
   if (a.rows_per_block > 128) return cudaErrorInvalidValue;
-  auto bucket = [&](auto kpl) {
-    constexpr int KPL = decltype(kpl)::value;
-    constexpr int NW = bucket_warps(KPL);
-    select_bucket_kernel<KPL><<<(rows + NW - 1) / NW, 32 * NW, 0, s>>>(a);
-  };
-  if (a.nkb <= 32) {
-    bucket(std::integral_constant<int, 1>());
-  } else if (a.nkb <= 64) {
-    bucket(std::integral_constant<int, 2>());
-  } else if (a.nkb <= 128) {
-    bucket(std::integral_constant<int, 4>());
-  } else if (a.nkb <= 256) {
-    bucket(std::integral_constant<int, 8>());
-  } else if (a.nkb <= 512) {
-    bucket(std::integral_constant<int, 16>());
-  } else if (a.nkb <= 1024) {
-    bucket(std::integral_constant<int, 32>());
+  if (a.nkb <= 1024) {
+    const size_t smem = static_cast<size_t>(kBucketWarps) * bucket_layout((a.nkb + 31) & ~31).bytes;
+    cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(&select_bucket_kernel), static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    select_bucket_kernel<<<(rows + kBucketWarps - 1) / kBucketWarps, 32 * kBucketWarps, smem, s>>>(a);
   } else {
     select_kernel<<<rows, kSelThreads, 0, s>>>(a);
   }
