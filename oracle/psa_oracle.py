@@ -71,6 +71,19 @@ reason in the design notes):
       the scaled values are computed in fp32; the score is the product of
       the e4m3 values times both scales.  Values and probabilities stay as
       in R1-R4.
+  R14 FP8 probabilities and values (the rest of the FP8 path; the pages say
+      no more than R13 does): the values of every level are rounded to e4m3
+      with one scale per KV head from level 0, as the keys in R13.  The
+      probabilities of a query row are P_p = 2^(a_p - M) with a_p = z_p /
+      ln 2 the logit in log2 units and M = ceil(max_p a_p), computed in fp32
+      and rounded to e4m3; the output is sum_p e4m3(P_p) V_p / sum_p P_p
+      (the normaliser sums the unrounded P), and lse is as in R1-R4.  e4m3
+      is a floating format, so moving M by a whole number of binades moves
+      every rounded P by the same power of two while the values stay in
+      its normal range (>= 2^-6): an online implementation whose running
+      reference is a whole number of binades at or below M rounds the same
+      values.  It differs only for probabilities that are below 2^-6 at
+      one reference and not at the other.
 
 Pins: every function here is checked by ``tests/test_oracle_pins.py``
 against closed forms, invariants, brute force or an independent library
@@ -496,16 +509,39 @@ def quantize_heads_e4m3(levels):
     return codes, scale
 
 
-def attention_fp8(q, kp, vp, mask, block: int, sm_scale: float, causal: bool, rows=None):
+def attention_fp8(q, kp, vp, mask, block: int, sm_scale: float, causal: bool, rows=None, pv: bool = False):
     """Adaptive pyramid attention (as :func:`attention`) with the query rows
     and the key levels replaced by their e4m3 values times their scales
-    (reading R13); values, bias and softmax unchanged.  kp / vp: the levels
-    as the attention receives them (level 0 first)."""
+    (reading R13); values, bias and softmax unchanged.  With ``pv`` the
+    value levels are rounded to e4m3 as the keys and the probabilities as
+    in reading R14.  kp / vp: the levels as the attention receives them
+    (level 0 first)."""
     qc, qs = quantize_rows_e4m3(q)
     kc, ks = quantize_heads_e4m3(kp)
     qd = e4m3_values(qc) * qs.astype(np.float64)[..., None]
     kd = [e4m3_values(c) * ks.astype(np.float64)[:, :, None, None] for c in kc]
+    if pv:
+        vc, vs = quantize_heads_e4m3(vp)
+        vd = [e4m3_values(c) * vs.astype(np.float64)[:, :, None, None] for c in vc]
+        return attention(qd, kd, vd, mask, block, sm_scale, causal, rows=rows, p_e4m3=True)
     return attention(qd, kd, [_f64(x) for x in vp], mask, block, sm_scale, causal, rows=rows)
+
+
+def softmax_pv_e4m3(z, vals) -> np.ndarray:
+    """Reading R14 for a set of query rows: z [r, n] natural-log logits
+    (-inf where masked), vals [n, d].  a = z / ln 2, M = ceil(max a) per
+    row, P = 2^(a - M) in fp32, rounded to e4m3; returns
+    sum e4m3(P) vals / sum P per row (rows with no visible key: 0)."""
+    z = np.asarray(z, dtype=np.float64)
+    a = z / LN2
+    amax = a.max(axis=1, keepdims=True) if a.shape[1] else np.full((a.shape[0], 1), -np.inf)
+    empty = ~np.isfinite(amax)
+    M = np.where(empty, 0.0, np.ceil(np.where(empty, 0.0, amax)))
+    p = np.exp2(a - M).astype(np.float32)
+    pq = e4m3_values(e4m3_codes(p))
+    den = p.astype(np.float64).sum(axis=1, keepdims=True)
+    out = (pq @ np.asarray(vals, dtype=np.float64)) / np.where(den > 0, den, 1.0)
+    return np.where(empty, 0.0, out)
 
 
 # ======================================================================================
@@ -544,7 +580,7 @@ def gather_keys(kp, vp, mask_row: Sequence[int], block: int, N: int, b: int, hk:
 
 
 def attention(q, kp, vp, mask, block: int, sm_scale: float, causal: bool,
-              rows: Optional[Iterable[Tuple[int, int, int]]] = None):
+              rows: Optional[Iterable[Tuple[int, int, int]]] = None, p_e4m3: bool = False):
     """Adaptive pyramid attention ([article] Method; [news] Methodology 4,
     ordinary scaled dot-product attention).  For query token i of block I:
 
@@ -555,7 +591,8 @@ def attention(q, kp, vp, mask, block: int, sm_scale: float, causal: bool,
     levels (level 0 first) as returned by :func:`build_pyramid`; mask
     [B, Hq, nQB, nKB].  Returns (o [B,Hq,N,d], lse [B,Hq,N]); when ``rows``
     lists (b, h, I) triples only those query blocks are computed (the rest
-    stay NaN)."""
+    stay NaN).  With ``p_e4m3`` the output's numerator uses the e4m3
+    probabilities of reading R14 (:func:`softmax_pv_e4m3`)."""
     q = _f64(q)
     mask = np.asarray(mask.cpu() if hasattr(mask, "cpu") else mask).astype(np.int64)
     B, Hq, N, d = q.shape
@@ -580,7 +617,11 @@ def attention(q, kp, vp, mask, block: int, sm_scale: float, causal: bool,
         m = np.where(empty[:, None], 0.0, m)
         e = np.exp(z - m)
         s = e.sum(axis=1)
-        o[b, h, i0:i1] = np.where(empty[:, None], 0.0, (e @ vals) / np.where(empty, 1.0, s)[:, None])
+        if p_e4m3:
+            o_rows = softmax_pv_e4m3(z, vals)
+        else:
+            o_rows = (e @ vals) / np.where(empty, 1.0, s)[:, None]
+        o[b, h, i0:i1] = np.where(empty[:, None], 0.0, o_rows)
         lse[b, h, i0:i1] = np.where(empty, -np.inf, m[:, 0] + np.log(np.where(empty, 1.0, s)))
     return o, lse
 

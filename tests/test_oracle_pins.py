@@ -37,6 +37,12 @@ something other than itself.
   e4m3_values /        saturation); decode of every byte by the format formula;
   quantize_*_e4m3 /    row and head maxima map to 448, shared level-0 key scale,
   attention_fp8         half-ulp error bound; e4m3-exact inputs give attention
+  softmax_pv_e4m3 /    hand-rounded e4m3 probabilities (e4m3_softmax_hand.json);
+  attention_fp8(pv)    exact-probability rows equal the softmax; whole-binade
+                        shifts change nothing, fractional ones do; identical
+                        keys give the bias-weighted mean by direct summation;
+                        mutations (rounded normaliser, no rounding, rounding
+                        after normalising, reference at the exact maximum)
   attention_backward /  torch autograd through torch avg_pool1d and softmax
   pool_backward         (independent routines), with and without causal
                         masking and GQA; central finite differences; all level
@@ -1099,6 +1105,115 @@ def test_mutation_head_scale_per_level(monkeypatch):
     monkeypatch.setattr(O, "quantize_heads_e4m3", bad)
     with pytest.raises(AssertionError):
         test_quantize_heads_e4m3_shares_level0_scale()
+
+
+# ======================================================================================
+# FP8 probabilities and values, reading R14
+# ======================================================================================
+
+def pin_softmax_pv_golden(golden_dir, mod=O):
+    """Largest deviation of softmax_pv_e4m3 from the hand-rounded rows."""
+    g = json.load(open(os.path.join(golden_dir, "e4m3_softmax_hand.json")))
+    worst = 0.0
+    for r in g["rows"]:
+        a = np.array(r["logits_log2"])
+        v = np.array(r["values"])[:, None]
+        den = np.sum(np.exp2(a - r["reference"]).astype(np.float32).astype(np.float64))   # P in fp32
+        want = float(np.dot(r["p_e4m3"], v[:, 0]) / den)
+        got = float(mod.softmax_pv_e4m3((a * np.log(2.0))[None, :], v)[0, 0])
+        worst = max(worst, abs(got - want) / abs(want))
+    return worst
+
+
+def test_softmax_pv_e4m3_golden(golden_dir):
+    assert pin_softmax_pv_golden(golden_dir) < 1e-14
+
+
+def test_softmax_pv_e4m3_exact_probabilities_equal_softmax():
+    """Logits a whole number of binades apart, all within 6 of the largest,
+    give probabilities that e4m3 holds exactly: the result is the plain
+    softmax times V."""
+    rng = np.random.default_rng(11)
+    a = rng.integers(-6, 1, size=(5, 9)).astype(np.float64) + 2.0
+    a[:, 0] = 2.0
+    v = rng.standard_normal((9, 3))
+    z = a * np.log(2.0)
+    e = np.exp(z - z.max(axis=1, keepdims=True))
+    want = (e @ v) / e.sum(axis=1, keepdims=True)
+    np.testing.assert_allclose(O.softmax_pv_e4m3(z, v), want, rtol=1e-13, atol=0)
+
+
+def test_softmax_pv_e4m3_binade_shifts():
+    """Moving every logit of a row by a whole number of binades changes
+    nothing while the probabilities stay in e4m3's normal range; a shift by
+    a fraction of a binade moves the rounding grid and changes the result."""
+    rng = np.random.default_rng(12)
+    a = rng.uniform(-4.5, 0.0, size=(6, 20))
+    v = rng.standard_normal((20, 4))
+    base = O.softmax_pv_e4m3(a * np.log(2.0), v)
+    for k in (-3, 1, 7):
+        np.testing.assert_array_equal(O.softmax_pv_e4m3((a + k) * np.log(2.0), v), base)
+    assert np.abs(O.softmax_pv_e4m3((a + 0.37) * np.log(2.0), v) - base).max() > 1e-4
+
+
+def test_attention_fp8_pv_uniform_keys_closed_form():
+    """Zero queries make every logit its level bias (a whole number of
+    binades), so the probabilities are powers of two (exact in e4m3);
+    values on the e4m3
+    grid with a largest magnitude of 448 keep a scale of 1, and pairs of
+    equal tokens pool to themselves.  The output is then the bias-weighted
+    mean of the values of the key set, by direct summation."""
+    rng = np.random.default_rng(13)
+    N, d, blk, L = 64, 4, 16, 2
+    grid = O.e4m3_values(np.array([c for c in range(256) if c & 0x7F != 0x7F], dtype=np.uint8))
+    grid = grid[np.abs(grid) <= 64]
+    q = np.zeros((1, 1, N, d))
+    k = rng.standard_normal((1, 1, N, d))
+    vh = rng.choice(grid, size=(1, 1, N // 2, d))
+    vh[0, 0, 0, 0] = 448.0
+    v = np.repeat(vh, 2, axis=2)
+    kl, vl = O.build_pyramid(k, v, L)
+    mask = np.array([[[[0, 1, SKIP, 1], [1, 0, 1, SKIP], [SKIP, SKIP, 0, 0], [1, 1, 1, 1]]]], dtype=np.uint8)
+    o, _ = O.attention_fp8(q, kl, vl, mask, blk, 0.3, False, pv=True)
+    for I in range(N // blk):
+        wts, vals = [], []
+        for J, lv in enumerate(mask[0, 0, I]):
+            if lv == SKIP:
+                continue
+            g = 1 << int(lv)
+            for p in range(J * blk // g, (J + 1) * blk // g):
+                wts.append(2.0 ** int(lv))
+                vals.append(vl[int(lv)][0, 0, p])
+        want = np.sum(np.array(wts)[:, None] * np.array(vals), axis=0) / np.sum(wts)
+        np.testing.assert_allclose(o[0, 0, I * blk:(I + 1) * blk], np.tile(want, (blk, 1)), rtol=1e-13, atol=1e-12)
+
+
+def _bad_softmax_pv(kind):
+    def bad(z, vals):
+        a = np.asarray(z, dtype=np.float64) / np.log(2.0)
+        amax = a.max(axis=1, keepdims=True)
+        M = amax if kind == "exact_max" else np.ceil(amax)
+        p = np.exp2(a - M).astype(np.float32)
+        pq = O.e4m3_values(O.e4m3_codes(p))
+        den = p.astype(np.float64).sum(axis=1, keepdims=True)
+        if kind == "rounded_sum":
+            return (pq @ vals) / pq.sum(axis=1, keepdims=True)
+        if kind == "no_rounding":
+            return (p.astype(np.float64) @ vals) / den
+        if kind == "round_after_normalising":
+            pn = O.e4m3_values(O.e4m3_codes((p / den).astype(np.float32)))
+            return pn @ vals
+        return (pq @ vals) / den
+    return bad
+
+
+@pytest.mark.parametrize("kind", ["rounded_sum", "no_rounding", "round_after_normalising", "exact_max"])
+def test_mutation_softmax_pv(monkeypatch, golden_dir, kind):
+    """Normalising by the rounded sum, not rounding, rounding the
+    normalised probabilities, or a reference at the exact (not whole-binade)
+    maximum each fail the hand-rounded golden."""
+    monkeypatch.setattr(O, "softmax_pv_e4m3", _bad_softmax_pv(kind))
+    assert pin_softmax_pv_golden(golden_dir, O) > 1e-3
 
 
 def test_backward_rows_filter_matches_full():
