@@ -47,8 +47,8 @@ METRIC = "PSA attn fwd ms/call & achieved TFLOP/s (executed FLOPs) vs B200 BF16 
 # ncu capture of the same workload at 4 heads scaled to the full head count (traffic grows with
 # the heads: the head-major queue keeps one head's KV in L2 at a time); valid only for the
 # attention source it was measured on, identified by its SHA-256.
-ATTN_TRAFFIC = {"wan14b": {"bytes_per_launch": 10 * (796.720384e6 + 72.149760e6),
-                           "attn_cu_sha256": "5b61d94266c01037c51aa8d054f153df9ab701c044f29eb211e1a91be54f8c3b"}}
+ATTN_TRAFFIC = {"wan14b": {"bytes_per_launch": 10 * (824.550144e6 + 72.312576e6),
+                           "attn_cu_sha256": "9465fd8804337046dccd787be24237362f6a682c1dc5d59b6e3b479e6c61bdb2"}}
 UNIT = "TFLOP/s"
 KERNELS_PER_STEP = {"pyramid": 1, "blockcos": 0, "score": 1, "select": 1, "plan": 3, "attention": 1}
 # kernels of psa_make_mask per scorer: score + select, or block means (Q, K),
@@ -528,37 +528,46 @@ def measure_backward(path, w, stream, flops_fwd, peaks_, reps=3):
 
 
 def measure_fp8(path, w, stream, flops_fwd, peaks_, reps=5):
-    """psa_attention_fwd_fp8 (e4m3 Q and K, reading R13) at the same
-    workload and mask, quantization included, and how far its output moves
-    from the bf16 path's."""
+    """psa_attention_fwd_fp8 (e4m3 Q and K, reading R13) and
+    psa_attention_fwd_fp8_pv (e4m3 probabilities and values as well,
+    reading R14) at the same workload and mask, quantization included, and
+    how far each output moves from the bf16 path's."""
     P = path.P
     if w.dtype != "bf16" or w.d != 128:
         return None
     ws = P.workspace(P.psa_attention_fp8_workspace_bytes(path.shape), path.q.device)
     out8 = torch.empty_like(path.out)
-
-    def call():
-        P.psa_attention_fwd_fp8(path.shape, path.q, path.k, path.v, path.kp, path.vp, path.mask, w.sm_scale, out8,
-                                None, ws)
-    call()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(reps):
-        call()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    st = P.psa_get_device_status(ws)
-    if st != P.PSA_OK:
-        raise RuntimeError("device status %d after the FP8 path: %s" % (st, P.psa_last_error()))
-    ms = e0.elapsed_time(e1) / reps
     path.attention()
     torch.cuda.synchronize()
-    diff = (out8.float() - path.out.float()).abs()
-    tf = flops_fwd / (ms * 1e-3) / 1e12
-    r = {"entry_point": "psa_attention_fwd_fp8", "ms": ms, "reps": reps, "tflops": tf,
-         "frac_of_burst_bf16": tf / peaks_[0], "includes": "e4m3 quantization of Q and every K level, plan, attention",
-         "vs_bf16_path": {"max_abs": diff.max().item(), "mean_abs": diff.mean().item()}}
+    ref = path.out.float()
+
+    def timed(fn):
+        def call():
+            fn(path.shape, path.q, path.k, path.v, path.kp, path.vp, path.mask, w.sm_scale, out8, None, ws)
+        call()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            call()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        st = P.psa_get_device_status(ws)
+        if st != P.PSA_OK:
+            raise RuntimeError("device status %d after the FP8 path: %s" % (st, P.psa_last_error()))
+        ms = e0.elapsed_time(e1) / reps
+        diff = (out8.float() - ref).abs()
+        tf = flops_fwd / (ms * 1e-3) / 1e12
+        return {"ms": ms, "tflops": tf, "frac_of_burst_bf16": tf / peaks_[0],
+                "vs_bf16_path": {"max_abs": diff.max().item(), "mean_abs": diff.mean().item()}}
+
+    r = {"entry_point": "psa_attention_fwd_fp8", "reps": reps,
+         "includes": "e4m3 quantization of Q and every K level, plan, attention"}
+    r.update(timed(P.psa_attention_fwd_fp8))
+    pv = {"entry_point": "psa_attention_fwd_fp8_pv",
+          "includes": "e4m3 quantization of Q and of every K and V level, plan, attention with e4m3 P"}
+    pv.update(timed(P.psa_attention_fwd_fp8_pv))
+    r["pv"] = pv
     del ws, out8
     torch.cuda.empty_cache()
     return r

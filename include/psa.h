@@ -224,6 +224,28 @@ PSA_API psa_status_t psa_attention_fwd_fp8(const psa_shape_t* shape, const void*
                                            void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * psa_attention_fwd_fp8_pv: the FP8 path with the probabilities and values
+ * in e4m3 as well (the same pages; this library's reading), so both
+ * products of the attention run on 8-bit operands.  Q and K as in
+ * psa_attention_fwd_fp8.  Every value of a KV head, at every pyramid
+ * level, is scaled by 448 / max|V| over that head's level 0 and rounded
+ * like the keys.  The probabilities of a query row are P_p = 2^(a_p - r)
+ * with a_p the logit in log2 units and r a whole number at or above the
+ * largest a_p seen so far (moved only when the maximum grows by more than
+ * 5), computed in fp32 and rounded to e4m3; because e4m3 is a floating
+ * format the rounded values do not depend on r while they stay in its
+ * normal range.  The output is v_scale[head] * sum_p e4m3(P_p) v8_p /
+ * sum_p P_p (the normaliser sums the unrounded fp32 probabilities); lse as
+ * in psa_attention_fwd.  Arguments, workspace (the same size as
+ * psa_attention_fwd_fp8's), layouts and errors as psa_attention_fwd_fp8;
+ * the values are coded into the workspace like the keys.
+ * ------------------------------------------------------------------------ */
+PSA_API psa_status_t psa_attention_fwd_fp8_pv(const psa_shape_t* shape, const void* q, const void* k, const void* v,
+                                              const void* k_pyr, const void* v_pyr, const uint8_t* mask,
+                                              float sm_scale, void* out, float* lse,
+                                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * Backward pass of stage 3 (the pages give none; news review, Methodology
  * 4, says the model trains end to end through the pooled attention, and the
  * summary article, Results, pairs PSA with distillation).  The derivative

@@ -194,6 +194,9 @@ def test_fp8_path_rejects_unsupported_shapes():
     st = P.lib().psa_attention_fwd_fp8(ctypes.byref(s64), *([ctypes.c_void_p(16)] * 6), ctypes.c_float(0.1),
                                        ctypes.c_void_p(16), None, ctypes.c_void_p(16), 1 << 30, None)
     assert st == P.PSA_ERR_UNSUPPORTED and "128" in P.psa_last_error()
+    st = P.lib().psa_attention_fwd_fp8_pv(ctypes.byref(s64), *([ctypes.c_void_p(16)] * 6), ctypes.c_float(0.1),
+                                          ctypes.c_void_p(16), None, ctypes.c_void_p(16), 1 << 30, None)
+    assert st == P.PSA_ERR_UNSUPPORTED and "128" in P.psa_last_error()
     sf = P.make_shape(1, 2, 2, 256, 128, 64, 4, dtype=P.PSA_DT_FP32)
     assert P.psa_attention_fp8_workspace_bytes(sf) == 0
     assert P.psa_attention_fp8_workspace_bytes(P.make_shape(1, 2, 2, 256, 128, 64, 4)) > 0

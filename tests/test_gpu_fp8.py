@@ -6,7 +6,22 @@
   operands (attention_fp8, fed the GPU's pyramid), with the bf16 path's
   tolerances (max-abs 2e-2, mean-abs 2e-3): the FP8 kernel's own arithmetic
   is the bf16 kernel's.  The accuracy cost of the rounding itself (against
-  the plain oracle attention) is reported, not bounded."""
+  the plain oracle attention) is reported, not bounded.
+* psa_attention_fwd_fp8_pv (reading R14: e4m3 probabilities and values)
+  against attention_fp8(pv=True).  The kernel's reference for the
+  probabilities is a whole binade at most 5 below the oracle's; e4m3
+  rounding is the same at both while a probability is in e4m3's normal
+  range, so:
+  - where every logit of a row lies within 5 binades of the row's largest
+    (small queries and keys, two levels), the two agree up to the bf16
+    output rounding (2^-9 relative) and rare one-step flips of a rounded
+    probability from the special-function unit's exp2 error near an e4m3
+    midpoint (each moves an output by at most 2^-4 |V| / sum P): every
+    element within 2^-8 |o| + 2e-3, mean-abs 4e-4;
+  - elsewhere probabilities below 2^-6 at one reference and not at the
+    other round differently.  Emulating the reference 1..5 binades lower
+    on rows of 1000 Gaussian logits (standard deviation 1-4) moved outputs
+    by at most 3.2e-2 (mean 2.8e-3): max-abs 5e-2, mean-abs 5e-3."""
 import numpy as np
 import pytest
 import torch
@@ -28,13 +43,17 @@ def gen(seed):
     return g
 
 
-def run_fp8(shape, q, k, v, kp, vp, mask, sm_scale):
+PV_EXACT_ABS, PV_EXACT_MEAN = 2e-3, 4e-4
+PV_MAX, PV_MEAN = 5e-2, 5e-3
+
+
+def run_fp8(shape, q, k, v, kp, vp, mask, sm_scale, pv=False):
     out = torch.empty_like(q)
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
     ws = P.workspace(P.psa_attention_fp8_workspace_bytes(shape), q.device)
     L1 = shape.levels > 1
-    P.psa_attention_fwd_fp8(shape, q, k, v, kp if L1 else None, vp if L1 else None, mask.contiguous(), sm_scale, out,
-                            lse, ws)
+    fn = P.psa_attention_fwd_fp8_pv if pv else P.psa_attention_fwd_fp8
+    fn(shape, q, k, v, kp if L1 else None, vp if L1 else None, mask.contiguous(), sm_scale, out, lse, ws)
     st = P.psa_get_device_status(ws)
     assert st == P.PSA_OK, P.psa_last_error()
     torch.cuda.synchronize()
@@ -122,4 +141,91 @@ def test_fp8_attention_generated_masks(name, grid, heads):
     o, _ = O.attention(q, kl, vl, mask.cpu(), w.block, w.sm_scale, w.causal)
     cmx, cmean, _ = attn_errors(out, o)
     note("fp8 %s: vs the e4m3 oracle max %.2e mean %.2e; cost vs plain attention max %.3f mean %.4f"
+         % (name, mx, mean, cmx, cmean))
+
+
+@pytest.mark.parametrize("block,causal,N,heads", [(128, False, 1000, (2, 1)), (128, True, 520, (4, 2)),
+                                                  (64, True, 456, (2, 2)), (64, False, 300, (3, 1))])
+def test_fp8_pv_exact_regime(block, causal, N, heads):
+    """Small queries and keys (logits with a standard deviation of 0.25)
+    and two levels keep every logit of a row within 5 binades of its
+    largest: no probability leaves e4m3's normal range at either reference."""
+    g = gen(31)
+    Hq, Hkv = heads
+    d, B, L = 128, 2, 2
+    q = (torch.randn(B, Hq, N, d, generator=g) * 0.5).bfloat16().to(DEV)
+    k = (torch.randn(B, Hkv, N, d, generator=g) * 0.5).bfloat16().to(DEV)
+    v = torch.randn(B, Hkv, N, d, generator=g).bfloat16().to(DEV)
+    nb = -(-N // block)
+    m = torch.randint(0, L + 1, (B, Hq, nb, nb), generator=g)
+    mask = torch.where(m == L, torch.full_like(m, SKIP), m).to(torch.uint8)
+    shape = P.make_shape(B, Hq, Hkv, N, d, block, L, causal)
+    kp, vp, _ = run_pyramid(shape, k, v)
+    out, lse = run_fp8(shape, q, k, v, kp, vp, mask.to(DEV), d ** -0.5, pv=True)
+    kl, vl = levels_of(shape, kp, k), levels_of(shape, vp, v)
+    o8, l8 = O.attention_fp8(q, [x.astype(np.float32) for x in kl], [x.astype(np.float32) for x in vl], mask, block,
+                             d ** -0.5, causal, pv=True)
+    mx, mean, _ = attn_errors(out, o8)
+    # elementwise: the bf16 rounding of the output (relative) plus the flips
+    err = np.abs(out.double().cpu().numpy() - o8)
+    bound = 2.0 ** -8 * np.abs(o8) + PV_EXACT_ABS
+    assert np.all(err <= bound), (float((err - bound).max()), mx)
+    assert mean <= PV_EXACT_MEAN, mean
+    lg = lse.cpu().numpy().astype(np.float64)
+    fin = np.isfinite(l8)
+    assert np.all(np.isneginf(lg[~fin])) and np.abs(lg[fin] - l8[fin]).max() <= 2e-2
+    note("fp8 P.V exact regime block %d causal %s: vs the e4m3 oracle max %.2e mean %.2e" % (block, causal, mx, mean))
+
+
+@pytest.mark.parametrize("block,causal,L,N,heads", [
+    (128, False, 4, 1000, (2, 1)),
+    (128, True, 4, 520, (4, 2)),
+    (64, True, 4, 456, (2, 2)),
+    (64, False, 3, 300, (3, 1)),
+    (128, False, 1, 256, (1, 1)),
+])
+def test_fp8_pv_random_masks(block, causal, L, N, heads):
+    g = gen(41)
+    Hq, Hkv = heads
+    d, B = 128, 2
+    q = torch.randn(B, Hq, N, d, generator=g).bfloat16().to(DEV)
+    k = torch.randn(B, Hkv, N, d, generator=g).bfloat16().to(DEV)
+    v = torch.randn(B, Hkv, N, d, generator=g).bfloat16().to(DEV)
+    nb = -(-N // block)
+    m = torch.randint(0, L + 1, (B, Hq, nb, nb), generator=g)
+    mask = torch.where(m == L, torch.full_like(m, SKIP), m).to(torch.uint8)
+    mask[0, 0, 0] = SKIP
+    shape = P.make_shape(B, Hq, Hkv, N, d, block, L, causal)
+    kp, vp, _ = run_pyramid(shape, k, v)
+    out, _ = run_fp8(shape, q, k, v, kp, vp, mask.to(DEV), d ** -0.5, pv=True)
+    kl = levels_of(shape, kp, k) if L > 1 else [k.double().cpu().numpy()]
+    vl = levels_of(shape, vp, v) if L > 1 else [v.double().cpu().numpy()]
+    o8, _ = O.attention_fp8(q, [x.astype(np.float32) for x in kl], [x.astype(np.float32) for x in vl], mask, block,
+                            d ** -0.5, causal, pv=True)
+    mx, mean, _ = attn_errors(out, o8)
+    assert mx <= PV_MAX and mean <= PV_MEAN, (mx, mean)
+    o, _ = O.attention(q, kl, vl, mask, block, d ** -0.5, causal)
+    cmx, cmean, _ = attn_errors(out, o)
+    note("fp8 P.V block %d causal %s: vs the e4m3 oracle max %.2e mean %.2e; cost vs plain attention max %.3f mean %.4f"
+         % (block, causal, mx, mean, cmx, cmean))
+    assert torch.all(out[0, 0, :min(block, N)] == 0)
+
+
+@pytest.mark.parametrize("name,grid,heads", [("wan14b", (4, 12, 16), (2, 2)), ("qwen2.5vl", (6, 8, 16), (7, 1))])
+def test_fp8_pv_generated_masks(name, grid, heads):
+    w = W.reduced(name, grid=grid, heads=heads)
+    q, k, v, _ = W.make_qkv(w, device="cpu")
+    q, k, v = q.to(DEV), k.to(DEV), v.to(DEV)
+    shape = shape_for(w)
+    kp, vp, bc = run_pyramid(shape, k, v, with_cos=w.cos_min > -2)
+    mask, _ = run_mask(shape, params_for(w), q, k, bc)
+    out, _ = run_fp8(shape, q, k, v, kp, vp, mask, w.sm_scale, pv=True)
+    kl, vl = levels_of(shape, kp, k), levels_of(shape, vp, v)
+    o8, _ = O.attention_fp8(q, [x.astype(np.float32) for x in kl], [x.astype(np.float32) for x in vl], mask.cpu(),
+                            w.block, w.sm_scale, w.causal, pv=True)
+    mx, mean, _ = attn_errors(out, o8)
+    assert mx <= PV_MAX and mean <= PV_MEAN, (mx, mean)
+    o, _ = O.attention(q, kl, vl, mask.cpu(), w.block, w.sm_scale, w.causal)
+    cmx, cmean, _ = attn_errors(out, o)
+    note("fp8 P.V %s: vs the e4m3 oracle max %.2e mean %.2e; cost vs plain attention max %.3f mean %.4f"
          % (name, mx, mean, cmx, cmean))

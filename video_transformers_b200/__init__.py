@@ -30,7 +30,7 @@ EXPORTS = [
     "psa_mask_workspace_bytes", "psa_make_mask",
     "psa_attention_workspace_bytes", "psa_attention_fwd", "psa_attention_fwd_static", "psa_attention_plan_stats",
     "psa_attention_bwd_workspace_bytes", "psa_attention_bwd",
-    "psa_quantize_qk_fp8", "psa_attention_fp8_workspace_bytes", "psa_attention_fwd_fp8",
+    "psa_quantize_qk_fp8", "psa_attention_fp8_workspace_bytes", "psa_attention_fwd_fp8", "psa_attention_fwd_fp8_pv",
     "psa_get_device_status", "psa_get_static_device_status", "psa_debug_wait_control",
     "psa_last_error", "psa_version",
 ]
@@ -75,6 +75,7 @@ def _load(path: str = LIB_PATH):
         "psa_quantize_qk_fp8": (I, [S, P, P, P, P, P, P, P, P, P]),
         "psa_attention_fp8_workspace_bytes": (Z, [S]),
         "psa_attention_fwd_fp8": (I, [S, P, P, P, P, P, P, F, P, P, P, Z, P]),
+        "psa_attention_fwd_fp8_pv": (I, [S, P, P, P, P, P, P, F, P, P, P, Z, P]),
         "psa_attention_bwd": (I, [S, P, P, P, P, P, P, F, P, P, P, P, P, P, P, Z, P]),
         "psa_attention_plan_stats": (I, [S, P, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64), P]),
         "psa_get_device_status": (I, [P, P]),
@@ -219,6 +220,16 @@ def psa_attention_fwd_fp8(shape: Shape, q, k, v, k_pyr, v_pyr, mask, sm_scale: f
                                        ctypes.c_float(sm_scale), _ptr(out, "out"), _ptr(lse, "lse", False),
                                        _ptr(workspace, "workspace"), workspace.numel() * workspace.element_size(),
                                        _stream(stream)))
+
+
+def psa_attention_fwd_fp8_pv(shape: Shape, q, k, v, k_pyr, v_pyr, mask, sm_scale: float, out, lse, workspace,
+                             stream=None):
+    L1 = shape.levels > 1
+    _check(lib().psa_attention_fwd_fp8_pv(ctypes.byref(shape), _ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"),
+                                          _ptr(k_pyr, "k_pyr", L1), _ptr(v_pyr, "v_pyr", L1), _ptr(mask, "mask"),
+                                          ctypes.c_float(sm_scale), _ptr(out, "out"), _ptr(lse, "lse", False),
+                                          _ptr(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+                                          _stream(stream)))
 
 
 def psa_attention_bwd_workspace_bytes(shape: Shape) -> int:

@@ -353,7 +353,7 @@ BwdLayout bwd_layout(const psa_shape_t* s) {
 // ------------------------------------------------------------------ FP8 workspace
 struct Fp8Layout {
   AttnLayout fwd;                  // the tile plan, at the start of the workspace
-  size_t q8, qs, k8, kp8, ks, total;
+  size_t q8, qs, k8, kp8, ks, v8, vp8, vs, total;
 };
 Fp8Layout fp8_layout(const psa_shape_t* s) {
   Fp8Layout L{};
@@ -365,6 +365,9 @@ Fp8Layout fp8_layout(const psa_shape_t* s) {
   L.k8 = off;  off = align_up(off + BHkv * s->N * s->d, 256);
   L.kp8 = off; off = align_up(off + pyr_bytes(s, 1), 256);
   L.ks = off;  off = align_up(off + BHkv * 4, 256);
+  L.v8 = off;  off = align_up(off + BHkv * s->N * s->d, 256);      // e4m3 values (the P.V path only)
+  L.vp8 = off; off = align_up(off + pyr_bytes(s, 1), 256);
+  L.vs = off;  off = align_up(off + BHkv * 4, 256);
   L.total = off;
   return L;
 }
@@ -373,6 +376,97 @@ psa_status_t check_fp8_shape(const psa_shape_t* s) {
   PSA_TRY(check_shape(s));
   if (s->dtype != PSA_DT_BF16) return fail(PSA_ERR_UNSUPPORTED, "the FP8 path takes bf16 tensors");
   if (s->d != 128) return fail(PSA_ERR_UNSUPPORTED, "the FP8 path is built for head dim 128");
+  return PSA_OK;
+}
+
+psa_status_t attention_fp8(const psa_shape_t* s, const void* q, const void* k, const void* v, const void* k_pyr,
+                           const void* v_pyr, const uint8_t* mask, float sm_scale, void* out, float* lse, void* ws,
+                           size_t ws_bytes, void* stream, bool pv) {
+  g_err[0] = 0;
+  PSA_TRY(check_fp8_shape(s));
+  PSA_TRY(check_ptr(q, "q"));
+  PSA_TRY(check_ptr(k, "k"));
+  PSA_TRY(check_ptr(v, "v"));
+  PSA_TRY(check_ptr(out, "out"));
+  if (s->levels > 1) {
+    PSA_TRY(check_ptr(k_pyr, "k_pyr"));
+    PSA_TRY(check_ptr(v_pyr, "v_pyr"));
+  }
+  if (!mask) return fail(PSA_ERR_INVALID_ARG, "mask is NULL");
+  PSA_TRY(check_ptr(lse, "lse", false));
+  if (!(sm_scale > 0.f) || sm_scale != sm_scale) return fail(PSA_ERR_INVALID_ARG, "sm_scale must be > 0");
+  const Fp8Layout L = fp8_layout(s);
+  if (L.fwd.max_segs >= (1ll << 31) || L.fwd.max_tiles >= (1ll << 31))
+    return fail(PSA_ERR_UNSUPPORTED, "tile plan would exceed 2^31 entries");
+  if (!ws || !aligned16(ws)) return fail(PSA_ERR_WORKSPACE, "workspace is NULL or not 16-byte aligned");
+  if (ws_bytes < L.total) return fail(PSA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, L.total);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  const int64_t BHq = static_cast<int64_t>(s->B) * s->Hq, BHkv = static_cast<int64_t>(s->B) * s->Hkv;
+  uint8_t* q8 = reinterpret_cast<uint8_t*>(w + L.q8);
+  uint8_t* k8 = reinterpret_cast<uint8_t*>(w + L.k8);
+  uint8_t* kp8 = reinterpret_cast<uint8_t*>(w + L.kp8);
+  float* qs = reinterpret_cast<float*>(w + L.qs);
+  float* ks = reinterpret_cast<float*>(w + L.ks);
+  size_t off[PSA_MAX_LEVELS] = {0, 0, 0, 0};
+  for (int l = 1; l < s->levels; ++l) off[l] = pyr_level_offset(s, l, 1);
+  PSA_CUDA(psa::launch_quantize_qk_fp8(q, k, k_pyr, off, BHq, BHkv, s->N, s->d, s->levels, q8, qs, k8, kp8, ks, st),
+           "fp8 quantize launch");
+  uint8_t* v8 = reinterpret_cast<uint8_t*>(w + L.v8);
+  uint8_t* vp8 = reinterpret_cast<uint8_t*>(w + L.vp8);
+  float* vs = reinterpret_cast<float*>(w + L.vs);
+  if (pv)
+    PSA_CUDA(psa::launch_quantize_heads_fp8(v, v_pyr, off, BHkv, s->N, s->d, s->levels, v8, vp8, vs, st),
+             "fp8 value quantize launch");
+  CUtensorMap maps[9];
+  PSA_TRY(map3_u8(&maps[0], q8, BHq, s->N, s->d, 128));
+  const char* vp = static_cast<const char*>(v_pyr);
+  for (int l = 0; l < s->levels; ++l) {
+    const void* kb = l == 0 ? static_cast<const void*>(k8) : static_cast<const void*>(kp8 + off[l]);
+    const void* vb = l == 0 ? v : static_cast<const void*>(vp + pyr_level_offset(s, l, 2));
+    const int box = (s->block >> l) < 64 ? (s->block >> l) : 64;
+    PSA_TRY(map3_u8(&maps[1 + l], kb, BHkv, s->N >> l, s->d, box));
+    if (pv) {
+      const void* vb8 = l == 0 ? static_cast<const void*>(v8) : static_cast<const void*>(vp8 + off[l]);
+      PSA_TRY(map3_u8(&maps[1 + s->levels + l], vb8, BHkv, s->N >> l, s->d, box));
+    } else {
+      PSA_TRY(map3(&maps[1 + s->levels + l], vb, BHkv, s->N >> l, s->d, box));
+    }
+  }
+  const int nkb = static_cast<int>(ceil_div(s->N, s->block));
+  psa::PlanArgs pa{};
+  pa.B = s->B; pa.Hq = s->Hq; pa.N = s->N; pa.block = s->block; pa.nqb = nkb; pa.nkb = nkb;
+  pa.levels = s->levels; pa.causal = s->causal != 0; pa.n_items = L.fwd.n_items; pa.mask = mask;
+  pa.item_nseg = reinterpret_cast<int*>(w + L.fwd.nseg);
+  pa.item_ntile = reinterpret_cast<int*>(w + L.fwd.ntile);
+  pa.item_rows = reinterpret_cast<int*>(w + L.fwd.nrows);
+  pa.item_seg_off = reinterpret_cast<int*>(w + L.fwd.seg_off);
+  pa.item_tile_off = reinterpret_cast<int*>(w + L.fwd.tile_off);
+  pa.tile_seg_off = reinterpret_cast<int*>(w + L.fwd.tile_seg_off);
+  pa.segs = reinterpret_cast<int*>(w + L.fwd.segs);
+  pa.queue = reinterpret_cast<int*>(w + L.fwd.queue);
+  pa.hist = reinterpret_cast<int*>(w + L.fwd.hist);
+  pa.n_hist = L.fwd.n_hist;
+  pa.lpt_queue = 0;
+  pa.stats = reinterpret_cast<long long*>(w + L.fwd.stats);
+  PSA_CUDA(psa::launch_plan(pa, st), "plan launch");
+  psa::AttnArgs aa{};
+  aa.B = s->B; aa.Hq = s->Hq; aa.Hkv = s->Hkv; aa.N = s->N; aa.d = s->d; aa.block = s->block;
+  aa.levels = s->levels; aa.causal = s->causal != 0; aa.n_items = L.fwd.n_items; aa.n_qtiles = L.fwd.n_qtiles;
+  aa.scale_log2 = sm_scale * 1.4426950408889634f;
+  aa.item_tile_off = pa.item_tile_off;
+  aa.item_rows = pa.item_rows;
+  aa.tile_seg_off = pa.tile_seg_off;
+  aa.segs = pa.segs;
+  aa.queue = pa.queue;
+  aa.out = out;
+  aa.out_fp32 = 0;
+  aa.lse = lse;
+  aa.status = reinterpret_cast<int*>(w + L.fwd.status);
+  aa.qscale = qs;
+  aa.kscale = ks;
+  aa.vscale = pv ? vs : nullptr;
+  PSA_CUDA(psa::launch_attention_fp8(maps, aa, pv, num_sms(), st), "fp8 attention launch");
   return PSA_OK;
 }
 
@@ -747,80 +841,13 @@ size_t psa_attention_fp8_workspace_bytes(const psa_shape_t* s) {
 psa_status_t psa_attention_fwd_fp8(const psa_shape_t* s, const void* q, const void* k, const void* v,
                                    const void* k_pyr, const void* v_pyr, const uint8_t* mask, float sm_scale,
                                    void* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
-  g_err[0] = 0;
-  PSA_TRY(check_fp8_shape(s));
-  PSA_TRY(check_ptr(q, "q"));
-  PSA_TRY(check_ptr(k, "k"));
-  PSA_TRY(check_ptr(v, "v"));
-  PSA_TRY(check_ptr(out, "out"));
-  if (s->levels > 1) {
-    PSA_TRY(check_ptr(k_pyr, "k_pyr"));
-    PSA_TRY(check_ptr(v_pyr, "v_pyr"));
-  }
-  if (!mask) return fail(PSA_ERR_INVALID_ARG, "mask is NULL");
-  PSA_TRY(check_ptr(lse, "lse", false));
-  if (!(sm_scale > 0.f) || sm_scale != sm_scale) return fail(PSA_ERR_INVALID_ARG, "sm_scale must be > 0");
-  const Fp8Layout L = fp8_layout(s);
-  if (L.fwd.max_segs >= (1ll << 31) || L.fwd.max_tiles >= (1ll << 31))
-    return fail(PSA_ERR_UNSUPPORTED, "tile plan would exceed 2^31 entries");
-  if (!ws || !aligned16(ws)) return fail(PSA_ERR_WORKSPACE, "workspace is NULL or not 16-byte aligned");
-  if (ws_bytes < L.total) return fail(PSA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, L.total);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  char* w = static_cast<char*>(ws);
-  const int64_t BHq = static_cast<int64_t>(s->B) * s->Hq, BHkv = static_cast<int64_t>(s->B) * s->Hkv;
-  uint8_t* q8 = reinterpret_cast<uint8_t*>(w + L.q8);
-  uint8_t* k8 = reinterpret_cast<uint8_t*>(w + L.k8);
-  uint8_t* kp8 = reinterpret_cast<uint8_t*>(w + L.kp8);
-  float* qs = reinterpret_cast<float*>(w + L.qs);
-  float* ks = reinterpret_cast<float*>(w + L.ks);
-  size_t off[PSA_MAX_LEVELS] = {0, 0, 0, 0};
-  for (int l = 1; l < s->levels; ++l) off[l] = pyr_level_offset(s, l, 1);
-  PSA_CUDA(psa::launch_quantize_qk_fp8(q, k, k_pyr, off, BHq, BHkv, s->N, s->d, s->levels, q8, qs, k8, kp8, ks, st),
-           "fp8 quantize launch");
-  CUtensorMap maps[9];
-  PSA_TRY(map3_u8(&maps[0], q8, BHq, s->N, s->d, 128));
-  const char* vp = static_cast<const char*>(v_pyr);
-  for (int l = 0; l < s->levels; ++l) {
-    const void* kb = l == 0 ? static_cast<const void*>(k8) : static_cast<const void*>(kp8 + off[l]);
-    const void* vb = l == 0 ? v : static_cast<const void*>(vp + pyr_level_offset(s, l, 2));
-    const int box = (s->block >> l) < 64 ? (s->block >> l) : 64;
-    PSA_TRY(map3_u8(&maps[1 + l], kb, BHkv, s->N >> l, s->d, box));
-    PSA_TRY(map3(&maps[1 + s->levels + l], vb, BHkv, s->N >> l, s->d, box));
-  }
-  const int nkb = static_cast<int>(ceil_div(s->N, s->block));
-  psa::PlanArgs pa{};
-  pa.B = s->B; pa.Hq = s->Hq; pa.N = s->N; pa.block = s->block; pa.nqb = nkb; pa.nkb = nkb;
-  pa.levels = s->levels; pa.causal = s->causal != 0; pa.n_items = L.fwd.n_items; pa.mask = mask;
-  pa.item_nseg = reinterpret_cast<int*>(w + L.fwd.nseg);
-  pa.item_ntile = reinterpret_cast<int*>(w + L.fwd.ntile);
-  pa.item_rows = reinterpret_cast<int*>(w + L.fwd.nrows);
-  pa.item_seg_off = reinterpret_cast<int*>(w + L.fwd.seg_off);
-  pa.item_tile_off = reinterpret_cast<int*>(w + L.fwd.tile_off);
-  pa.tile_seg_off = reinterpret_cast<int*>(w + L.fwd.tile_seg_off);
-  pa.segs = reinterpret_cast<int*>(w + L.fwd.segs);
-  pa.queue = reinterpret_cast<int*>(w + L.fwd.queue);
-  pa.hist = reinterpret_cast<int*>(w + L.fwd.hist);
-  pa.n_hist = L.fwd.n_hist;
-  pa.lpt_queue = 0;
-  pa.stats = reinterpret_cast<long long*>(w + L.fwd.stats);
-  PSA_CUDA(psa::launch_plan(pa, st), "plan launch");
-  psa::AttnArgs aa{};
-  aa.B = s->B; aa.Hq = s->Hq; aa.Hkv = s->Hkv; aa.N = s->N; aa.d = s->d; aa.block = s->block;
-  aa.levels = s->levels; aa.causal = s->causal != 0; aa.n_items = L.fwd.n_items; aa.n_qtiles = L.fwd.n_qtiles;
-  aa.scale_log2 = sm_scale * 1.4426950408889634f;
-  aa.item_tile_off = pa.item_tile_off;
-  aa.item_rows = pa.item_rows;
-  aa.tile_seg_off = pa.tile_seg_off;
-  aa.segs = pa.segs;
-  aa.queue = pa.queue;
-  aa.out = out;
-  aa.out_fp32 = 0;
-  aa.lse = lse;
-  aa.status = reinterpret_cast<int*>(w + L.fwd.status);
-  aa.qscale = qs;
-  aa.kscale = ks;
-  PSA_CUDA(psa::launch_attention_fp8(maps, aa, num_sms(), st), "fp8 attention launch");
-  return PSA_OK;
+  return attention_fp8(s, q, k, v, k_pyr, v_pyr, mask, sm_scale, out, lse, ws, ws_bytes, stream, false);
+}
+
+psa_status_t psa_attention_fwd_fp8_pv(const psa_shape_t* s, const void* q, const void* k, const void* v,
+                                      const void* k_pyr, const void* v_pyr, const uint8_t* mask, float sm_scale,
+                                      void* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  return attention_fp8(s, q, k, v, k_pyr, v_pyr, mask, sm_scale, out, lse, ws, ws_bytes, stream, true);
 }
 
 psa_status_t psa_attention_plan_stats(const psa_shape_t* s, const void* ws, int64_t* n_tiles, int64_t* n_rows,

@@ -39,6 +39,9 @@ namespace {
 constexpr int kThreads = 192;
 constexpr int kSub = 64;                    // KV rows per sub-tile
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: P stays <= 2^(8+3)
+// With e4m3 probabilities the reference max moves in whole binades and at
+// most 5 below the running max, so P <= 2^(5+3) stays under e4m3's 448.
+constexpr float kRescaleThresholdP8 = 5.0f;
 // Of every 8 column pairs of a full sub-tile, this many take their
 // exponential on the FMA pipe (exp2_fma2) instead of the special-function
 // unit.  Measured on B200 the special-function unit is not the limit of
@@ -119,6 +122,44 @@ __device__ __forceinline__ float sub_probs(const float* s, float sc, const float
   return t.x + t.y;
 }
 
+// two fp32 values as e4m3 codes (nearest, ties to even, saturating): lo in
+// the low byte, hi in the high byte
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// sub_probs with the probabilities rounded to e4m3, four per 32-bit word
+// (column c in byte c % 4 of word c / 4: the 8-bit A-operand layout of a TS
+// MMA); returns the sum of the unrounded fp32 probabilities
+__device__ __forceinline__ float sub_probs8(const float* s, float sc, const float (&cb)[4], float mu,
+                                            uint32_t (&pk)[16]) {
+  const float2 sc2 = make_float2(sc, sc);
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float2 off = make_float2(cb[k] - mu, cb[k] - mu);
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      const float2 x0 = __ffma2_rn(make_float2(s[16 * k + 2 * i], s[16 * k + 2 * i + 1]), sc2, off);
+      const float2 x1 = __ffma2_rn(make_float2(s[16 * k + 2 * i + 2], s[16 * k + 2 * i + 3]), sc2, off);
+      const float2 p0 = make_float2(fast_exp2(x0.x), fast_exp2(x0.y));
+      const float2 p1 = make_float2(fast_exp2(x1.x), fast_exp2(x1.y));
+      acc[i & 3] = __fadd2_rn(acc[i & 3], p0);
+      acc[(i + 1) & 3] = __fadd2_rn(acc[(i + 1) & 3], p1);
+      pk[4 * k + i / 2] = e4m3x2(p0.x, p0.y) | (e4m3x2(p1.x, p1.y) << 16);
+    }
+  }
+  const float2 t = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+  return t.x + t.y;
+}
+
+// 2^x for a whole number x <= 0, exactly (0 below the normal range)
+__device__ __forceinline__ float exp2_whole(float x) {
+  return x < -126.0f ? 0.0f : __int_as_float((127 + static_cast<int>(x)) << 23);
+}
+
 // number of 64-row sub-tiles of an item with `rows` real KV rows
 __device__ __forceinline__ uint32_t sub_count(int rows) { return static_cast<uint32_t>((rows + kSub - 1) / kSub); }
 
@@ -129,13 +170,19 @@ __device__ __forceinline__ uint32_t sub_count(int rows) { return static_cast<uin
 // one 128-byte-swizzled chunk), S = Q K^T runs as kind::f8f6f4 MMAs (K = 32
 // per instruction), and the softmax scale of a row carries the row's query
 // scale times its KV head's key scale; V, P and O are as in the bf16 path.
-template <int D, bool OUT_F32, int NST, int CTAS, bool H2, bool QK8 = false>
+// PV8 (with QK8): V arrives as e4m3 codes too (one 128-byte-swizzled chunk
+// per 64-row stage) and O += P V runs as kind::f8f6f4 MMAs (K = 32) with P
+// as e4m3 in TMEM and V as an MN-major B operand; the reference max moves
+// in whole binades (P's e4m3 rounding then does not depend on when it
+// moved), and the output carries the KV head's value scale.
+template <int D, bool OUT_F32, int NST, int CTAS, bool H2, bool QK8 = false, bool PV8 = false>
 __global__ void __launch_bounds__(kThreads, CTAS)
     attn_kernel(const __grid_constant__ AttnMaps maps, const AttnArgs a) {
   static_assert(!QK8 || D == 128, "the FP8 path is built for d = 128");
+  static_assert(!PV8 || QK8, "e4m3 probabilities come with e4m3 queries and keys");
   constexpr int QB = QK8 ? D * 128 : D * 256;    // bytes of the 128-row Q tile
   constexpr int SBK = QK8 ? D * 64 : D * 128;    // bytes of a 64-row K stage
-  constexpr int SB = D * 128;                    // bytes of a 64-row V stage
+  constexpr int SB = PV8 ? D * 64 : D * 128;     // bytes of a 64-row V stage
   constexpr int KC = D / 64;                     // 64-channel bf16 chunks
   constexpr uint32_t kTmemCols = 256;
   using Shared = AttnShared<NST>;
@@ -288,10 +335,15 @@ __global__ void __launch_bounds__(kThreads, CTAS)
           if (lane == 0) mbar_arrive_expect_tx(smem_u32(&sh->v_full[pst]), SB);
           __syncwarp();
           if (pv_mine) {
+            if (PV8) {
+              tma_load_3d(smem_u32(sV + pst * SB + pv_dst * 128), &maps.m[1 + L + pv_l], smem_u32(&sh->v_full[pst]), 0,
+                          pv_prow, hkv);
+            } else {
 #pragma unroll
-            for (int kc = 0; kc < KC; ++kc)
-              tma_load_3d(smem_u32(sV + pst * SB + kc * 8192 + pv_dst * 128), &maps.m[1 + L + pv_l],
-                          smem_u32(&sh->v_full[pst]), kc * 64, pv_prow, hkv);
+              for (int kc = 0; kc < KC; ++kc)
+                tma_load_3d(smem_u32(sV + pst * SB + kc * 8192 + pv_dst * 128), &maps.m[1 + L + pv_l],
+                            smem_u32(&sh->v_full[pst]), kc * 64, pv_prow, hkv);
+            }
           }
           ++viss;
         }
@@ -304,10 +356,15 @@ __global__ void __launch_bounds__(kThreads, CTAS)
         if (lane == 0) mbar_arrive_expect_tx(smem_u32(&sh->v_full[pst]), SB);
         __syncwarp();
         if (pv_mine) {
+          if (PV8) {
+            tma_load_3d(smem_u32(sV + pst * SB + pv_dst * 128), &maps.m[1 + L + pv_l], smem_u32(&sh->v_full[pst]), 0,
+                        pv_prow, hkv);
+          } else {
 #pragma unroll
-          for (int kc = 0; kc < KC; ++kc)
-            tma_load_3d(smem_u32(sV + pst * SB + kc * 8192 + pv_dst * 128), &maps.m[1 + L + pv_l],
-                        smem_u32(&sh->v_full[pst]), kc * 64, pv_prow, hkv);
+            for (int kc = 0; kc < KC; ++kc)
+              tma_load_3d(smem_u32(sV + pst * SB + kc * 8192 + pv_dst * 128), &maps.m[1 + L + pv_l],
+                          smem_u32(&sh->v_full[pst]), kc * 64, pv_prow, hkv);
+          }
         }
         ++viss;
       }
@@ -330,6 +387,7 @@ __global__ void __launch_bounds__(kThreads, CTAS)
       constexpr uint32_t idS = idesc_bf16_f32(128, kSub, false);
       constexpr uint32_t idS8 = idesc_e4m3_f32(128, kSub);
       constexpr uint32_t idO = idesc_bf16_f32(128, D, true);
+      constexpr uint32_t idO8 = idesc_e4m3_f32(128, D, true);
       uint32_t it = 0, qcnt = 0, icnt = 0;
       bool ok = true;
       // shared-memory descriptors of the tile bases; a K step or stage is an
@@ -346,10 +404,18 @@ __global__ void __launch_bounds__(kThreads, CTAS)
         if (!bounded_wait(smem_u32(&sh->p_full[sb2]), (g >> 1) & 1, abort, a.status, 22, icnt, jj, g, 0)) return false;
         if (!bounded_wait(smem_u32(&sh->v_full[st]), (g / NST) & 1, abort, a.status, 26, icnt, jj, g, 0)) return false;
         tc_fence_after();
+        if (PV8) {
+          // K = 32 rows of V (4 KB of the stage) and 8 TMEM columns of P per MMA
 #pragma unroll
-        for (int k = 0; k < kSub / 16; ++k) {
-          umma_ts(tO, tmem + sb2 * kSub + k * 8, dV + ((st * SB + k * 2048) >> 4), idO,
-                  (first_of_item && k == 0) ? 0u : 1u);
+          for (int k = 0; k < kSub / 32; ++k)
+            umma_ts_f8(tO, tmem + sb2 * kSub + k * 8, dV + ((st * SB + k * 4096) >> 4), idO8,
+                       (first_of_item && k == 0) ? 0u : 1u);
+        } else {
+#pragma unroll
+          for (int k = 0; k < kSub / 16; ++k) {
+            umma_ts(tO, tmem + sb2 * kSub + k * 8, dV + ((st * SB + k * 2048) >> 4), idO,
+                    (first_of_item && k == 0) ? 0u : 1u);
+          }
         }
         umma_commit(smem_u32(&sh->v_empty[st]));
         umma_commit(smem_u32(&sh->o_ready));
@@ -428,10 +494,12 @@ __global__ void __launch_bounds__(kThreads, CTAS)
       // softmax scale of this row (log2 units); the FP8 path folds in the
       // row's query scale and its KV head's key scale
       float row_sc = a.scale_log2;
+      float out_sc = 1.0f;          // the KV head's value scale (e4m3 values only)
       if (QK8) {
         const int b = bh / a.Hq, h = bh - b * a.Hq;
         const int hkv = b * a.Hkv + h / (a.Hq / a.Hkv);
         row_sc *= (tok < a.N ? a.qscale[orow] : 0.f) * a.kscale[hkv];
+        if (PV8) out_sc = a.vscale[hkv];
       }
       for (uint32_t j = 0; j < n; ++j, ++it) {
         const uint32_t st = it % NST, sb2 = it & 1;
@@ -508,11 +576,13 @@ __global__ void __launch_bounds__(kThreads, CTAS)
         // PV_j waits for this sub-tile's P, so the awaited phase is one of
         // the two the barrier can be in).
         const bool first = m == -CUDART_INF_F && mnew != -CUDART_INF_F;
-        const bool grow = m != -CUDART_INF_F && mnew > m + kRescaleThreshold;
+        const bool grow = m != -CUDART_INF_F && mnew > m + (PV8 ? kRescaleThresholdP8 : kRescaleThreshold);
+        // e4m3 probabilities: the reference is the next whole binade
+        const float mref = PV8 ? ceilf(mnew) : mnew;
         if (__any_sync(0xffffffffu, grow)) {
-          const float f = grow ? fast_exp2(m - mnew) : 1.0f;
+          const float f = grow ? (PV8 ? exp2_whole(m - mref) : fast_exp2(m - mnew)) : 1.0f;
           lsum *= f;
-          if (grow) m = mnew;
+          if (grow) m = mref;
           if (!warp_wait(smem_u32(&sh->o_ready), (it - 1) & 1, abort, a.status, 33, idx, j, it, 0)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll 1
@@ -524,13 +594,19 @@ __global__ void __launch_bounds__(kThreads, CTAS)
             tmem_st32(tO + c * 32 + lane_off, o);
           }
         }
-        if (first) m = mnew;
+        if (first) m = mref;
         const float mu = m == -CUDART_INF_F ? 0.f : m;
-        uint32_t pk[32];
-        // sub-tiles with masked columns (p must be exactly 0 there) use the
-        // special-function unit only
-        lsum += fast_tile ? sub_probs<kPolyPairs>(s, sc, cb, mu, pk) : sub_probs<0>(s, sc, cb, mu, pk);
-        tmem_st32(tmem + sb2 * kSub + lane_off, pk);
+        if (PV8) {
+          uint32_t pk8[16];
+          lsum += sub_probs8(s, sc, cb, mu, pk8);
+          tmem_st16(tmem + sb2 * kSub + lane_off, pk8);
+        } else {
+          uint32_t pk[32];
+          // sub-tiles with masked columns (p must be exactly 0 there) use the
+          // special-function unit only
+          lsum += fast_tile ? sub_probs<kPolyPairs>(s, sc, cb, mu, pk) : sub_probs<0>(s, sc, cb, mu, pk);
+          tmem_st32(tmem + sb2 * kSub + lane_off, pk);
+        }
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(smem_u32(&sh->p_full[sb2]));
@@ -542,7 +618,7 @@ __global__ void __launch_bounds__(kThreads, CTAS)
       if (!warp_wait(smem_u32(&sh->o_final), icnt & 1, abort, a.status, 35, idx, n, it, icnt)) { ok = false; break; }
       ++icnt;
       tc_fence_after();
-      const float inv = lsum > 0.f ? 1.0f / lsum : 0.f;
+      const float inv = lsum > 0.f ? out_sc / lsum : 0.f;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -592,24 +668,25 @@ __global__ void __launch_bounds__(kThreads, CTAS)
 #define PSA_ATTN_CTAS 2
 #endif
 
-template <int D, bool F32, bool QK8 = false>
+template <int D, bool F32, bool QK8 = false, bool PV8 = false>
 cudaError_t launch_one(const AttnMaps& maps, const AttnArgs& a, int num_sms, cudaStream_t s) {
   constexpr int CTAS = PSA_ATTN_CTAS;
   constexpr int NST = CTAS == 1 ? (D == 128 ? 5 : 8) : 2;
   constexpr size_t QB = QK8 ? static_cast<size_t>(D) * 128 : static_cast<size_t>(D) * 256;
   constexpr size_t SBK = QK8 ? static_cast<size_t>(D) * 64 : static_cast<size_t>(D) * 128;
-  const size_t smem = 1024 + QB + NST * (SBK + static_cast<size_t>(D) * 128) + sizeof(AttnShared<NST>);
+  constexpr size_t SBV = PV8 ? static_cast<size_t>(D) * 64 : static_cast<size_t>(D) * 128;
+  const size_t smem = 1024 + QB + NST * (SBK + SBV) + sizeof(AttnShared<NST>);
   const int grid = a.n_items < CTAS * num_sms ? a.n_items : CTAS * num_sms;
   if (a.block == 64) {
-    cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(attn_kernel<D, F32, NST, CTAS, true, QK8>),
+    cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(attn_kernel<D, F32, NST, CTAS, true, QK8, PV8>),
                                    static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    attn_kernel<D, F32, NST, CTAS, true, QK8><<<grid, kThreads, smem, s>>>(maps, a);
+    attn_kernel<D, F32, NST, CTAS, true, QK8, PV8><<<grid, kThreads, smem, s>>>(maps, a);
   } else {
-    cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(attn_kernel<D, F32, NST, CTAS, false, QK8>),
+    cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(attn_kernel<D, F32, NST, CTAS, false, QK8, PV8>),
                                    static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    attn_kernel<D, F32, NST, CTAS, false, QK8><<<grid, kThreads, smem, s>>>(maps, a);
+    attn_kernel<D, F32, NST, CTAS, false, QK8, PV8><<<grid, kThreads, smem, s>>>(maps, a);
   }
   return cudaGetLastError();
 }
@@ -624,12 +701,12 @@ cudaError_t launch_attention(const CUtensorMap* maps, const AttnArgs& a, int num
   return a.out_fp32 ? launch_one<64, true>(m, a, num_sms, s) : launch_one<64, false>(m, a, num_sms, s);
 }
 
-cudaError_t launch_attention_fp8(const CUtensorMap* maps, const AttnArgs& a, int num_sms, cudaStream_t s) {
+cudaError_t launch_attention_fp8(const CUtensorMap* maps, const AttnArgs& a, bool pv, int num_sms, cudaStream_t s) {
   if (a.d != 128 || a.out_fp32) return cudaErrorInvalidValue;
   AttnMaps m;
   for (int i = 0; i < 1 + 2 * a.levels; ++i) m.m[i] = maps[i];
   for (int i = 1 + 2 * a.levels; i < 9; ++i) m.m[i] = maps[0];
-  return launch_one<128, false, true>(m, a, num_sms, s);
+  return pv ? launch_one<128, false, true, true>(m, a, num_sms, s) : launch_one<128, false, true, false>(m, a, num_sms, s);
 }
 
 }  // namespace psa

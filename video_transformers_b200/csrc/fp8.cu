@@ -7,6 +7,9 @@
 // values are fp32; each is rounded to the nearest e4m3 value, ties to even,
 // saturating at +-448 (cvt.rn.satfinite).
 //
+// The values of the FP8 probability path are coded like the keys, with
+// their own per-head scale.
+//
 // kabsmax_kernel   one CTA per KV head: max |K| over level 0.
 // quant_rows_kernel  one warp per query row: its max, scale and codes.
 // quant_head_kernel  every key of every level, with its head's multiplier.
@@ -125,6 +128,25 @@ int grid_cap(int64_t work, int threads) {
 
 }  // namespace
 
+cudaError_t launch_quantize_heads_fp8(const void* x, const void* x_pyr, const size_t* level_off, int64_t BH, int N,
+                                     int d, int levels, uint8_t* x8, uint8_t* x8_pyr, float* scale, cudaStream_t s) {
+  // scale holds the per-head maxima until every level is coded
+  kabsmax_kernel<<<static_cast<unsigned>(BH), 1024, 0, s>>>(static_cast<const __nv_bfloat16*>(x), scale,
+                                                            static_cast<int64_t>(N) * d);
+  const int64_t t0 = BH * N * d;
+  quant_head_kernel<<<grid_cap(t0 / 8, 256), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), x8, scale,
+                                                          static_cast<int64_t>(N) * d, t0);
+  for (int l = 1; l < levels; ++l) {
+    const int64_t per = static_cast<int64_t>(N >> l) * d;
+    const int64_t tl = BH * per;
+    quant_head_kernel<<<grid_cap(tl / 8, 256), 256, 0, s>>>(
+        reinterpret_cast<const __nv_bfloat16*>(static_cast<const char*>(x_pyr) + level_off[l] * 2), x8_pyr + level_off[l],
+        scale, per, tl);
+  }
+  head_scale_kernel<<<static_cast<unsigned>((BH + 255) / 256), 256, 0, s>>>(scale, static_cast<int>(BH));
+  return cudaGetLastError();
+}
+
 cudaError_t launch_quantize_qk_fp8(const void* q, const void* k, const void* k_pyr, const size_t* level_off,
                                    int64_t BHq, int64_t BHkv, int N, int d, int levels, uint8_t* q8, float* q_scale,
                                    uint8_t* k8, uint8_t* k8_pyr, float* k_scale, cudaStream_t s) {
@@ -135,21 +157,7 @@ cudaError_t launch_quantize_qk_fp8(const void* q, const void* k, const void* k_p
     quant_rows_kernel<128><<<qgrid, 32 * warps_per_cta, 0, s>>>(static_cast<const __nv_bfloat16*>(q), q8, q_scale, qrows);
   else
     quant_rows_kernel<64><<<qgrid, 32 * warps_per_cta, 0, s>>>(static_cast<const __nv_bfloat16*>(q), q8, q_scale, qrows);
-  // k_scale holds the per-head maxima until every level is coded
-  kabsmax_kernel<<<static_cast<unsigned>(BHkv), 1024, 0, s>>>(static_cast<const __nv_bfloat16*>(k), k_scale,
-                                                              static_cast<int64_t>(N) * d);
-  const int64_t t0 = BHkv * N * d;
-  quant_head_kernel<<<grid_cap(t0 / 8, 256), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(k), k8, k_scale,
-                                                          static_cast<int64_t>(N) * d, t0);
-  for (int l = 1; l < levels; ++l) {
-    const int64_t per = static_cast<int64_t>(N >> l) * d;
-    const int64_t tl = BHkv * per;
-    quant_head_kernel<<<grid_cap(tl / 8, 256), 256, 0, s>>>(
-        reinterpret_cast<const __nv_bfloat16*>(static_cast<const char*>(k_pyr) + level_off[l] * 2), k8_pyr + level_off[l],
-        k_scale, per, tl);
-  }
-  head_scale_kernel<<<static_cast<unsigned>((BHkv + 255) / 256), 256, 0, s>>>(k_scale, static_cast<int>(BHkv));
-  return cudaGetLastError();
+  return launch_quantize_heads_fp8(k, k_pyr, level_off, BHkv, N, d, levels, k8, k8_pyr, k_scale, s);
 }
 
 }  // namespace psa

@@ -123,14 +123,16 @@ struct AttnArgs {
   int* status;
   const float* qscale;    // FP8 path only: per query row [B*Hq*N]
   const float* kscale;    // FP8 path only: per KV head [B*Hkv]
+  const float* vscale;    // FP8 path with e4m3 P and V only: per KV head [B*Hkv]
 };
 // maps: [0] = Q (3D view [d, N, B*Hq], box 64 x 128), [1 + l] = K level l,
 // [1 + L + l] = V level l (3D views [d, N/2^l, B*Hkv], box 64 x min(block/2^l, 64)).
 cudaError_t launch_attention(const CUtensorMap* maps, const AttnArgs& a, int num_sms,
                              cudaStream_t s);
-// The FP8 path (d = 128, bf16 V and output): Q and K maps over e4m3 codes,
-// box 128 bytes wide (Q 128 rows, K levels min(block/2^l, 64) rows).
-cudaError_t launch_attention_fp8(const CUtensorMap* maps, const AttnArgs& a, int num_sms, cudaStream_t s);
+// The FP8 path (d = 128, bf16 output): Q and K maps over e4m3 codes, box
+// 128 bytes wide (Q 128 rows, K levels min(block/2^l, 64) rows).  With pv,
+// the V maps are over e4m3 codes too (same boxes as K) and P is e4m3.
+cudaError_t launch_attention_fp8(const CUtensorMap* maps, const AttnArgs& a, bool pv, int num_sms, cudaStream_t s);
 
 // ---- stage 3, backward ----------------------------------------------------
 // D_i = dO_i . O_i and lse_i * log2(e) per query row, written into arrays
@@ -208,6 +210,11 @@ cudaError_t launch_pool_bwd(const float* gl, const int64_t* level_off, void* out
 // k (level 0) and the levels of k_pyr (element offsets level_off[l] of level l
 // inside the pyramid buffer) -> k8 and k8_pyr codes at the same element
 // offsets, and k_scale [BHkv] (fp32, head max of level 0 / 448).
+// e4m3 codes of a per-head tensor and its pyramid levels ([BH][N >> l][d]
+// bf16 each; level l > 0 at element offset level_off[l] of x_pyr / x8_pyr),
+// one scale per head from level 0's largest magnitude: scale = max / 448.
+cudaError_t launch_quantize_heads_fp8(const void* x, const void* x_pyr, const size_t* level_off, int64_t BH, int N,
+                                     int d, int levels, uint8_t* x8, uint8_t* x8_pyr, float* scale, cudaStream_t s);
 cudaError_t launch_quantize_qk_fp8(const void* q, const void* k, const void* k_pyr, const size_t* level_off,
                                    int64_t BHq, int64_t BHkv, int N, int d, int levels, uint8_t* q8, float* q_scale,
                                    uint8_t* k8, uint8_t* k8_pyr, float* k_scale, cudaStream_t s);
