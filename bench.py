@@ -547,18 +547,19 @@ def measure_fp8(path, w, stream, flops_fwd, peaks_, reps=5):
         call()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(reps):
-            call()
-        e1.record(stream)
-        torch.cuda.synchronize()
+        with ClockSampler(path.q.device.index or 0) as cs:
+            e0.record(stream)
+            for _ in range(reps):
+                call()
+            e1.record(stream)
+            torch.cuda.synchronize()
         st = P.psa_get_device_status(ws)
         if st != P.PSA_OK:
             raise RuntimeError("device status %d after the FP8 path: %s" % (st, P.psa_last_error()))
         ms = e0.elapsed_time(e1) / reps
         diff = (out8.float() - ref).abs()
         tf = flops_fwd / (ms * 1e-3) / 1e12
-        return {"ms": ms, "tflops": tf, "frac_of_burst_bf16": tf / peaks_[0],
+        return {"ms": ms, "tflops": tf, "frac_of_burst_bf16": tf / peaks_[0], "clocks": cs.summary(),
                 "vs_bf16_path": {"max_abs": diff.max().item(), "mean_abs": diff.mean().item()}}
 
     r = {"entry_point": "psa_attention_fwd_fp8", "reps": reps,
