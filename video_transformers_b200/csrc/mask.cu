@@ -713,18 +713,19 @@ __device__ __forceinline__ double exp2_split_exp(double x) {
 
 // per-warp shared memory of select_bucket_kernel for P = nkb rounded up to 32
 struct BucketLayout {
-  int hs, tfx, rlse, mass, hc, lend, bk, list, ex, mixed, lv, bytes;
+  int hs, tfx, rlse, mass, hc, lend, rth, list, ex, mixed, lv, bytes;
 };
-__host__ __device__ inline BucketLayout bucket_layout(int P) {
+// P = nkb rounded up to 32, R = score rows per query block (<= 128)
+__host__ __device__ inline BucketLayout bucket_layout(int P, int R) {
   BucketLayout L{};
   int o = 0;
   L.hs = o;    o += 8 * kBucketSlots;   // u64 fixed-point sums, then their exclusive prefix
   L.tfx = o;   o += 8 * 8;              // u64 thresholds in fixed point
-  L.rlse = o;  o += 8 * 128;            // f64 row LSEs of the row block's score rows
+  L.rlse = o;  o += 8 * ((R + 1) & ~1); // f64 row LSEs of the row block's score rows
   L.mass = o;  o += 4 * P;              // f32 block masses
   L.hc = o;    o += 4 * kBucketSlots;   // counts, then the exclusive rank
   L.lend = o;  o += 4 * kBucketSlots;   // start of a bucket's list group, then its end
-  L.bk = o;    o += 2 * P;              // u16 bucket of every block
+  L.rth = o;   o += 4 * 8;              // quantile policy: first rank of each level
   L.list = o;  o += 2 * P;              // u16 blocks of mixed buckets, grouped by bucket
   L.ex = o;    o += P;                  // exact level of every listed block
   L.mixed = o; o += kBucketSlots;       // a threshold falls inside the bucket
@@ -738,7 +739,7 @@ __global__ void __launch_bounds__(32 * kBucketWarps) select_bucket_kernel(const 
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int row = blockIdx.x * kBucketWarps + wid;              // (b*Hq + h)*nqb + I
   if (row >= a.B * a.Hq * a.nqb) return;
-  const BucketLayout L = bucket_layout((a.nkb + 31) & ~31);
+  const BucketLayout L = bucket_layout((a.nkb + 31) & ~31, a.rows_per_block);
   uint8_t* base = sel_smem + wid * L.bytes;
   unsigned long long* hs = reinterpret_cast<unsigned long long*>(base + L.hs);
   unsigned long long* tfx = reinterpret_cast<unsigned long long*>(base + L.tfx);
@@ -746,7 +747,7 @@ __global__ void __launch_bounds__(32 * kBucketWarps) select_bucket_kernel(const 
   float* mass = reinterpret_cast<float*>(base + L.mass);
   int* hc = reinterpret_cast<int*>(base + L.hc);
   int* lend = reinterpret_cast<int*>(base + L.lend);
-  uint16_t* bk = reinterpret_cast<uint16_t*>(base + L.bk);
+  int* rth = reinterpret_cast<int*>(base + L.rth);
   uint16_t* list = reinterpret_cast<uint16_t*>(base + L.list);
   uint8_t* ex = base + L.ex;
   uint8_t* mixed = base + L.mixed;
@@ -829,6 +830,14 @@ __global__ void __launch_bounds__(32 * kBucketWarps) select_bucket_kernel(const 
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mmax = fmaxf(mmax, __shfl_xor_sync(0xffffffffu, mmax, o));
   __syncwarp();
+  // bucket of a block: any function monotone in the mass keeps the rank
+  // order; the product by one reciprocal and the floor are (fp32 rounding is
+  // monotone), and recomputing it gives the same bucket every time
+  const float inv_max = mmax > 0.f ? 1.0f / mmax : 0.f;
+  auto bucket_of = [&](float m) {
+    return m == 0.f ? kBuckets
+                    : max(0, min(kBuckets - 1, static_cast<int>(floorf(static_cast<float>(kBuckets) * (1.0f - m * inv_max)))));
+  };
 
   // buckets (monotone in the mass: the fp32 quotient and product round
   // monotonically) and the histogram.  Exact zeros (every block past the
@@ -840,14 +849,10 @@ __global__ void __launch_bounds__(32 * kBucketWarps) select_bucket_kernel(const 
     const float m = valid ? mass[J] : 1.f;
     const unsigned zeros = __ballot_sync(0xffffffffu, m == 0.f);
     if (lane == 0 && zeros) atomicAdd(&hc[kBuckets], __popc(zeros));
-    if (valid) {
-      int bb = kBuckets;
-      if (m != 0.f) {
-        bb = max(0, min(kBuckets - 1, static_cast<int>(floorf(static_cast<float>(kBuckets) * (1.0f - m / mmax)))));
-        atomicAdd(&hc[bb], 1);
-        atomicAdd(&hs[bb], mass_fix(m));
-      }
-      bk[J] = static_cast<uint16_t>(bb);
+    if (valid && m != 0.f) {
+      const int bb = bucket_of(m);
+      atomicAdd(&hc[bb], 1);
+      atomicAdd(&hs[bb], mass_fix(m));
     }
   }
   __syncwarp();
@@ -889,10 +894,29 @@ __global__ void __launch_bounds__(32 * kBucketWarps) select_bucket_kernel(const 
   __syncwarp();
 
   const int n_vis = a.causal ? min(I + 1, a.nkb) : a.nkb;
+  // quantile policy: level l applies from rank r on when t_l <= r / n_vis
+  // (an fp64 quotient, as the definition is written); the quotient never
+  // decreases with r, so that set of ranks is [rth[l], inf) and every test
+  // is one integer comparison.  ceil(t n) is within one of the boundary.
+  if (a.policy == 1 && lane < a.levels) {
+    const double t = static_cast<double>(a.thresholds[lane]);
+    const double n = static_cast<double>(n_vis);
+    int r;
+    if (t <= 0.0) {
+      r = 0;
+    } else if (!(t < 2.0)) {
+      r = 0x7FFFFFFF;                              // beyond every rank (r < n_vis <= 1024); NaN too
+    } else {
+      r = static_cast<int>(ceil(t * n));
+      for (int it = 0; it < 4 && r > 0 && t <= static_cast<double>(r - 1) / n; ++it) --r;
+      for (int it = 0; it < 4 && !(t <= static_cast<double>(r) / n); ++it) ++r;
+    }
+    rth[lane] = r;
+  }
+  __syncwarp();
   auto lev_rank = [&](int r) {
     int lev = 0;
-    for (int l = 0; l < a.levels; ++l)
-      lev += (static_cast<double>(a.thresholds[l]) <= static_cast<double>(r) / static_cast<double>(n_vis));
+    for (int l = 0; l < a.levels; ++l) lev += r >= rth[l];
     return lev;
   };
   auto lev_fix = [&](unsigned long long C) {
@@ -946,7 +970,7 @@ __global__ void __launch_bounds__(32 * kBucketWarps) select_bucket_kernel(const 
   // list the blocks of mixed buckets (within a group in any order)
   if (nmix > 0) {
     for (int J = lane; J < a.nkb; J += 32) {
-      const int bb = bk[J];
+      const int bb = bucket_of(mass[J]);
       if (mixed[bb]) list[atomicAdd(&lend[bb], 1)] = static_cast<uint16_t>(J);
     }
     __syncwarp();
@@ -955,7 +979,7 @@ __global__ void __launch_bounds__(32 * kBucketWarps) select_bucket_kernel(const 
     for (int i = lane; i < nmix; i += 32) {
       const int Jj = list[i];
       const unsigned long long kj = rank_key(mass[Jj], Jj);
-      const int bj = bk[Jj];
+      const int bj = bucket_of(mass[Jj]);
       const int end = lend[bj], beg = end - (hc[bj + 1] - hc[bj]);
       unsigned long long psum = 0ull;
       int pcnt = 0;
@@ -974,7 +998,7 @@ __global__ void __launch_bounds__(32 * kBucketWarps) select_bucket_kernel(const 
 
   // levels, forced rules, the mask
   for (int J = lane; J < a.nkb; J += 32) {
-    const int bb = bk[J];
+    const int bb = bucket_of(mass[J]);
     const int lev = mixed[bb] ? ex[J] : lv[bb];
     int out = lev >= a.levels ? PSA_SKIP : lev;
     if (a.n_dense_prefix > 0 &&
@@ -1045,7 +1069,7 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t s) {
   // antidiagonal groups), which both kernels' row-LSE arrays rely on
   if (a.rows_per_block > 128) return cudaErrorInvalidValue;
   if (a.nkb <= 1024) {
-    const size_t smem = static_cast<size_t>(kBucketWarps) * bucket_layout((a.nkb + 31) & ~31).bytes;
+    const size_t smem = static_cast<size_t>(kBucketWarps) * bucket_layout((a.nkb + 31) & ~31, a.rows_per_block).bytes;
     cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(&select_bucket_kernel), static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     select_bucket_kernel<<<(rows + kBucketWarps - 1) / kBucketWarps, 32 * kBucketWarps, smem, s>>>(a);
