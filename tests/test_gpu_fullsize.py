@@ -199,35 +199,39 @@ def test_fullsize_fp8_wan14b_sampled():
         assert mx <= 2e-2 and mean <= 2e-3, (h, Is, mx, mean)
 
 
-def test_fullsize_fp8_pv_wan14b_sampled():
+@pytest.mark.parametrize("name", ["wan14b", "qwen2.5vl"])
+def test_fullsize_fp8_pv_sampled(name):
     """The FP8 path with e4m3 probabilities and values (reading R14) at the
-    Wan2.1-14B shape on the generated mask, on sampled query-block rows,
-    against the oracle's attention_fp8(pv=True) on the whole head's levels
-    (the value scale is per head), with the reference-shift tolerance of
-    test_gpu_fp8.py (max-abs 5e-2, mean-abs 5e-3)."""
-    w = W.PRESETS["wan14b"]
+    preset's full shape on its generated mask (Qwen2.5-VL: causal, 7 query
+    heads per KV head, antidiagonal scorer with the cosine gate), on sampled
+    query-block rows, against the oracle's attention_fp8(pv=True) on the
+    whole KV head's levels (the value scale is per KV head), with the
+    reference-shift tolerance of test_gpu_fp8.py (max-abs 5e-2, mean-abs
+    5e-3)."""
+    w = W.PRESETS[name]
     q, k, v, _ = W.make_qkv(w, device=DEV)
     shape = shape_for(w)
-    kp, vp, _ = run_pyramid(shape, k, v)
-    mask, _ = run_mask(shape, params_for(w), q, k)
+    kp, vp, bc = run_pyramid(shape, k, v, with_cos=w.cos_min > -2)
+    mask, _ = run_mask(shape, params_for(w), q, k, bc)
     out = torch.empty_like(q)
     ws = P.workspace(P.psa_attention_fp8_workspace_bytes(shape), DEV)
     P.psa_attention_fwd_fp8_pv(shape, q, k, v, kp, vp, mask, w.sm_scale, out, None, ws)
     torch.cuda.synchronize()
     assert P.psa_get_device_status(ws) == P.PSA_OK
     rows = sample_rows(w, 10, seed=6)
+    grp = w.Hq // w.Hkv
     worst = (0.0, 0.0)
     for (b, h), Is in by_head(rows).items():
         hrows = [(0, 0, I) for I in Is]
-        kl = head_levels(shape, k, kp, b, h, w.levels)
-        vl = head_levels(shape, v, vp, b, h, w.levels)
+        kl = head_levels(shape, k, kp, b, h // grp, w.levels)
+        vl = head_levels(shape, v, vp, b, h // grp, w.levels)
         o, _ = O.attention_fp8(q[b:b + 1, h:h + 1].cpu(), [x.astype(np.float32) for x in kl],
                                [x.astype(np.float32) for x in vl], mask[b:b + 1, h:h + 1].cpu(), w.block, w.sm_scale,
-                               False, rows=hrows, pv=True)
+                               w.causal, rows=hrows, pv=True)
         mx, mean, _ = attn_errors(out[b:b + 1, h:h + 1], o)
         assert mx <= 5e-2 and mean <= 5e-3, (h, Is, mx, mean)
         worst = (max(worst[0], mx), max(worst[1], mean))
-    note("fp8 P.V wan14b full size, sampled rows: vs the e4m3 oracle max %.2e mean %.2e" % worst)
+    note("fp8 P.V %s full size, sampled rows: vs the e4m3 oracle max %.2e mean %.2e" % ((name,) + worst))
 
 
 def test_fullsize_backward_dq_wan14b_sampled():
