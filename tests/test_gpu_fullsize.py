@@ -199,11 +199,12 @@ def test_fullsize_fp8_wan14b_sampled():
         assert mx <= 2e-2 and mean <= 2e-3, (h, Is, mx, mean)
 
 
-@pytest.mark.parametrize("name", ["wan14b", "qwen2.5vl"])
+@pytest.mark.parametrize("name", ["wan14b", "qwen2.5vl", "wan1.3b"])
 def test_fullsize_fp8_pv_sampled(name):
     """The FP8 path with e4m3 probabilities and values (reading R14) at the
     preset's full shape on its generated mask (Qwen2.5-VL: causal, 7 query
-    heads per KV head, antidiagonal scorer with the cosine gate), on sampled
+    heads per KV head, antidiagonal scorer with the cosine gate; Wan2.1-1.3B:
+    64-token blocks, two query blocks per tile), on sampled
     query-block rows, against the oracle's attention_fp8(pv=True) on the
     whole KV head's levels (the value scale is per KV head), with the
     reference-shift tolerance of test_gpu_fp8.py (max-abs 5e-2, mean-abs
