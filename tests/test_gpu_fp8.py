@@ -21,7 +21,8 @@
   - elsewhere probabilities below 2^-6 at one reference and not at the
     other round differently.  Emulating the reference 1..5 binades lower
     on rows of 1000 Gaussian logits (standard deviation 1-4) moved outputs
-    by at most 3.2e-2 (mean 2.8e-3): max-abs 5e-2, mean-abs 5e-3."""
+    by at most 3.2e-2 (mean 2.8e-3): max-abs 5e-2, mean-abs 5e-3.  Both
+    facts are checked on the CPU by test_fp8_tolerance.py."""
 import numpy as np
 import pytest
 import torch
