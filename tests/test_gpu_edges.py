@@ -3,6 +3,8 @@
   * More than 1024 KV blocks: the mask generator's CTA-wide select kernel
     (the warp kernel holds at most 1024 keys per row), with both level
     policies and causal masking, and attention on the resulting mask.
+  * Determinism of the mask (select kernel atomics) and of the FP8
+    probability-and-value attention: repeated calls are bit-equal.
   * A bounded device wait that runs out: with the debug trap armed, every
     CTA of the attention kernel waits once on a barrier nothing arrives at
     (limit 1 ms), gives up, unwinds, and PSA_ERR_TIMEOUT with that wait's
@@ -119,3 +121,43 @@ def test_attention_wait_timeout_is_reported_and_recoverable():
     o, _ = O.attention(q, kl, vl, mask.cpu(), shape.block, shape.d ** -0.5, False, rows=rows)
     mx, mean, _ = attn_errors(out2, o)
     assert mx <= 2e-2 and mean <= 2e-3, (mx, mean)
+
+
+@pytest.mark.parametrize("name,heads,policy", [("wan14b", (1, 1), P.PSA_POLICY_MASS),
+                                               ("wan1.3b", (2, 2), P.PSA_POLICY_QUANTILE),
+                                               ("qwen2.5vl", (7, 1), P.PSA_POLICY_MASS)])
+def test_mask_is_deterministic(name, heads, policy):
+    """Three calls of psa_make_mask give the same mask and masses bit for
+    bit, at the presets' full sequence lengths (591, 512 and 256 key
+    blocks): the select kernel's shared-memory atomics add integers (counts
+    and fixed-point sums, the same in any order) or place a block in its
+    bucket's list, whose order the exact count does not depend on."""
+    from psa_run import params_for
+    w = W.PRESETS[name].replace(Hq=heads[0], Hkv=heads[1])
+    q, k, v, _ = W.make_qkv(w, device=DEV)
+    shape = shape_for(w)
+    _, _, bc = run_pyramid(shape, k, v, with_cos=w.cos_min > -2)
+    runs = [run_mask(shape, params_for(w, policy), q, k, bc) for _ in range(3)]
+    for m, s in runs[1:]:
+        assert torch.equal(m, runs[0][0]) and torch.equal(s, runs[0][1])
+
+
+def test_fp8_pv_attention_is_deterministic():
+    """Two calls of the FP8 probability-and-value path give the same output
+    and lse bit for bit (no atomics; a fixed order of work per query tile)."""
+    w = W.reduced("wan14b", grid=(4, 12, 16), heads=(2, 2))
+    q, k, v, _ = W.make_qkv(w, device=DEV)
+    shape = shape_for(w)
+    kp, vp, _ = run_pyramid(shape, k, v)
+    from psa_run import params_for
+    mask, _ = run_mask(shape, params_for(w), q, k)
+    outs = []
+    for _ in range(2):
+        out = torch.empty_like(q)
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=DEV)
+        ws = P.workspace(P.psa_attention_fp8_workspace_bytes(shape), DEV)
+        P.psa_attention_fwd_fp8_pv(shape, q, k, v, kp, vp, mask, w.sm_scale, out, lse, ws)
+        torch.cuda.synchronize()
+        assert P.psa_get_device_status(ws) == P.PSA_OK
+        outs.append((out, lse))
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
