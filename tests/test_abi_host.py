@@ -200,3 +200,12 @@ def test_fp8_path_rejects_unsupported_shapes():
     sf = P.make_shape(1, 2, 2, 256, 128, 64, 4, dtype=P.PSA_DT_FP32)
     assert P.psa_attention_fp8_workspace_bytes(sf) == 0
     assert P.psa_attention_fp8_workspace_bytes(P.make_shape(1, 2, 2, 256, 128, 64, 4)) > 0
+
+
+def test_psa_forward_rejects_bad_arguments():
+    """The whole-path convenience call checks its options before any launch."""
+    x = torch.zeros(1, 1, 128, 64)
+    with pytest.raises(ValueError):
+        P.psa_forward(x, x, x, precision="int4")
+    with pytest.raises(ValueError):
+        P.psa_forward(x, x, x, levels=4, thresholds=(0.5, 0.9))

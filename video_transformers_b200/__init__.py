@@ -288,3 +288,66 @@ def workspace(nbytes: int, device) -> torch.Tensor:
     """A zero-filled workspace (the status word must start at 0)."""
     n16 = max(1, (nbytes + 15) // 16)
     return torch.zeros(2 * n16, dtype=torch.int64, device=device).view(torch.uint8)[:max(nbytes, 16)]
+
+
+# ------------------------------------------------------------------------- whole path
+
+_CACHE = {}
+
+
+def psa_forward(q, k, v, *, block: int = 128, levels: int = 4, thresholds: Sequence[float] = (0.6, 0.8, 0.9, 0.95),
+                mode: int = PSA_MASK_SAMPLE, policy: int = PSA_POLICY_MASS, causal: bool = False,
+                sm_scale: Optional[float] = None, stride: int = 8, cos_min: float = -3.0, n_dense_prefix: int = 0,
+                mask=None, precision: str = "bf16", want_lse: bool = False, stream=None):
+    """The whole forward path on device tensors: psa_build_pyramid (and the
+    block cosines when cos_min > -2), psa_make_mask (unless a mask is given)
+    and the attention (precision "bf16": psa_attention_fwd; "fp8":
+    psa_attention_fwd_fp8; "fp8_pv": psa_attention_fwd_fp8_pv), on one
+    stream.  q [B, Hq, N, d], k and v [B, Hkv, N, d], contiguous, bf16 (fp32
+    for "bf16" only).  Pyramid buffers and workspaces are allocated on first
+    use for a shape and reused.  Returns (out, mask, lse or None); a kernel
+    time-out is reported by psa_forward_status()."""
+    if precision not in ("bf16", "fp8", "fp8_pv"):
+        raise ValueError("precision must be 'bf16', 'fp8' or 'fp8_pv', not %r" % (precision,))
+    if len(thresholds) != levels:
+        raise ValueError("%d thresholds for %d levels" % (len(thresholds), levels))
+    shape = shape_of(q, k, block, levels, causal)
+    scale = float(q.shape[-1]) ** -0.5 if sm_scale is None else float(sm_scale)
+    params = make_params(mode, thresholds, scale, stride=stride, cos_min=cos_min, n_dense_prefix=n_dense_prefix,
+                         policy=policy)
+    key = (q.device, tuple(q.shape), tuple(k.shape), q.dtype, block, levels, causal, mode, stride, precision)
+    c = _CACHE.get(key)
+    if c is None:
+        kp, vp = pyramid_buffers(shape, q.device, q.dtype)
+        nb = -(-shape.N // block)
+        attn_bytes = psa_attention_workspace_bytes(shape) if precision == "bf16" else \
+            psa_attention_fp8_workspace_bytes(shape)
+        c = {"kp": kp, "vp": vp,
+             "bc": torch.empty(shape.B, shape.Hkv, nb, dtype=torch.float32, device=q.device),
+             "mws": workspace(psa_mask_workspace_bytes(shape, params), q.device),
+             "aws": workspace(attn_bytes, q.device)}
+        _CACHE.clear()                        # one shape at a time: the buffers can be large
+        _CACHE[key] = c
+    bc = c["bc"] if cos_min > -2 else None
+    L1 = levels > 1
+    psa_build_pyramid(shape, k, v, c["kp"] if L1 else None, c["vp"] if L1 else None, bc, stream)
+    if mask is None:
+        nb = -(-shape.N // block)
+        mask = torch.empty(shape.B, shape.Hq, nb, nb, dtype=torch.uint8, device=q.device)
+        psa_make_mask(shape, params, q, k, bc, mask, None, c["mws"], stream)
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device) if want_lse else None
+    fn = {"bf16": psa_attention_fwd, "fp8": psa_attention_fwd_fp8, "fp8_pv": psa_attention_fwd_fp8_pv}[precision]
+    fn(shape, q, k, v, c["kp"] if L1 else None, c["vp"] if L1 else None, mask, scale, out, lse, c["aws"], stream)
+    return out, mask, lse
+
+
+def psa_forward_status(stream=None) -> int:
+    """Device status of the last psa_forward call (PSA_OK, or the first
+    error of the mask or attention stage), read after the stream's work."""
+    for c in _CACHE.values():
+        for ws in (c["mws"], c["aws"]):
+            st = psa_get_device_status(ws, stream)
+            if st != PSA_OK:
+                return st
+    return PSA_OK
