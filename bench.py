@@ -216,6 +216,20 @@ def executed_flops(mask: torch.Tensor, N: int, block: int, d: int, levels: int, 
     return 4.0 * d * float(total.item())
 
 
+def diagonal_excess_flops(mask: torch.Tensor, N: int, block: int, d: int) -> float:
+    """FLOPs that executed_flops counts for the key-after-query pairs of the
+    causal diagonal blocks (always level 0): q_I^2 - q_I (q_I + 1) / 2 per
+    (b, h, I) whose diagonal is not skipped.  Subtracting them gives the
+    FlashAttention convention, where a causal block counts only its visible
+    pairs."""
+    dev = mask.device
+    nb = mask.shape[-1]
+    idx = torch.arange(nb, device=dev)
+    qrows = (torch.clamp((idx + 1) * block, max=N) - idx * block).double()
+    diag = (mask.diagonal(dim1=-2, dim2=-1) == 0).double()
+    return 4.0 * d * float((diag * (qrows * qrows - qrows * (qrows + 1) / 2)).sum().item())
+
+
 class Path:
     """Device buffers and the three ABI calls of one workload instance."""
 
@@ -358,6 +372,10 @@ def config_record(w, path, m, clocks, peaks_):
            "dense_equiv_speedup": (m["dense_ms"] / m["attn_ms"]) if m["dense_ms"] else None,
            "pyramid_gbs": pyr_gbs, "pyramid_frac_of_hbm": pyr_gbs / hbm,
            "plan_padding_frac": 1 - m["n_rows"] / max(1, 128 * m["n_tiles"])}
+    if w.causal:
+        fa = m["flops"] - diagonal_excess_flops(path.mask, w.N, w.block, w.d)
+        rec["attn_tflops_fa_causal"] = fa / (m["attn_ms"] * 1e-3) / 1e12
+        rec["fa_causal_convention"] = "only the key <= query pairs of the diagonal blocks count"
     mr = mask_roofline(w, m["mask_ms"], hbm, clocks, elem)
     if mr is not None:
         rec["mask_frac"] = mr["frac"]

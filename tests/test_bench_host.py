@@ -1,35 +1,48 @@
-"""Host-side arithmetic of bench.py's report (no GPU): the mask-stage
-roofline object and the per-scorer launch counts."""
-import math
+"""Host-side arithmetic of bench.py against brute force (CPU): the executed
+FLOPs of a mask (4 d x query rows x pooled key rows over the non-skipped
+pairs, causal blocks above the diagonal left out) and the FlashAttention
+convention for causal masks (only the key <= query pairs of the diagonal
+blocks)."""
+import numpy as np
+import pytest
+import torch
 
-import bench
-import workloads as W
+import bench as B
 
-
-def test_mask_roofline_sampling_counts_one_exp2_per_score_element():
-    w = W.PRESETS["wan14b"]
-    r = bench.mask_roofline(w, mask_ms=10.0, hbm=6541.5, clocks={"sm_mhz": 1800.0}, elem=2)
-    exps = (-(-75600 // 128) * 8) * 75600 * 40
-    assert r["bound"] == "alu" and r["unit"] == "Gexp2/s"
-    assert math.isclose(r["achieved"], exps / 10e-3 / 1e9)
-    assert math.isclose(r["peak"], 16 * 148 * 1800e6 / 1e9)
-    assert math.isclose(r["frac"], r["achieved"] / r["peak"])
+SKIP = 255
 
 
-def test_mask_roofline_antidiag_causal_halves():
-    w = W.PRESETS["qwen2.5vl"]
-    r = bench.mask_roofline(w, mask_ms=1.0, hbm=6541.5, clocks=None, elem=2)
-    n = 32768 // 8
-    assert math.isclose(r["achieved"], n * n * 28 * 0.5 / 1e-3 / 1e9)
+def brute(mask, N, block, d, causal, pairs_only):
+    total = 0
+    nb = mask.shape[-1]
+    for b in range(mask.shape[0]):
+        for h in range(mask.shape[1]):
+            for I in range(nb):
+                q0, q1 = I * block, min((I + 1) * block, N)
+                for J in range(nb):
+                    l = int(mask[b, h, I, J])
+                    if l == SKIP or (causal and J > I):
+                        continue
+                    k0, k1 = J * block, min((J + 1) * block, N)
+                    krows = (k1 - k0) >> l
+                    if causal and pairs_only and J == I:
+                        total += sum(1 for i in range(q0, q1) for j in range(k0, k1) if j <= i)
+                    else:
+                        total += (q1 - q0) * krows
+    return 4 * d * total
 
 
-def test_mask_roofline_meankey_reads_q_and_k_once():
-    w = W.PRESETS["wan14b"].replace(mask_mode="meankey")
-    r = bench.mask_roofline(w, mask_ms=2.0, hbm=6541.5, clocks=None, elem=2)
-    byts = (40 + 40) * 75600 * 128 * 2
-    assert r["bound"] == "hbm" and math.isclose(r["achieved"], byts / 2e-3 / 1e9)
-    assert bench.mask_roofline(W.PRESETS["tiny"], 1.0, 6541.5, None, 4) is None
-
-
-def test_launch_counts_per_scorer():
-    assert bench.MASK_KERNELS == {"sample": 2, "antidiag": 2, "meankey": 5, "given": 0}
+@pytest.mark.parametrize("causal", [False, True])
+def test_executed_flops_brute_force(causal):
+    g = torch.Generator().manual_seed(3)
+    N, block, d, L, nb = 300, 64, 16, 3, 5
+    m = torch.randint(0, L + 1, (2, 2, nb, nb), generator=g)
+    mask = torch.where(m == L, torch.full_like(m, SKIP), m).to(torch.uint8)
+    if causal:
+        idx = torch.arange(nb)
+        mask[:, :, idx, idx] = 0
+    got = B.executed_flops(mask, N, block, d, L, causal)
+    assert got == brute(mask.numpy(), N, block, d, causal, False)
+    if causal:
+        fa = got - B.diagonal_excess_flops(mask, N, block, d)
+        assert fa == brute(mask.numpy(), N, block, d, True, True)
