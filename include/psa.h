@@ -57,7 +57,7 @@ extern "C" {
 
 typedef enum {
   PSA_OK = 0,
-  PSA_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad enum, misaligned pointer */
+  PSA_ERR_INVALID_ARG = 1,   /* null pointer, size <= 0 (empty inputs included), bad enum, misaligned pointer */
   PSA_ERR_UNSUPPORTED = 2,   /* outside the supported set above */
   PSA_ERR_WORKSPACE = 3,     /* workspace null or smaller than the query says */
   PSA_ERR_CUDA = 4,          /* a CUDA runtime/driver call or a launch failed */

@@ -81,6 +81,9 @@ def _attn(shape, q=FAKE, k=FAKE, v=FAKE, kp=FAKE, vp=FAKE, mask=FAKE, scale=0.1,
     ("Hkv", 3, P.PSA_ERR_UNSUPPORTED),       # 4 % 3 != 0
     ("dtype", 7, P.PSA_ERR_INVALID_ARG),
     ("B", -1, P.PSA_ERR_INVALID_ARG),
+    ("B", 0, P.PSA_ERR_INVALID_ARG),         # empty inputs are rejected, nothing is written
+    ("Hq", 0, P.PSA_ERR_INVALID_ARG),
+    ("N", 0, P.PSA_ERR_INVALID_ARG),
 ])
 def test_attention_rejects_bad_shape(field, value, code):
     s = P.make_shape(1, 4, 2, 1000 if field != "N" else 1000, 64, 64, 4)
