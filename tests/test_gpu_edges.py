@@ -1,7 +1,8 @@
 """GPU edge cases of the PSA path (through the C ABI), each against the oracle.
 
   * More than 1024 KV blocks: the mask generator's CTA-wide select kernel
-    (the warp kernel holds at most 1024 keys per row), with both level
+    (the one-warp-per-row bucketed select takes at most 1024 keys per
+    row), with both level
     policies and causal masking, and attention on the resulting mask.
   * Determinism of the mask (select kernel atomics) and of the FP8
     probability-and-value attention: repeated calls are bit-equal.
@@ -32,7 +33,7 @@ TRAP_SITE = 10          # the attention kernel's debug trap wait
 @pytest.mark.parametrize("policy,causal", [("mass", False), ("quantile", True)])
 def test_select_over_1024_key_blocks(policy, causal):
     """N = 70,000 tokens in blocks of 64: 1094 KV blocks (the last holds 48
-    tokens), beyond the warp select kernel's 1024."""
+    tokens), beyond the one-warp-per-row select kernel's 1024."""
     N, d, block = 70000, 64, 64
     th = (0.6, 0.8, 0.9, 0.95) if policy == "mass" else (0.25, 0.5, 0.75, 0.875)
     w = W.Workload("nkb1094", B=1, Hq=2, Hkv=1, d=d, block=block, levels=4, causal=causal, dtype="bf16",
