@@ -173,28 +173,31 @@ def test_fullsize_mask_variants_sampled(mode, policy):
     check_band("wan14b full size, %s/%s" % (mode, policy), n_amb, n_pairs)
 
 
-def test_fullsize_fp8_wan14b_sampled():
-    """The FP8 path at the Wan2.1-14B shape on the generated mask, checked
-    on sampled query-block rows against the oracle's attention on the same
-    e4m3 operands (the GPU's quantizer codes are pinned bit for bit in
-    test_gpu_fp8.py; here the oracle quantizes the head itself)."""
-    w = W.PRESETS["wan14b"]
+@pytest.mark.parametrize("name", ["wan14b", "qwen2.5vl", "wan1.3b"])
+def test_fullsize_fp8_sampled(name):
+    """The FP8 path (e4m3 Q and K) at the preset's full shape on its
+    generated mask, checked on sampled query-block rows against the
+    oracle's attention on the same e4m3 operands (the GPU's quantizer codes
+    are pinned bit for bit in test_gpu_fp8.py; here the oracle quantizes
+    the whole KV head itself), at the bf16 tolerances."""
+    w = W.PRESETS[name]
     q, k, v, _ = W.make_qkv(w, device=DEV)
     shape = shape_for(w)
-    kp, vp, _ = run_pyramid(shape, k, v)
-    mask, _ = run_mask(shape, params_for(w), q, k)
+    kp, vp, bc = run_pyramid(shape, k, v, with_cos=w.cos_min > -2)
+    mask, _ = run_mask(shape, params_for(w), q, k, bc)
     out = torch.empty_like(q)
     ws = P.workspace(P.psa_attention_fp8_workspace_bytes(shape), DEV)
     P.psa_attention_fwd_fp8(shape, q, k, v, kp, vp, mask, w.sm_scale, out, None, ws)
     torch.cuda.synchronize()
     assert P.psa_get_device_status(ws) == P.PSA_OK
+    grp = w.Hq // w.Hkv
     rows = sample_rows(w, 10, seed=5)
     for (b, h), Is in by_head(rows).items():
         hrows = [(0, 0, I) for I in Is]
-        kl = head_levels(shape, k, kp, b, h, w.levels)
-        vl = head_levels(shape, v, vp, b, h, w.levels)
+        kl = head_levels(shape, k, kp, b, h // grp, w.levels)
+        vl = head_levels(shape, v, vp, b, h // grp, w.levels)
         o, _ = O.attention_fp8(q[b:b + 1, h:h + 1].cpu(), [x.astype(np.float32) for x in kl], vl,
-                               mask[b:b + 1, h:h + 1].cpu(), w.block, w.sm_scale, False, rows=hrows)
+                               mask[b:b + 1, h:h + 1].cpu(), w.block, w.sm_scale, w.causal, rows=hrows)
         mx, mean, _ = attn_errors(out[b:b + 1, h:h + 1], o)
         assert mx <= 2e-2 and mean <= 2e-3, (h, Is, mx, mean)
 
