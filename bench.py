@@ -580,12 +580,20 @@ def measure_fp8(path, w, stream, flops_fwd, peaks_, reps=5):
         return {"ms": ms, "tflops": tf, "frac_of_burst_bf16": tf / peaks_[0], "clocks": cs.summary(),
                 "vs_bf16_path": {"max_abs": diff.max().item(), "mean_abs": diff.mean().item()}}
 
+    # peaks of the path's own MMA types: e4m3 at the nominal 2x of the measured
+    # bf16 burst rate; with only S on e4m3, half the FLOPs at each rate
+    fp8_peak = 2.0 * peaks_[0]
+    mixed_peak = 1.0 / (0.5 / fp8_peak + 0.5 / peaks_[0])
     r = {"entry_point": "psa_attention_fwd_fp8", "reps": reps,
          "includes": "e4m3 quantization of Q and every K level, plan, attention"}
     r.update(timed(P.psa_attention_fwd_fp8))
+    r["peak_own_dtype"] = {"tflops": mixed_peak, "kind": "S on e4m3 (2x the measured bf16 burst, nominal ratio), "
+                           "P.V on bf16: half the FLOPs at each rate", "frac": r["tflops"] / mixed_peak}
     pv = {"entry_point": "psa_attention_fwd_fp8_pv",
           "includes": "e4m3 quantization of Q and of every K and V level, plan, attention with e4m3 P"}
     pv.update(timed(P.psa_attention_fwd_fp8_pv))
+    pv["peak_own_dtype"] = {"tflops": fp8_peak, "kind": "e4m3: 2x the measured bf16 burst (nominal ratio)",
+                            "frac": pv["tflops"] / fp8_peak}
     r["pv"] = pv
     del ws, out8
     torch.cuda.empty_cache()
