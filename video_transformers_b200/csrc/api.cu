@@ -212,7 +212,7 @@ MaskLayout mask_layout(const psa_shape_t* s, const psa_mask_params_t* p) {
   size_t off = 256;
   L.status = 0;
   L.blocklse = off; off = align_up(off + BHq * nkb * L.rows * 4, 256);
-  L.rowlse = off;   off = align_up(off + 2 * BHq * L.rows * 4, 256);   // one partial per epilogue warpgroup
+  L.rowlse = off;   off = align_up(off + psa::kScore2Parts * BHq * L.rows * 4, 256);   // row-LSE partials
   if (p->mode == PSA_MASK_MEANKEY) {
     // block means in fp64; the mean-key scorer reads the inputs directly
     L.qmean = off; off = align_up(off + BHq * nqb * s->d * 8, 256);
@@ -545,6 +545,9 @@ psa_status_t psa_make_mask(const psa_shape_t* s, const psa_mask_params_t* p, con
   se.mass_out = mass_out;
   se.blocklse = reinterpret_cast<float*>(w + L.blocklse);
   se.rowlse = reinterpret_cast<float*>(w + L.rowlse);
+  // partials per row: one per column part of the paired sampling score,
+  // else two (the one-row-tile score's warpgroups; the mean-key scorer)
+  se.n_part = (p->mode == PSA_MASK_SAMPLE && s->d == 128) ? psa::kScore2Parts : 2;
   if (p->mode == PSA_MASK_MEANKEY) {
     const int es = static_cast<int>(elem_size(s->dtype));
     double* qm = reinterpret_cast<double*>(w + L.qmean);

@@ -40,6 +40,10 @@ cudaError_t launch_blockcos(const void* k, float* out, int64_t BH, int N, int d,
 cudaError_t launch_cast_bf16(const float* src, void* dst, int64_t n, cudaStream_t s);
 
 // ---- stage 2 -------------------------------------------------------------
+// column parts of the paired sampling score (score2_kernel): a work item is
+// (head, row-tile pair, part), and part e writes row-LSE partial e
+constexpr int kScore2Parts = 4;
+
 struct ScoreArgs {
   int BHq, Hq, Hkv, N, d, block, nkb;
   int mode;            // 0 sampling, 1 antidiagonal
@@ -52,7 +56,8 @@ struct ScoreArgs {
   int causal;
   float scale_log2;    // softmax scale * log2(e)
   float* blocklse;     // [BHq][nkb][rows]  log2-domain logsumexp of each block
-  float* rowlse;       // [2][BHq][rows]  partial row LSEs of the two epilogue warpgroups
+  float* rowlse;       // [n_part][BHq][rows]  partial row LSEs (score_kernel: 2, one per epilogue
+                       // warpgroup; score2_kernel: kScore2Parts, one per column part)
   int* status;
 };
 cudaError_t launch_score(const CUtensorMap* mapA, const CUtensorMap* mapB, const ScoreArgs& a,
@@ -81,7 +86,8 @@ struct SelectArgs {
   float cos_min;
   int n_dense_prefix;
   const float* blocklse;
-  const float* rowlse;      // [2][B*Hq][rows]
+  const float* rowlse;      // [n_part][B*Hq][rows]
+  int n_part;               // row-LSE partials to combine per row
   const float* blockcos;
   uint8_t* mask;
   float* mass_out;

@@ -14,7 +14,8 @@
 //                d = 64.
 // score2_kernel  the sampling score at d = 128: two row tiles share every K
 //                tile, epilogue warpgroup x owns row tile x, and a work item
-//                covers half of the column tiles (row-LSE partial = half).
+//                covers a quarter of the column tiles (one row-LSE partial
+//                per quarter).
 // select_bucket_kernel  one warp per (b, h, query block), up to 1024 key
 //                blocks: the same levels as select_kernel without a sort --
 //                a histogram of the masses in 256 buckets and its scan give
@@ -327,9 +328,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 // score2_kernel: the sampling score with two row tiles per work item, so
 // every K tile brought into shared memory serves 256 sampled rows instead of
 // 128 (half the K traffic per flop).  A work item is (head, row-tile pair,
-// half of the column tiles); the two sampled-query tiles stay resident;
-// TMEM holds two S buffers per row tile (512 columns); epilogue warpgroup x
-// owns row tile x and writes row-LSE partial e for column half e.  Used for
+// part e of kScore2Parts of the column tiles); the two sampled-query tiles
+// stay resident; TMEM holds two S buffers per row tile (512 columns);
+// epilogue warpgroup x owns row tile x and writes row-LSE partial e.  Used for
 // d = 128, where it halves the K traffic that bounds the one-row-tile
 // kernel; at d = 64 (half the MMA work per tile) it measured slower.
 // ----------------------------------------------------------------------------
@@ -357,10 +358,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int row_tiles = (a.rows + 127) / 128;
   const int pairs = (row_tiles + 1) / 2;
   const int col_tiles = (a.cols + 127) / 128;
-  // item = (bh, row-tile pair, column half): the two halves of a pair's
-  // column sweep are separate items (finer work for the persistent grid);
-  // half e writes row-LSE partial e
-  const int n_items = a.BHq * pairs * 2;
+  // item = (bh, row-tile pair, column part): the parts of a pair's column
+  // sweep are separate items (finer work, a shorter last wave of the
+  // persistent grid); part e writes row-LSE partial e
+  const int n_items = a.BHq * pairs * kScore2Parts;
   const int nk = a.d / 64;                 // 64-channel chunks per tile
   const int nst = kRegion2 - 2 * nk;       // K ring stages (8 for d = 128, 10 for d = 64)
 
@@ -388,11 +389,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int rlast = min((2 * p + n_rt(p)) * 128 - 1, a.rows - 1);
     return min(col_tiles, rlast * a.step / 128 + 1);
   };
-  // column tiles [lo, hi) of item half e
+  // column tiles [lo, hi) of item part e (possibly empty for short causal rows)
   auto range_of = [&](int p, int e, int& lo, int& hi) {
-    const int nct = tiles_for(p), h = (nct + 1) / 2;
-    lo = e == 0 ? 0 : h;
-    hi = e == 0 ? h : nct;
+    const int nct = tiles_for(p);
+    lo = nct * e / kScore2Parts;
+    hi = nct * (e + 1) / kScore2Parts;
   };
 
   if (warp == 0) {
@@ -403,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t it = 0, icnt = 0;
       bool ok = true;
       for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-        const int e = item & 1, bh = (item >> 1) / pairs, p = (item >> 1) - bh * pairs;
+        const int e = item % kScore2Parts, bh = (item / kScore2Parts) / pairs, p = item / kScore2Parts - bh * pairs;
         const int hkv = kv_head_of(bh, a.Hq, a.Hkv);
         const int nrt = n_rt(p);
         int lo, hi;
@@ -438,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t it = 0, t = 0, icnt = 0;
       bool ok = true;
       for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-        const int e = item & 1, bh = (item >> 1) / pairs, p = (item >> 1) - bh * pairs;
+        const int e = item % kScore2Parts, bh = (item / kScore2Parts) / pairs, p = item / kScore2Parts - bh * pairs;
         (void)bh;
         const int nrt = n_rt(p);
         int lo, hi;
@@ -481,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t t = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-      const int e = item & 1, bh = (item >> 1) / pairs, p = (item >> 1) - bh * pairs;
+      const int e = item % kScore2Parts, bh = (item / kScore2Parts) / pairs, p = item / kScore2Parts - bh * pairs;
       const bool mine = x < n_rt(p);
       const int nct = tiles_for(p);
       int lo, hi;
@@ -489,8 +490,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int r = (2 * p + x) * 128 + lrow;
       const int pos = r * a.step;
       const int climit = a.causal ? min(a.cols, pos + 1) : a.cols;
-      // this half's running LSE: row-LSE partial e (the select kernel
-      // combines the two in fp64)
+      // this part's running LSE: row-LSE partial e (the select kernel
+      // combines the partials in fp64)
       float M = -CUDART_INF_F, Ssum = 0.f;
       float* bl = a.blocklse + static_cast<int64_t>(bh) * a.nkb * a.rows + r;
       for (int ct = lo; ct < hi; ++ct, ++t) {
@@ -540,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       if (mine && r < a.rows) {
         // column tiles never visited (causal) hold no probability
-        if (e == 1)
+        if (e == kScore2Parts - 1)
           for (int J = nct * BPT; J < a.nkb; ++J) bl[static_cast<int64_t>(J) * a.rows] = -CUDART_INF_F;
         a.rowlse[(static_cast<int64_t>(e) * a.BHq + bh) * a.rows + r] =
             M == -CUDART_INF_F ? -CUDART_INF_F : M + __log2f(Ssum);
@@ -555,6 +556,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     tmem_dealloc(tmem, 512);
   }
+}
+
+// a score row's log2-domain LSE from its n_part partials, in fp64
+__device__ __forceinline__ double combine_partials(const SelectArgs& a, int bh, int r) {
+  const int64_t plane = static_cast<int64_t>(a.B) * a.Hq * a.rows;
+  const float* p = a.rowlse + static_cast<int64_t>(bh) * a.rows + r;
+  double mx = -CUDART_INF;
+  for (int e = 0; e < a.n_part; ++e) mx = fmax(mx, static_cast<double>(p[e * plane]));
+  if (mx == -CUDART_INF) return mx;
+  double sum = 0.0;
+  for (int e = 0; e < a.n_part; ++e) sum += exp2(static_cast<double>(p[e * plane]) - mx);
+  return mx + log2(sum);
 }
 
 // ----------------------------------------------------------------------------
@@ -586,10 +599,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectArgs a)
   // LSE of the column tiles they handled; combine them (log2 domain)
   __shared__ double rlse[128];
   for (int s = threadIdx.x; s < nvalid; s += blockDim.x) {
-    const double x = a.rowlse[static_cast<int64_t>(bh) * a.rows + rbeg + s];
-    const double y = a.rowlse[(static_cast<int64_t>(a.B) * a.Hq + bh) * a.rows + rbeg + s];
-    const double mx = fmax(x, y);
-    rlse[s] = mx == -CUDART_INF ? mx : mx + log2(exp2(x - mx) + exp2(y - mx));
+    rlse[s] = combine_partials(a, bh, rbeg + s);
   }
   __syncthreads();
 
@@ -765,10 +775,7 @@ __global__ void __launch_bounds__(32 * kBucketWarps) select_bucket_kernel(const 
     nvalid = min(a.rows_per_block, a.rows - rbeg);
   }
   for (int s = lane; s < nvalid; s += 32) {
-    const double x = a.rowlse[static_cast<int64_t>(bh) * a.rows + rbeg + s];
-    const double y = a.rowlse[(static_cast<int64_t>(a.B) * a.Hq + bh) * a.rows + rbeg + s];
-    const double mx = fmax(x, y);
-    rlse[s] = mx == -CUDART_INF ? mx : mx + log2(exp2(x - mx) + exp2(y - mx));
+    rlse[s] = combine_partials(a, bh, rbeg + s);
   }
   for (int i = lane; i < kBucketSlots; i += 32) {
     hs[i] = 0ull;
@@ -1022,7 +1029,7 @@ cudaError_t launch_score(const CUtensorMap* mapA, const CUtensorMap* mapB, const
   const int row_tiles = (a.rows + 127) / 128;
   if (a.mode == 0 && a.d == 128) {
     // sampling: two row tiles per item share each K tile
-    const int n2 = a.BHq * ((row_tiles + 1) / 2) * 2;
+    const int n2 = a.BHq * ((row_tiles + 1) / 2) * kScore2Parts;
     const int grid2 = n2 < num_sms ? n2 : num_sms;
     const size_t smem2 = 1024 + kRegion2 * kChunk + sizeof(Score2Shared);
     switch (a.cols_per_block) {
