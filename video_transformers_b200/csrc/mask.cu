@@ -721,11 +721,11 @@ __device__ __forceinline__ double exp2_split_exp(double x) {
   return static_cast<double>(p) * __longlong_as_double(static_cast<long long>(static_cast<int>(n) + 1023) << 52);
 }
 
-// per-warp shared memory of select_bucket_kernel for P = nkb rounded up to 32
+// per-warp shared memory of select_bucket_kernel (byte offsets), for
+// P = nkb rounded up to 32 and R = score rows per query block (<= 128)
 struct BucketLayout {
   int hs, tfx, rlse, mass, hc, lend, rth, list, ex, mixed, lv, bytes;
 };
-// P = nkb rounded up to 32, R = score rows per query block (<= 128)
 __host__ __device__ inline BucketLayout bucket_layout(int P, int R) {
   BucketLayout L{};
   int o = 0;
